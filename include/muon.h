@@ -1,0 +1,154 @@
+/*
+ * muon.h -- C ABI of the B200 (sm_100a) Muon optimizer step.
+ *
+ * What the library computes (Modded-NanoGPT news article, "Muon optimizer"
+ * section):
+ *   - the lessons paragraph: Nesterov momentum on the gradient, with the
+ *     orthogonalisation applied after the momentum, run in bf16;
+ *   - the zeroth_power_via_newtonschulz5 listing: X = G / (||G||_F + eps),
+ *     transpose when rows > cols, `ns_steps` quintic iterations
+ *     A = X X^T, B = b A + c A A, X = a X + B X with
+ *     (a, b, c) = (3.4445, -4.7750, 2.0315), transpose back;
+ *   - the update itself (the article's formula did not survive extraction;
+ *     the plainest reading is used): buf <- mu*buf + g, G = g + mu*buf,
+ *     W <- W - lr * NS5(G).
+ *
+ * Conventions shared by every entry point
+ *   - Matrices are fp32, row-major, contiguous; matrix i has shapes[2i] rows
+ *     and shapes[2i+1] columns.  Only 2-D matrices can be expressed.
+ *   - All pointers inside the pointer arrays are DEVICE pointers on the
+ *     current CUDA device, owned by the caller.  The pointer arrays and the
+ *     shapes array themselves are HOST memory, read during the call only.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous with respect to the host: results are ready once the
+ *     stream has reached this call.
+ *   - Argument errors are detected on the host, before anything is launched,
+ *     and returned synchronously.  Errors found by kernels (a bounded wait
+ *     that ran out) are recorded in a per-(device, stream) status word; they
+ *     are returned by the next call on that stream, by muon_sync_status(), and
+ *     described by muon_last_error().  Kernels never trap.
+ *   - The library keeps, per (device, stream), a workspace in device memory
+ *     (bf16 iterates, Gram and polynomial matrices, norms, TMA descriptors).
+ *     It is allocated by the first call that needs it (cudaMalloc, which is
+ *     not allowed during stream capture: make the first call for a given set
+ *     of shapes outside capture) and freed by muon_release().
+ *   - Concurrent calls on different streams use different workspaces; calls
+ *     on one stream are serialised by the stream.
+ *   - NaN / Inf in the inputs propagate to the outputs; nothing checks them.
+ */
+#ifndef MUON_B200_H
+#define MUON_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MUON_OK = 0,
+  MUON_ERR_INVALID_ARG = -1,  /* null pointer, n <= 0, ns_steps < 0, bad flag  */
+  MUON_ERR_SHAPE = -2,        /* a dimension <= 0 or too large for int32 math  */
+  MUON_ERR_CUDA = -3,         /* a CUDA runtime / driver call failed           */
+  MUON_ERR_NOMEM = -4,        /* workspace allocation failed                   */
+  MUON_ERR_TIMEOUT = -5,      /* a kernel gave up on a bounded wait            */
+  MUON_ERR_DEVICE = -6,       /* no usable sm_100 device                       */
+  MUON_ERR_UNSUPPORTED = -7   /* configuration this build does not handle      */
+} muon_status;
+
+/* Default quintic coefficients, step count and eps of the NS5 listing. */
+#define MUON_NS_A 3.4445f
+#define MUON_NS_B (-4.7750f)
+#define MUON_NS_C 2.0315f
+#define MUON_NS_STEPS 5
+#define MUON_NS_EPS 1e-7f
+
+/*
+ * One Muon step over n independent weight matrices (Nesterov momentum,
+ * NS5 with the listing's defaults, W -= lr*O).
+ *   params[i]        in/out  W_i, updated in place.
+ *   grads[i]         in      g_i, read only.
+ *   momentum_bufs[i] in/out  buf_i (fp32 state), updated in place to
+ *                            mu*buf_i + g_i.
+ *   shapes           in      2n int64: rows_i, cols_i.
+ *   ns_steps         >= 0    quintic iterations (5 in the listing; 0 gives
+ *                            O = G/(||G||_F + eps) rounded to bf16).
+ * Returns MUON_OK or a muon_status error code.
+ */
+int muon_step(float* const* params, const float* const* grads, float* const* momentum_bufs,
+              const int64_t* shapes, int n, float lr, float mu, int ns_steps, void* stream);
+
+/*
+ * muon_step with every constant of the method exposed: quintic coefficients
+ * (a, b, c), eps added to the Frobenius norm, and nesterov (1: G = g + mu*buf
+ * after the buffer update, as in the lessons paragraph; 0: G = buf).
+ */
+int muon_step_ex(float* const* params, const float* const* grads, float* const* momentum_bufs,
+                 const int64_t* shapes, int n, float lr, float mu, int ns_steps,
+                 float a, float b, float c, float eps, int nesterov, void* stream);
+
+/*
+ * NS5 alone (the zeroth_power_via_newtonschulz5 listing): O_i = NS5(G_i)
+ * with the listing's defaults and `ns_steps` iterations.  G_i is read only,
+ * O_i (m x n fp32, caller-owned device memory) is overwritten.
+ */
+int muon_orthogonalize(const float* const* G, float* const* O, const int64_t* shapes, int n,
+                       int ns_steps, void* stream);
+
+/*
+ * muon_step on HOST buffers: params, grads and momentum_bufs point to host
+ * memory (pinned memory gives full PCIe bandwidth; pageable works).  The
+ * library copies the inputs to device staging buffers, runs the step and
+ * copies W and buf back, all on `stream`, and returns after the stream has
+ * finished (the host buffers hold the results on return).
+ */
+int muon_step_host(float* const* params, const float* const* grads, float* const* momentum_bufs,
+                   const int64_t* shapes, int n, float lr, float mu, int ns_steps, void* stream);
+
+/* Bytes of device workspace a call with these shapes uses (0 on bad input). */
+size_t muon_workspace_size(const int64_t* shapes, int n);
+
+/* Waits for `stream`, then returns and clears the status its kernels recorded
+ * (MUON_OK, MUON_ERR_TIMEOUT, ...). */
+int muon_sync_status(void* stream);
+
+/* Human-readable description of the last error seen by this thread. */
+const char* muon_last_error(void);
+
+/* Frees every cached workspace and staging buffer on every device. */
+void muon_release(void);
+
+/* ---- measurement hooks (used by the benchmark; off by default) ---------- */
+
+/* Kernel kinds reported by the profiling hooks. */
+#define MUON_KIND_PROLOGUE 0
+#define MUON_KIND_GRAM 1
+#define MUON_KIND_POLY 2
+#define MUON_KIND_UPDATE 3
+#define MUON_KIND_UPDATE_APPLY 4
+#define MUON_KIND_APPLY_X0 5
+#define MUON_NUM_KINDS 6
+
+/* 1: bracket every kernel launch with CUDA events on its stream; 0: stop. */
+int muon_profile_enable(int enable);
+/* Synchronises the recorded events and adds, per kind, the summed device
+ * milliseconds and the launch count into ms[kind] / launches[kind]
+ * (arrays of nkinds entries); then forgets them. */
+int muon_profile_read(double* ms, int64_t* launches, int nkinds);
+/* Number of kernels this library has launched since it was loaded. */
+int64_t muon_launch_count(void);
+
+/* ---- test hooks -------------------------------------------------------- */
+
+/* wait_limit_ns: bound of every device-side wait (0 keeps the default, 2 s).
+ * flags bit 0: the next GEMM launch skips filling its first pipeline stage,
+ * so its MMA warp's wait runs out and the call reports MUON_ERR_TIMEOUT
+ * (fault injection that neither faults nor hangs the GPU). */
+int muon_debug_set(int flags, int64_t wait_limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_B200_H */

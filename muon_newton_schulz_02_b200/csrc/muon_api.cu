@@ -1,0 +1,684 @@
+// Host side of the C ABI declared in include/muon.h.
+//
+// A call is planned once per set of shapes: matrices are grouped into shape
+// classes (same padded short side kp and long side lp), each class gets
+// contiguous [batch][kp][lp] bf16 iterates and [batch][kp][kp] Gram /
+// polynomial buffers in the workspace, and one TMA descriptor per buffer and
+// box shape.  A step is then 1 + 3*ns_steps kernel launches on the caller's
+// stream: the fused momentum/norm/cast prologue, then per NS iteration one
+// persistent tcgen05 GEMM launch per phase over all matrices of the group.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <list>
+#include <map>
+#include <memory>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "muon.h"
+#include "kernels.cuh"
+
+using namespace muon;
+
+namespace {
+
+thread_local std::string g_last_error = "no error";
+std::mutex g_mu;
+std::atomic<int64_t> g_launches{0};
+bool g_profile = false;
+int g_debug_flags = 0;
+uint64_t g_wait_limit_ns = 2000000000ull;
+
+int fail(int code, const std::string& msg) {
+  g_last_error = msg;
+  return code;
+}
+
+#define CUDA_TRY(expr)                                                                        \
+  do {                                                                                        \
+    cudaError_t e_ = (expr);                                                                  \
+    if (e_ != cudaSuccess) return fail(MUON_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int round_up(int v, int a) { return (v + a - 1) / a * a; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// ------------------------------------------------------------------ plan ---
+struct MatDesc {
+  int m, n, k, l, kp, lp, trans;
+  int user;                 // index in the caller's arrays
+};
+
+struct ClassDesc {
+  int kp, lp;
+  std::vector<int> mats;    // group-order indices
+  size_t off_x0, off_x1, off_a, off_b;
+};
+
+struct Group {
+  std::vector<MatDesc> mats;     // group order (class by class)
+  std::vector<ClassDesc> classes;
+  std::vector<int> pro_tile_begin;
+  int pro_tiles = 0;
+  size_t off_partials = 0, off_tickets = 0, off_scale = 0, off_tmaps = 0;
+  size_t data_bytes = 0;
+  int sym_tiles = 0, upd_tiles = 0;
+  std::vector<GemmClass> sym_cls, upd_cls;
+};
+
+// The first kTicketBytes of every workspace hold the per-matrix arrival
+// counters of the prologue's norm reduction.  They are zeroed when the
+// workspace is allocated and every prologue leaves them at zero again, so no
+// plan may place anything else there.
+constexpr size_t kTicketBytes = 4096;
+static_assert(kMaxMats * 4 <= kTicketBytes, "ticket region too small");
+
+struct Plan {
+  std::vector<int64_t> shapes;
+  std::vector<Group> groups;
+  size_t ws_bytes = 0;
+  size_t tmap_bytes = 0;
+  void* ws = nullptr;                       // workspace the tensor maps point into
+  void* tmaps = nullptr;                    // this plan's own device copy of its tensor maps
+  ~Plan() {
+    if (tmaps) cudaFree(tmaps);
+  }
+};
+
+// Splits the matrices into groups (each within the per-launch limits) and lays
+// out each group's workspace; groups run one after another and share the
+// data region, each keeps its own tensor-map table at the end.
+int build_layout(const int64_t* shapes, int n, Plan& plan) {
+  plan.shapes.assign(shapes, shapes + 2 * (size_t)n);
+  std::vector<MatDesc> all(n);
+  for (int i = 0; i < n; ++i) {
+    const int64_t m = shapes[2 * i], c = shapes[2 * i + 1];
+    if (m <= 0 || c <= 0) return fail(MUON_ERR_SHAPE, "matrix " + std::to_string(i) + " has a dimension <= 0");
+    if (m > (1 << 20) || c > (1 << 20) || m * c > (int64_t(1) << 31))
+      return fail(MUON_ERR_SHAPE, "matrix " + std::to_string(i) + " is too large (dims <= 2^20, elements <= 2^31)");
+    MatDesc d;
+    d.m = (int)m; d.n = (int)c;
+    d.trans = m > c ? 1 : 0;
+    d.k = (int)std::min(m, c); d.l = (int)std::max(m, c);
+    d.kp = round_up(d.k, kPad); d.lp = round_up(d.l, kPad);
+    if (d.kp > 16384) return fail(MUON_ERR_SHAPE, "short side above 16384 is not supported");
+    d.user = i;
+    all[i] = d;
+  }
+  // greedy grouping in caller order, respecting kMaxMats and kMaxClasses
+  std::vector<std::vector<MatDesc>> raw;
+  {
+    std::vector<MatDesc> cur;
+    std::vector<std::pair<int, int>> keys;
+    for (const auto& d : all) {
+      const std::pair<int, int> key(d.kp, d.lp);
+      const bool new_key = std::find(keys.begin(), keys.end(), key) == keys.end();
+      if ((int)cur.size() == kMaxMats || (new_key && (int)keys.size() == kMaxClasses)) {
+        raw.push_back(cur); cur.clear(); keys.clear();
+      }
+      if (std::find(keys.begin(), keys.end(), key) == keys.end()) keys.push_back(key);
+      cur.push_back(d);
+    }
+    if (!cur.empty()) raw.push_back(cur);
+  }
+  size_t data_max = 0;
+  for (auto& gm : raw) {
+    Group g;
+    g.off_tickets = 0;          // fixed region, see kTicketBytes
+    // classes ordered by decreasing long side (longest GEMM K first)
+    std::map<std::pair<int, int>, std::vector<MatDesc>> by;
+    for (const auto& d : gm) by[{-d.lp, -d.kp}].push_back(d);
+    size_t off = kTicketBytes;
+    for (auto& kv : by) {
+      ClassDesc c;
+      c.kp = -kv.first.second; c.lp = -kv.first.first;
+      const size_t batch = kv.second.size();
+      const size_t xb = batch * (size_t)c.kp * c.lp * 2, ab = batch * (size_t)c.kp * c.kp * 2;
+      c.off_x0 = off; off = align_up(off + xb, 1024);
+      c.off_x1 = off; off = align_up(off + xb, 1024);
+      c.off_a = off; off = align_up(off + ab, 1024);
+      c.off_b = off; off = align_up(off + ab, 1024);
+      for (auto& d : kv.second) { c.mats.push_back((int)g.mats.size()); g.mats.push_back(d); }
+      g.classes.push_back(c);
+    }
+    for (const auto& d : g.mats) {
+      g.pro_tile_begin.push_back(g.pro_tiles);
+      g.pro_tiles += (d.kp / kProRows) * (d.lp / kProCols);
+    }
+    g.off_partials = off; off = align_up(off + (size_t)g.pro_tiles * 4, 1024);
+    g.off_scale = off; off = align_up(off + g.mats.size() * 4, 1024);
+    g.data_bytes = off;
+    data_max = std::max(data_max, off);
+    // GEMM tile bookkeeping
+    int sym = 0, upd = 0, first = 0;
+    for (size_t ci = 0; ci < g.classes.size(); ++ci) {
+      const ClassDesc& c = g.classes[ci];
+      GemmClass s{}, u{};
+      s.batch = u.batch = (int)c.mats.size();
+      s.kp = u.kp = c.kp; s.lp = u.lp = c.lp;
+      s.mat_first = u.mat_first = first;
+      s.tiles_m = u.tiles_m = c.kp / kBM;
+      s.tiles_n = s.tiles_m;
+      u.tiles_n = c.lp / kBN;
+      s.tiles_per_mat = s.tiles_m * (s.tiles_m + 1) / 2;
+      u.tiles_per_mat = u.tiles_m * u.tiles_n;
+      s.tile_begin = sym; u.tile_begin = upd;
+      sym += s.tiles_per_mat * s.batch;
+      upd += u.tiles_per_mat * u.batch;
+      s.kblocks = c.lp / kBK;   // GRAM; POLY overrides with kp / 64
+      u.kblocks = c.kp / kBK;
+      s.tmap_base = u.tmap_base = (int)ci * kTmapsPerClass;
+      first += (int)c.mats.size();
+      g.sym_cls.push_back(s);
+      g.upd_cls.push_back(u);
+    }
+    g.sym_tiles = sym; g.upd_tiles = upd;
+    plan.groups.push_back(std::move(g));
+  }
+  size_t off = 0;
+  for (auto& g : plan.groups) {
+    g.off_tmaps = off;
+    off = align_up(off + g.classes.size() * kTmapsPerClass * sizeof(CUtensorMap), 1024);
+  }
+  plan.tmap_bytes = off;
+  plan.ws_bytes = data_max;
+  return MUON_OK;
+}
+
+int encode_map(CUtensorMap* map, void* base, int cols, int rows, int batch, int box_cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * rows * 2};
+  cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return MUON_OK;
+}
+
+// ---------------------------------------------------------------- context ---
+struct ProfRec { int kind; cudaEvent_t a, b; };
+
+struct Ctx {
+  int dev = 0;
+  cudaStream_t stream = nullptr;
+  void* ws = nullptr;
+  size_t ws_cap = 0;
+  std::list<std::unique_ptr<Plan>> plans;   // most recent first
+  int* status_h = nullptr;
+  int* status_d = nullptr;
+  float* stage = nullptr;                   // device staging of muon_step_host
+  size_t stage_cap = 0;
+  std::vector<ProfRec> prof;
+  std::vector<cudaEvent_t> event_pool;
+  int sm_count = 148;
+};
+
+std::map<std::pair<int, void*>, std::unique_ptr<Ctx>> g_ctx;
+std::map<int, bool> g_dev_ready;
+
+int device_setup(int dev) {
+  if (g_dev_ready[dev]) return MUON_OK;
+  cudaDeviceProp prop;
+  CUDA_TRY(cudaGetDeviceProperties(&prop, dev));
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(MUON_ERR_DEVICE, "this library is built for sm_100a (B200); device is sm_" +
+                                     std::to_string(prop.major) + std::to_string(prop.minor));
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+  g_dev_ready[dev] = true;
+  return MUON_OK;
+}
+
+int get_ctx(void* stream, Ctx** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  int rc = device_setup(dev);
+  if (rc) return rc;
+  auto key = std::make_pair(dev, stream);
+  auto it = g_ctx.find(key);
+  if (it == g_ctx.end()) {
+    auto c = std::make_unique<Ctx>();
+    c->dev = dev;
+    c->stream = (cudaStream_t)stream;
+    CUDA_TRY(cudaHostAlloc((void**)&c->status_h, sizeof(int), cudaHostAllocMapped));
+    *c->status_h = 0;
+    CUDA_TRY(cudaHostGetDevicePointer((void**)&c->status_d, c->status_h, 0));
+    CUDA_TRY(cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, dev));
+    it = g_ctx.emplace(key, std::move(c)).first;
+  }
+  *out = it->second.get();
+  return MUON_OK;
+}
+
+int ensure_workspace(Ctx& c, size_t bytes) {
+  if (c.ws_cap >= bytes) return MUON_OK;
+  CUDA_TRY(cudaStreamSynchronize(c.stream));
+  if (c.ws) { cudaFree(c.ws); c.ws = nullptr; c.ws_cap = 0; }
+  c.plans.clear();                                     // their tensor maps point into the old workspace
+  const size_t cap = align_up(bytes, size_t(1) << 21);
+  if (cudaMalloc(&c.ws, cap) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MUON_ERR_NOMEM, "workspace allocation of " + std::to_string(cap) + " bytes failed");
+  }
+  c.ws_cap = cap;
+  CUDA_TRY(cudaMemset(c.ws, 0, cap));                  // tickets start at zero
+  return MUON_OK;
+}
+
+int get_plan(Ctx& c, const int64_t* shapes, int n, Plan** out) {
+  for (auto it = c.plans.begin(); it != c.plans.end(); ++it) {
+    Plan& p = **it;
+    if ((int)p.shapes.size() == 2 * n && std::memcmp(p.shapes.data(), shapes, sizeof(int64_t) * 2 * n) == 0 &&
+        p.ws == c.ws) {
+      c.plans.splice(c.plans.begin(), c.plans, it);
+      *out = c.plans.front().get();
+      return MUON_OK;
+    }
+  }
+  auto p = std::make_unique<Plan>();
+  int rc = build_layout(shapes, n, *p);
+  if (rc) return rc;
+  rc = ensure_workspace(c, p->ws_bytes);
+  if (rc) return rc;
+  p->ws = c.ws;
+  char* base = (char*)c.ws;
+  if (cudaMalloc(&p->tmaps, p->tmap_bytes) != cudaSuccess) {
+    cudaGetLastError();
+    p->tmaps = nullptr;
+    return fail(MUON_ERR_NOMEM, "tensor-map table allocation failed");
+  }
+  for (auto& g : p->groups) {
+    std::vector<CUtensorMap> maps(g.classes.size() * kTmapsPerClass);
+    for (size_t ci = 0; ci < g.classes.size(); ++ci) {
+      const ClassDesc& cd = g.classes[ci];
+      const int batch = (int)cd.mats.size();
+      CUtensorMap* m = &maps[ci * kTmapsPerClass];
+      if ((rc = encode_map(&m[kTmX0], base + cd.off_x0, cd.lp, cd.kp, batch, 64, 128))) return rc;
+      if ((rc = encode_map(&m[kTmX1], base + cd.off_x1, cd.lp, cd.kp, batch, 64, 128))) return rc;
+      if ((rc = encode_map(&m[kTmX0mn], base + cd.off_x0, cd.lp, cd.kp, batch, 64, 64))) return rc;
+      if ((rc = encode_map(&m[kTmX1mn], base + cd.off_x1, cd.lp, cd.kp, batch, 64, 64))) return rc;
+      if ((rc = encode_map(&m[kTmA], base + cd.off_a, cd.kp, cd.kp, batch, 64, 128))) return rc;
+      if ((rc = encode_map(&m[kTmB], base + cd.off_b, cd.kp, cd.kp, batch, 64, 128))) return rc;
+    }
+    CUDA_TRY(cudaMemcpy((char*)p->tmaps + g.off_tmaps, maps.data(), maps.size() * sizeof(CUtensorMap),
+                        cudaMemcpyHostToDevice));
+  }
+  c.plans.push_front(std::move(p));
+  if (c.plans.size() > 4) {
+    CUDA_TRY(cudaStreamSynchronize(c.stream));
+    while (c.plans.size() > 4) c.plans.pop_back();
+  }
+  *out = c.plans.front().get();
+  return MUON_OK;
+}
+
+// ---------------------------------------------------------------- launches ---
+cudaEvent_t pool_event(Ctx& c) {
+  if (!c.event_pool.empty()) {
+    cudaEvent_t e = c.event_pool.back();
+    c.event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+template <class F>
+int launch(Ctx& c, int kind, F&& f) {
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if (g_profile) {
+    e0 = pool_event(c);
+    e1 = pool_event(c);
+    cudaEventRecord(e0, c.stream);
+  }
+  f();
+  cudaError_t err = cudaGetLastError();
+  if (g_profile) {
+    cudaEventRecord(e1, c.stream);
+    c.prof.push_back({kind, e0, e1});
+  }
+  if (err != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
+  g_launches.fetch_add(1);
+  return MUON_OK;
+}
+
+struct StepIO {
+  float* const* W;          // outputs (W, or O when assign)
+  const float* const* g;
+  float* const* buf;        // may be null (no momentum)
+  float lr, mu, a, b, c, eps;
+  int ns_steps, nesterov, assign;
+};
+
+int check_status(Ctx& c) {
+  const int s = *(volatile int*)c.status_h;
+  if (s != 0) {
+    *(volatile int*)c.status_h = 0;
+    return fail(MUON_ERR_TIMEOUT, "an earlier launch on this stream gave up on a bounded wait (device code " +
+                                      std::to_string(s) + ")");
+  }
+  return MUON_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int run_group(Ctx& c, const Plan& plan, const Group& g, const StepIO& io) {
+  char* base = (char*)c.ws;
+  float* scale = (float*)(base + g.off_scale);
+  const CUtensorMap* tmaps = (const CUtensorMap*)((char*)plan.tmaps + g.off_tmaps);
+  const int nm = (int)g.mats.size();
+
+  // 1. prologue
+  {
+    auto pa = std::make_unique<ProArgs>();
+    std::memset(pa.get(), 0, sizeof(ProArgs));
+    pa->nmats = nm;
+    pa->total_tiles = g.pro_tiles;
+    pa->mu = io.mu;
+    pa->eps = io.eps;
+    pa->nesterov = io.nesterov;
+    pa->has_buf = io.buf != nullptr;
+    pa->partials = (float*)(base + g.off_partials);
+    pa->tickets = (unsigned*)(base + g.off_tickets);
+    pa->scale = scale;
+    for (const auto& cd : g.classes) {
+      for (size_t b = 0; b < cd.mats.size(); ++b) {
+        const int gi = cd.mats[b];
+        const MatDesc& d = g.mats[gi];
+        ProMat& pm = pa->mats[gi];
+        pm.g = io.g[d.user];
+        pm.buf = io.buf ? io.buf[d.user] : nullptr;
+        pm.x = (__nv_bfloat16*)(base + cd.off_x0 + b * (size_t)cd.kp * cd.lp * 2);
+        pm.m = d.m; pm.n = d.n; pm.kp = d.kp; pm.lp = d.lp;
+        pm.trans = d.trans;
+        pm.vec = (d.n % 4 == 0) && aligned16(pm.g) && (!pm.buf || aligned16(pm.buf));
+        pm.tile_begin = g.pro_tile_begin[gi];
+        pm.tiles_c = d.lp / kProCols;
+        pm.tiles = (d.kp / kProRows) * pm.tiles_c;
+      }
+    }
+    int rc = launch(c, MUON_KIND_PROLOGUE,
+                    [&] { prologue_kernel<<<g.pro_tiles, kProThreads, 0, c.stream>>>(*pa); });
+    if (rc) return rc;
+  }
+
+  auto fill_out = [&](OutMat* out) {
+    for (const auto& cd : g.classes)
+      for (size_t b = 0; b < cd.mats.size(); ++b) {
+        const int gi = cd.mats[b];
+        const MatDesc& d = g.mats[gi];
+        OutMat& o = out[gi];
+        o.w = io.W[d.user];
+        o.m = d.m; o.n = d.n; o.trans = d.trans;
+        o.vec = (d.n % 4 == 0) && aligned16(o.w);
+      }
+  };
+
+  if (io.ns_steps == 0) {
+    auto aa = std::make_unique<ApplyArgs>();
+    std::memset(aa.get(), 0, sizeof(ApplyArgs));
+    aa->scale = scale;
+    aa->lr = io.lr;
+    aa->assign = io.assign;
+    aa->nmats = nm;
+    fill_out(aa->out);
+    for (const auto& cd : g.classes)
+      for (size_t b = 0; b < cd.mats.size(); ++b) {
+        aa->x[cd.mats[b]] = (const __nv_bfloat16*)(base + cd.off_x0 + b * (size_t)cd.kp * cd.lp * 2);
+        aa->lp[cd.mats[b]] = cd.lp;
+      }
+    return launch(c, MUON_KIND_APPLY_X0,
+                  [&] { apply_x0_kernel<<<dim3(64, nm), 256, 0, c.stream>>>(*aa); });
+  }
+
+  auto ga = std::make_unique<GemmArgs>();
+  std::memset(ga.get(), 0, sizeof(GemmArgs));
+  ga->tmaps = tmaps;
+  ga->scale = scale;
+  ga->status = c.status_d;
+  ga->wait_limit_ns = g_wait_limit_ns;
+  ga->nclasses = (int)g.classes.size();
+  ga->a = io.a; ga->b = io.b; ga->c = io.c; ga->lr = io.lr;
+  ga->assign = io.assign;
+  fill_out(ga->out);
+
+  for (int it = 0; it < io.ns_steps; ++it) {
+    for (int mode = kModeGram; mode <= kModeUpdate; ++mode) {
+      const bool sym = mode != kModeUpdate;
+      const auto& cls = sym ? g.sym_cls : g.upd_cls;
+      for (size_t ci = 0; ci < cls.size(); ++ci) {
+        ga->cls[ci] = cls[ci];
+        if (mode == kModePoly) ga->cls[ci].kblocks = cls[ci].kp / kBK;
+      }
+      ga->total_tiles = sym ? g.sym_tiles : g.upd_tiles;
+      ga->mode = mode;
+      ga->x_in = it & 1;
+      ga->first = it == 0;
+      ga->final_apply = (mode == kModeUpdate) && (it == io.ns_steps - 1);
+      ga->debug_flags = 0;
+      if (g_debug_flags & 1) { ga->debug_flags = 1; g_debug_flags &= ~1; }
+      const int grid = std::min(ga->total_tiles, c.sm_count);
+      const int kind = mode == kModeGram ? MUON_KIND_GRAM
+                       : mode == kModePoly ? MUON_KIND_POLY
+                       : (ga->final_apply ? MUON_KIND_UPDATE_APPLY : MUON_KIND_UPDATE);
+      int rc = launch(c, kind, [&] {
+        ns_gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, c.stream>>>(*ga);
+      });
+      if (rc) return rc;
+    }
+  }
+  return MUON_OK;
+}
+
+int validate_common(const int64_t* shapes, int n, int ns_steps) {
+  if (!shapes) return fail(MUON_ERR_INVALID_ARG, "shapes is null");
+  if (n <= 0) return fail(MUON_ERR_INVALID_ARG, "n must be > 0");
+  if (ns_steps < 0 || ns_steps > 1000) return fail(MUON_ERR_INVALID_ARG, "ns_steps must be in [0, 1000]");
+  for (int i = 0; i < 2 * n; ++i)
+    if (shapes[i] <= 0) return fail(MUON_ERR_SHAPE, "shape entry " + std::to_string(i) + " is <= 0");
+  return MUON_OK;
+}
+
+int validate_ptrs(const void* const* arr, int n, const char* what) {
+  if (!arr) return fail(MUON_ERR_INVALID_ARG, std::string(what) + " array is null");
+  for (int i = 0; i < n; ++i)
+    if (!arr[i]) return fail(MUON_ERR_INVALID_ARG, std::string(what) + "[" + std::to_string(i) + "] is null");
+  return MUON_OK;
+}
+
+int step_impl(const StepIO& io, const int64_t* shapes, int n, void* stream) {
+  Ctx* c = nullptr;
+  int rc = get_ctx(stream, &c);
+  if (rc) return rc;
+  if ((rc = check_status(*c))) return rc;
+  Plan* plan = nullptr;
+  if ((rc = get_plan(*c, shapes, n, &plan))) return rc;
+  for (const auto& g : plan->groups)
+    if ((rc = run_group(*c, *plan, g, io))) return rc;
+  return MUON_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI ===
+extern "C" {
+
+int muon_step_ex(float* const* params, const float* const* grads, float* const* momentum_bufs,
+                 const int64_t* shapes, int n, float lr, float mu, int ns_steps,
+                 float a, float b, float c, float eps, int nesterov, void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int rc = validate_common(shapes, n, ns_steps);
+  if (rc) return rc;
+  if ((rc = validate_ptrs((const void* const*)params, n, "params"))) return rc;
+  if ((rc = validate_ptrs((const void* const*)grads, n, "grads"))) return rc;
+  if ((rc = validate_ptrs((const void* const*)momentum_bufs, n, "momentum_bufs"))) return rc;
+  if (nesterov != 0 && nesterov != 1) return fail(MUON_ERR_INVALID_ARG, "nesterov must be 0 or 1");
+  if (!(eps >= 0.f)) return fail(MUON_ERR_INVALID_ARG, "eps must be >= 0");
+  StepIO io{params, grads, momentum_bufs, lr, mu, a, b, c, eps, ns_steps, nesterov, 0};
+  return step_impl(io, shapes, n, stream);
+}
+
+int muon_step(float* const* params, const float* const* grads, float* const* momentum_bufs,
+              const int64_t* shapes, int n, float lr, float mu, int ns_steps, void* stream) {
+  return muon_step_ex(params, grads, momentum_bufs, shapes, n, lr, mu, ns_steps, MUON_NS_A, MUON_NS_B, MUON_NS_C,
+                      MUON_NS_EPS, 1, stream);
+}
+
+int muon_orthogonalize(const float* const* G, float* const* O, const int64_t* shapes, int n, int ns_steps,
+                       void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int rc = validate_common(shapes, n, ns_steps);
+  if (rc) return rc;
+  if ((rc = validate_ptrs((const void* const*)G, n, "G"))) return rc;
+  if ((rc = validate_ptrs((const void* const*)O, n, "O"))) return rc;
+  StepIO io{O, G, nullptr, 0.f, 0.f, MUON_NS_A, MUON_NS_B, MUON_NS_C, MUON_NS_EPS, ns_steps, 1, 1};
+  return step_impl(io, shapes, n, stream);
+}
+
+int muon_step_host(float* const* params, const float* const* grads, float* const* momentum_bufs,
+                   const int64_t* shapes, int n, float lr, float mu, int ns_steps, void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int rc = validate_common(shapes, n, ns_steps);
+  if (rc) return rc;
+  if ((rc = validate_ptrs((const void* const*)params, n, "params"))) return rc;
+  if ((rc = validate_ptrs((const void* const*)grads, n, "grads"))) return rc;
+  if ((rc = validate_ptrs((const void* const*)momentum_bufs, n, "momentum_bufs"))) return rc;
+  Ctx* c = nullptr;
+  if ((rc = get_ctx(stream, &c))) return rc;
+  size_t total = 0;
+  for (int i = 0; i < n; ++i) total += align_up((size_t)(shapes[2 * i] * shapes[2 * i + 1]), 64);
+  const size_t need = 3 * total * sizeof(float);
+  if (c->stage_cap < need) {
+    CUDA_TRY(cudaStreamSynchronize(c->stream));
+    if (c->stage) cudaFree(c->stage);
+    c->stage = nullptr;
+    c->stage_cap = 0;
+    if (cudaMalloc((void**)&c->stage, need) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(MUON_ERR_NOMEM, "staging allocation failed");
+    }
+    c->stage_cap = need;
+  }
+  std::vector<float*> dW(n), dg(n), db(n);
+  size_t off = 0;
+  for (int i = 0; i < n; ++i) {
+    const size_t e = (size_t)(shapes[2 * i] * shapes[2 * i + 1]);
+    dW[i] = c->stage + off;
+    dg[i] = c->stage + total + off;
+    db[i] = c->stage + 2 * total + off;
+    off += align_up(e, 64);
+    CUDA_TRY(cudaMemcpyAsync(dW[i], params[i], e * 4, cudaMemcpyHostToDevice, c->stream));
+    CUDA_TRY(cudaMemcpyAsync(dg[i], grads[i], e * 4, cudaMemcpyHostToDevice, c->stream));
+    CUDA_TRY(cudaMemcpyAsync(db[i], momentum_bufs[i], e * 4, cudaMemcpyHostToDevice, c->stream));
+  }
+  if ((rc = check_status(*c))) return rc;
+  Plan* plan = nullptr;
+  if ((rc = get_plan(*c, shapes, n, &plan))) return rc;
+  StepIO io{dW.data(), (const float* const*)dg.data(), db.data(), lr, mu, MUON_NS_A, MUON_NS_B, MUON_NS_C,
+            MUON_NS_EPS, ns_steps, 1, 0};
+  for (const auto& g : plan->groups)
+    if ((rc = run_group(*c, *plan, g, io))) return rc;
+  for (int i = 0; i < n; ++i) {
+    const size_t e = (size_t)(shapes[2 * i] * shapes[2 * i + 1]);
+    CUDA_TRY(cudaMemcpyAsync(params[i], dW[i], e * 4, cudaMemcpyDeviceToHost, c->stream));
+    CUDA_TRY(cudaMemcpyAsync(momentum_bufs[i], db[i], e * 4, cudaMemcpyDeviceToHost, c->stream));
+  }
+  CUDA_TRY(cudaStreamSynchronize(c->stream));
+  return check_status(*c);
+}
+
+size_t muon_workspace_size(const int64_t* shapes, int n) {
+  if (!shapes || n <= 0) return 0;
+  for (int i = 0; i < 2 * n; ++i)
+    if (shapes[i] <= 0) return 0;
+  Plan p;
+  if (build_layout(shapes, n, p)) return 0;
+  return p.ws_bytes;
+}
+
+int muon_sync_status(void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  Ctx* c = nullptr;
+  int rc = get_ctx(stream, &c);
+  if (rc) return rc;
+  CUDA_TRY(cudaStreamSynchronize(c->stream));
+  return check_status(*c);
+}
+
+const char* muon_last_error(void) { return g_last_error.c_str(); }
+
+void muon_release(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (auto& kv : g_ctx) {
+    Ctx& c = *kv.second;
+    cudaSetDevice(c.dev);
+    cudaStreamSynchronize(c.stream);
+    if (c.ws) cudaFree(c.ws);
+    if (c.stage) cudaFree(c.stage);
+    if (c.status_h) cudaFreeHost(c.status_h);
+    for (auto& r : c.prof) { cudaEventDestroy(r.a); cudaEventDestroy(r.b); }
+    for (auto e : c.event_pool) cudaEventDestroy(e);
+  }
+  g_ctx.clear();
+  cudaSetDevice(cur);
+}
+
+int muon_profile_enable(int enable) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_profile = enable != 0;
+  return MUON_OK;
+}
+
+int muon_profile_read(double* ms, int64_t* launches, int nkinds) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!ms || !launches || nkinds <= 0) return fail(MUON_ERR_INVALID_ARG, "bad profile buffers");
+  for (auto& kv : g_ctx) {
+    Ctx& c = *kv.second;
+    for (auto& r : c.prof) {
+      if (cudaEventSynchronize(r.b) != cudaSuccess) return fail(MUON_ERR_CUDA, "event synchronize failed");
+      float t = 0.f;
+      cudaEventElapsedTime(&t, r.a, r.b);
+      if (r.kind < nkinds) { ms[r.kind] += t; launches[r.kind] += 1; }
+      c.event_pool.push_back(r.a);
+      c.event_pool.push_back(r.b);
+    }
+    c.prof.clear();
+  }
+  return MUON_OK;
+}
+
+int64_t muon_launch_count(void) { return g_launches.load(); }
+
+int muon_debug_set(int flags, int64_t wait_limit_ns) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_debug_flags = flags;
+  g_wait_limit_ns = wait_limit_ns > 0 ? (uint64_t)wait_limit_ns : 2000000000ull;
+  return MUON_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,111 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every
+function include/muon.h declares, validates arguments on the host before any
+CUDA call, and sizes its workspace as documented."""
+
+import ctypes
+
+import pytest
+
+import __graft_entry__
+import muon_newton_schulz_02_b200 as muon
+
+INVALID, SHAPE = -1, -2
+
+
+@pytest.fixture(scope="module")
+def L():
+    __graft_entry__.build()
+    return muon.lib()
+
+
+def test_exports_every_declared_function(L):
+    names = muon.header_functions()
+    assert {"muon_step", "muon_step_ex", "muon_orthogonalize", "muon_step_host", "muon_workspace_size",
+            "muon_sync_status", "muon_last_error", "muon_release", "muon_profile_enable",
+            "muon_profile_read", "muon_launch_count", "muon_debug_set"} <= set(names)
+    for f in names:
+        assert hasattr(L, f), f
+
+
+def _arr(n, v=1):
+    return (ctypes.c_void_p * n)(*[ctypes.c_void_p(v)] * n)
+
+
+def _shapes(*dims):
+    return (ctypes.c_int64 * len(dims))(*dims)
+
+
+def test_argument_errors_are_reported_before_any_launch(L):
+    p = _arr(1)
+    sh = _shapes(4, 8)
+    assert L.muon_step(p, p, p, None, 1, 0.02, 0.95, 5, None) == INVALID
+    assert "shapes" in muon.last_error()
+    assert L.muon_step(p, p, p, sh, 0, 0.02, 0.95, 5, None) == INVALID
+    assert L.muon_step(p, p, p, sh, 1, 0.02, 0.95, -1, None) == INVALID
+    assert L.muon_step(p, p, p, _shapes(0, 8), 1, 0.02, 0.95, 5, None) == SHAPE
+    assert L.muon_step(p, p, p, _shapes(4, -3), 1, 0.02, 0.95, 5, None) == SHAPE
+    assert L.muon_step(None, p, p, sh, 1, 0.02, 0.95, 5, None) == INVALID
+    assert L.muon_step(p, p, _arr(1, 0), sh, 1, 0.02, 0.95, 5, None) == INVALID
+    assert "momentum_bufs[0]" in muon.last_error()
+    assert L.muon_step_ex(p, p, p, sh, 1, 0.02, 0.95, 5, 3.4445, -4.775, 2.0315, 1e-7, 2, None) == INVALID
+    assert L.muon_step_ex(p, p, p, sh, 1, 0.02, 0.95, 5, 3.4445, -4.775, 2.0315, -1.0, 1, None) == INVALID
+    assert L.muon_orthogonalize(p, _arr(1, 0), sh, 1, 5, None) == INVALID
+    assert L.muon_step_host(p, None, p, sh, 1, 0.02, 0.95, 5, None) == INVALID
+
+
+def _ws(shapes):
+    flat = [v for s in shapes for v in s]
+    return muon.lib().muon_workspace_size((ctypes.c_int64 * len(flat))(*flat), len(shapes))
+
+
+def _expect_ws(shapes):
+    """Layout documented in the C source: a fixed 4 KiB region of norm
+    arrival counters, then per shape class (padded short side kp, long side
+    lp, both multiples of 128) two bf16 iterates [B][kp][lp] and two bf16
+    [B][kp][kp] matrices, then per-tile norm partials (64x128 tiles) and
+    per-matrix scales, each region rounded to 1 KiB."""
+    up = lambda v, a: (v + a - 1) // a * a
+    classes = {}
+    for r, c in shapes:
+        k, l = min(r, c), max(r, c)
+        classes.setdefault((up(k, 128), up(l, 128)), []).append((r, c))
+    off = 4096
+    tiles = 0
+    for (kp, lp), mats in classes.items():
+        b = len(mats)
+        off = up(off + b * kp * lp * 2, 1024)
+        off = up(off + b * kp * lp * 2, 1024)
+        off = up(off + b * kp * kp * 2, 1024)
+        off = up(off + b * kp * kp * 2, 1024)
+        tiles += b * (kp // 64) * (lp // 128)
+    n = len(shapes)
+    off = up(off + tiles * 4, 1024)
+    off = up(off + n * 4, 1024)
+    return off
+
+
+@pytest.mark.parametrize("shapes", [
+    [(128, 512)],
+    [(768, 768)] * 4 + [(768, 3072), (3072, 768)],
+    [(1, 1), (127, 129), (129, 127), (1000, 300)],
+])
+def test_workspace_size_matches_layout(L, shapes):
+    assert _ws(shapes) == _expect_ws(shapes)
+
+
+def test_workspace_size_rejects_bad_input(L):
+    assert _ws([(0, 4)]) == 0
+    assert muon.lib().muon_workspace_size(None, 1) == 0
+
+
+def test_many_matrices_split_into_groups(L):
+    # more matrices than one launch holds: groups share the data region
+    shapes = [(64, 64)] * 700
+    one_group = _expect_ws([(64, 64)] * 320)
+    got = _ws(shapes)
+    assert got == one_group
+
+
+def test_launch_count_and_debug_hooks_run_without_gpu(L):
+    assert muon.launch_count() == 0
+    muon.debug_set(0, 0)
