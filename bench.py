@@ -1,0 +1,426 @@
+"""Benchmark of the Muon step on B200: prints ONE JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gpt2_124m]
+                    [--impl ours|reference]
+
+A step is one Muon update (Nesterov momentum, NS5, W -= lr*O) over every
+matrix of the workload, with inputs resident in HBM.  ``value`` is
+algorithmic NS5 TFLOP/s of the whole job (symmetry of X X^T and A A
+exploited, 5*(k(k+1)l + k^2(k+1) + 2k^2 l) per k x l matrix, k <= l);
+``ms_per_step`` the device time per step.  Under torchrun every rank runs its
+own copy of the workload (independent problems, no collective on the data
+path: weak scaling) and the time is the maximum over ranks.
+
+``--impl reference`` times the CPU oracle (float64 numpy) on the host cores on
+a bounded sample of the same workload, per the same metric.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Muon NS5 bf16 TFLOP/s (% of B200 tensor peak); ms per GPT-2-124M Muon step"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def ns_flops(shapes, ns_steps=5) -> float:
+    tot = 0.0
+    for r, c in shapes:
+        k, l = min(r, c), max(r, c)
+        tot += ns_steps * (k * (k + 1) * l + k * k * (k + 1) + 2 * k * k * l)
+    return tot
+
+
+def flops_by_kind(shapes, ns_steps=5):
+    g = p = u = 0.0
+    for r, c in shapes:
+        k, l = min(r, c), max(r, c)
+        g += k * (k + 1) * l
+        p += k * k * (k + 1)
+        u += 2 * k * k * l
+    return {"gram": g * ns_steps, "poly": p * ns_steps, "update": u * ns_steps}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("kernels.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "muon_newton_schulz_02_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic():
+    """DRAM bytes per launch of the GEMM kernel from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "ns_gemm_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch_full_workload")
+
+
+# ---------------------------------------------------------------- clocks ---
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.dev = self._smi_id(device_index)
+
+    @staticmethod
+    def _smi_id(i):
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(i)
+            return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            return vis.split(",")[i] if vis else str(i)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.dev, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------- CPU oracle ---
+def cpu_oracle_rate(w, budget_s=12.0):
+    """Times the oracle as it stands on a bounded sample of the workload's
+    matrices (cycling through its distinct shapes) on the host cores."""
+    import numpy as np
+    from muon_newton_schulz_02_b200 import workloads
+    from oracle import muon_oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"] or [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    idx = workloads.sample_indices(w, per_shape=64)
+    order = []
+    by_shape = {}
+    for i in idx:
+        by_shape.setdefault(w.shapes[i], []).append(i)
+    while any(by_shape.values()):
+        for s in list(by_shape):
+            if by_shape[s]:
+                order.append(by_shape[s].pop(0))
+    done, flops, t_used = [], 0.0, 0.0
+    for i in order:
+        g = workloads.grad(w, 0, i).numpy()
+        W = workloads.weight(w, i).numpy()
+        buf = np.zeros_like(g)
+        t0 = time.perf_counter()
+        muon_oracle.muon_update(W, g, buf, w.lr, w.mu)
+        t_used += time.perf_counter() - t0
+        flops += ns_flops([w.shapes[i]])
+        done.append(w.shapes[i])
+        if t_used >= budget_s:
+            break
+    shapes_desc = {}
+    for s in done:
+        shapes_desc[f"{s[0]}x{s[1]}"] = shapes_desc.get(f"{s[0]}x{s[1]}", 0) + 1
+    return {"value": flops / t_used / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{len(done)} of {w.n_matrices} matrices ({shapes_desc}), one Muon step each, "
+                      f"{t_used:.1f} s of float64 numpy",
+            "seconds": t_used}
+
+
+# ------------------------------------------------------------------ main ---
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), ws
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    from muon_newton_schulz_02_b200 import workloads
+    w = workloads.get(args.workload)
+    # each step: a bounded sample (at least one matrix), sized so the whole
+    # run stays within --ref-total seconds of CPU work
+    per_step = args.ref_total / max(1, args.steps + args.warmup)
+    flops = secs = 0.0
+    base = None
+    for s in range(args.warmup + args.steps):
+        r = cpu_oracle_rate(w, budget_s=per_step)
+        if s >= args.warmup:
+            flops += r["value"] * 1e12 * r["seconds"]
+            secs += r["seconds"]
+        base = r
+    val = flops / secs / 1e12
+    flops_step = ns_flops(w.shapes)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": flops_step / (val * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,0.02) gradients of the GPT-2-124M hidden-matrix shapes)",
+        "config": workload_config(w, args),
+        "cpu_baseline": {k: base[k] for k in ("kind", "cores", "sample")} | {"value": val, "unit": UNIT},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, args):
+    shapes = {}
+    for s in w.shapes:
+        shapes[f"{s[0]}x{s[1]}"] = shapes.get(f"{s[0]}x{s[1]}", 0) + 1
+    return {"workload": w.name, "matrices": w.n_matrices, "shapes": shapes, "ns_steps": 5,
+            "mu": w.mu, "lr": w.lr, "nesterov": True, "grad_sets": args.grad_sets,
+            "l2": f"inputs larger than L2: W, g, buf are {w.n_elements * 12 / 1e9:.2f} GB per step",
+            "parallelism": f"independent replicas x{args.gpus}"}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import __graft_entry__
+    __graft_entry__.build()
+    import muon_newton_schulz_02_b200 as muon
+    from muon_newton_schulz_02_b200 import workloads
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = workloads.get(args.workload)
+    n = w.n_matrices
+    W = workloads.weights(w, device=dev)
+    bufs = workloads.zero_bufs(w, device=dev)
+    gsets = [workloads.grads(w, s, device=dev) for s in range(args.grad_sets)]
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def one_step(s):
+        muon.step(W, gsets[s % args.grad_sets], bufs, lr=w.lr, mu=w.mu, stream=stream)
+
+    for s in range(args.warmup):
+        one_step(s)
+    torch.cuda.synchronize(dev)
+    if muon.sync_status(stream) != 0:
+        raise RuntimeError("device status after warm-up: " + muon.last_error())
+
+    # ---- timed region: device time with CUDA events on the launching stream
+    muon.profile_read()                         # drop anything recorded so far
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.start()
+        time.sleep(0.2)
+    l0 = muon.launch_count()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(args.steps):
+        one_step(s)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = muon.launch_count() - l0
+    barrier()
+    clk = clocks.stop() if clocks else None
+    ms = e0.elapsed_time(e1)
+
+    # ---- second pass, same steps, every launch bracketed by CUDA events on its
+    # stream: per-kernel device durations for the roofline (the events cost a
+    # few percent, so the headline value comes from the pass above)
+    prof = {k: (0.0, 0) for k in muon.KINDS}
+    ms_prof = None
+    if args.kernel_events:
+        muon.profile_enable(True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        p0 = torch.cuda.Event(enable_timing=True)
+        p1 = torch.cuda.Event(enable_timing=True)
+        p0.record(stream)
+        for s in range(args.steps):
+            one_step(s)
+        p1.record(stream)
+        torch.cuda.synchronize(dev)
+        muon.profile_enable(False)
+        prof = muon.profile_read()
+        ms_prof = p0.elapsed_time(p1)
+    if muon.sync_status(stream) != 0:
+        raise RuntimeError("device status after timing: " + muon.last_error())
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    flops_step = ns_flops(w.shapes)
+    value = flops_step * args.steps * world / (ms_max / 1e3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    fk = flops_by_kind(w.shapes)
+    kinds = {}
+    gemm_ms = sum(prof[k][0] for k in ("gram", "poly", "update", "update_apply"))
+    gemm_launches = sum(prof[k][1] for k in ("gram", "poly", "update", "update_apply"))
+    for k, (tms, cnt) in prof.items():
+        if cnt:
+            kinds[k] = {"launches": cnt, "ms_total": tms, "us_per_launch": tms / cnt * 1e3,
+                        "share_of_step": tms / ms_prof}
+    roofline = None
+    if gemm_launches and args.kernel_events:
+        gemm_flops_per_launch = flops_step * args.steps / gemm_launches
+        achieved = gemm_flops_per_launch / (gemm_ms / gemm_launches / 1e3) / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        roofline = {"bound": "tensor", "kernel": "ns_gemm_kernel", "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak, "traffic": ncu_traffic(),
+                    "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)",
+                    "flops_per_launch": gemm_flops_per_launch,
+                    "us_per_launch": gemm_ms / gemm_launches * 1e3}
+        if "prologue" in kinds:
+            pro_bytes = 14.0 * w.n_elements
+            pro_s = prof["prologue"][0] / prof["prologue"][1] / 1e3
+            roofline["prologue"] = {"bound": "hbm", "achieved": pro_bytes / pro_s / 1e9,
+                                    "peak": float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
+                                    "unit": "GB/s",
+                                    "frac": pro_bytes / pro_s / 1e9 / float(peaks.get("hbm_gbs", 6650.0)),
+                                    "bytes_per_launch": pro_bytes}
+
+    # ---- end to end through the host-buffer entry point
+    e2e = None
+    if not args.no_e2e:
+        Wh = [x.cpu().pin_memory() for x in W]
+        bh = [x.cpu().pin_memory() for x in bufs]
+        gh = [[x.cpu().pin_memory() for x in gs] for gs in gsets[:2]]
+        for s in range(2):
+            muon.step_host(Wh, gh[s % 2], bh, lr=w.lr, mu=w.mu, stream=stream)
+        barrier()
+        k2 = max(2, min(args.steps, args.e2e_steps))
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        for s in range(k2):
+            muon.step_host(Wh, gh[s % 2], bh, lr=w.lr, mu=w.mu, stream=stream)
+        el = time.perf_counter() - t0
+        te = torch.tensor([el], device=dev, dtype=torch.float64)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        el = float(te.item())
+        e2e = {"value": flops_step * k2 * world / el / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": 12 * w.n_elements, "d2h_bytes_per_step": 8 * w.n_elements,
+               "ms_per_step": el / k2 * 1e3, "steps": k2,
+               "path": "muon_step_host: pinned host W, g, buf -> device, step, W and buf -> host"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = cpu_oracle_rate(w, budget_s=args.ref_budget)
+        cpu = {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) gradients, N(0,0.02) weights, zero-initialised momentum; "
+                "GPT-2-124M hidden-matrix shapes)",
+        "config": workload_config(w, args),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+        "kernels": kinds,
+        "frac_of_dense_peak": value / world / float(peaks.get("bf16_tflops", 1647.8)),
+        "peaks": {"source": peak_src, "bf16_tflops": peaks.get("bf16_tflops"),
+                  "bf16_tflops_sustained": peaks.get("bf16_tflops_sustained"), "hbm_gbs": peaks.get("hbm_gbs")},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="gpt2_124m")
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--grad-sets", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of CPU oracle work (cpu_baseline)")
+    ap.add_argument("--ref-total", type=float, default=90.0, help="seconds of CPU oracle work (--impl reference)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-events", type=int, default=1, help="per-launch CUDA events in the timed region")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

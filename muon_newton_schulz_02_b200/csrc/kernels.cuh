@@ -62,10 +62,12 @@ struct OutMat {       // destination of the final UPDATE epilogue
   int m, n;
   int trans;          // 1: X holds W^T (m > n)
   int vec;            // 1: n % 4 == 0 and w 16-byte aligned
+  int tma;            // 1: wmaps[] holds a valid fp32 tensor map of w (needs vec)
 };
 
 struct GemmArgs {
   const CUtensorMap* tmaps;
+  const CUtensorMap* wmaps;   // per matrix (group order): W as fp32 [m][n]; box 32x128 (X = W) or 32x32 (X = W^T)
   const float* scale;     // per matrix (group order): 1/(||G||_F + eps)
   int* status;
   unsigned long long wait_limit_ns;
@@ -291,6 +293,51 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& p, int t, bool 
 // box stored with the 128-byte swizzle (the pattern TMA writes / reads).
 __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t u) { return r * 128u + ((u ^ (r & 7u)) << 4); }
 
+// Read-modify-write of one 128 x 32 slice of the final result into W (or
+// O), staged in shared memory by the epilogue.  X row gi0 + r, col gj0 + c maps
+// to W[gi][gj] (X = W) or W[gj][gi] (X = W^T).  Each warp touches whole rows.
+__device__ __forceinline__ void store_w_slice(const OutMat& O, const float* S, int gi0, int gj0, int et, float lr,
+                                              int assign) {
+  // all loads of the slice are issued before any store (8 in flight per thread)
+  float4 o[8], w[8];
+  float* wp[8];
+  bool ok[8], full[8];
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    int row, col, sidx;
+    if (!O.trans) {
+      const int rr = it * 16 + (et >> 3), q = et & 7;
+      row = gi0 + rr; col = gj0 + 4 * q;
+      sidx = rr * 32 + ((q ^ (rr & 7)) << 2);
+      ok[it] = row < O.m && col < O.n;
+    } else {
+      const int c = it * 4 + (et >> 5), q = et & 31;
+      row = gj0 + c; col = gi0 + 4 * q;          // W[row][col..col+3]
+      sidx = c * kBM + 4 * q;
+      ok[it] = row < O.m && col < O.n;
+    }
+    full[it] = O.vec && col + 3 < O.n;
+    wp[it] = O.w + (size_t)row * O.n + col;
+    o[it] = *reinterpret_cast<const float4*>(S + sidx);
+    w[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (ok[it] && full[it] && !assign) w[it] = *reinterpret_cast<const float4*>(wp[it]);
+  }
+  const float sg = assign ? -1.f : lr;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    if (!ok[it]) continue;
+    if (full[it]) {
+      float4 r4 = w[it];
+      r4.x -= sg * o[it].x; r4.y -= sg * o[it].y; r4.z -= sg * o[it].z; r4.w -= sg * o[it].w;
+      *reinterpret_cast<float4*>(wp[it]) = r4;
+    } else {
+      const float ov[4] = {o[it].x, o[it].y, o[it].z, o[it].w};
+      const int col = (int)((wp[it] - O.w) % O.n);
+      for (int e = 0; e < 4 && col + e < O.n; ++e) wp[it][e] = assign ? ov[e] : wp[it][e] - lr * ov[e];
+    }
+  }
+}
+
 struct __align__(8) GemmCtrl {
   uint64_t full[kStages];
   uint64_t empty[kStages];
@@ -441,9 +488,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     const int q = warp & 3;                       // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;                  // tile row owned by this thread
     const float alpha_first = 1.0f;
-    if (et == 0)
+    if (et == 0) {
       for (int c = 0; c < p.nclasses; ++c)
         for (int k = 0; k < kTmapsPerClass; ++k) tmap_acquire(&p.tmaps[p.cls[c].tmap_base + k]);
+      if (p.mode == kModeUpdate && p.final_apply)
+        for (int c = 0; c < p.nclasses; ++c)
+          for (int b = 0; b < p.cls[c].batch; ++b)
+            if (p.out[p.cls[c].mat_first + b].tma) tmap_acquire(&p.wmaps[p.cls[c].mat_first + b]);
+    }
     int it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
@@ -455,7 +507,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       if (ok) ok = mbar_wait(&ctl->tmem_full[acc], acc_phase, wc, kDevTimeoutAccum);
       tc_fence_after();
       if (ok && has_d) ok = mbar_wait(&ctl->dfull, (uint32_t)(it & 1), wc, kDevTimeoutEpi);
-      ok = __all_sync(0xffffffffu, ok);             // tcgen05.ld below needs the whole warp
+      // one outcome for all 128 epilogue threads: the branch below holds named
+      // barriers and warp-collective tcgen05.ld
+      ok = named_bar_and(1, kEpiThreads, ok);
       const float s = p.first ? p.scale[mat] : alpha_first;
       const bool mirror = sym && tc.tm != tc.tn;
       const bool final_w = p.mode == kModeUpdate && p.final_apply;
@@ -488,44 +542,62 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
               }
             }
           }
-          if (final_w) {
+          if (final_w && p.out[mat].tma) {
+            // -lr*O (or O) for a 128 x 32 slice, staged 128-byte swizzled; TMA adds
+            // it to W in L2 (or stores it), so W never passes through the SM.
             const OutMat& O = p.out[mat];
-            const int gi = tc.tm * kBM + r;               // row of X
-            const int gj0 = tc.tn * kBN + cc * 32;        // first col of X in this chunk
+            const float sg = p.assign ? 1.f : -p.lr;
+            uint8_t* S = mtile + (cc & 1) * kChunkBytes;
             if (!O.trans) {
-              if (gi < O.m) {
-                float* wrow = O.w + (size_t)gi * O.n;
-                if (O.vec) {
 #pragma unroll
-                  for (int i = 0; i < 32; i += 4) {
-                    const int gj = gj0 + i;
-                    if (gj < O.n) {
-                      float4* wp = reinterpret_cast<float4*>(wrow + gj);
-                      float4 w4 = p.assign ? make_float4(0.f, 0.f, 0.f, 0.f) : *wp;
-                      const float sg = p.assign ? -1.f : p.lr;
-                      w4.x -= sg * v[i]; w4.y -= sg * v[i + 1]; w4.z -= sg * v[i + 2]; w4.w -= sg * v[i + 3];
-                      *wp = w4;
-                    }
-                  }
-                } else {
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<float4*>(S + sw128_off((uint32_t)r, (uint32_t)j)) =
+                    make_float4(sg * v[4 * j], sg * v[4 * j + 1], sg * v[4 * j + 2], sg * v[4 * j + 3]);
+            } else {
+              // box h = r / 32 holds W rows gj0..gj0+31 x W cols gi0+32h..+31
+              uint8_t* Sh = S + (r >> 5) * 4096;
+              const int rr = r & 31;
 #pragma unroll
-                  for (int i = 0; i < 32; ++i) {
-                    const int gj = gj0 + i;
-                    if (gj < O.n) wrow[gj] = p.assign ? v[i] : wrow[gj] - p.lr * v[i];
-                  }
-                }
-              }
-            } else if (gi < O.n) {
-              // X = W^T: element (gi, gj) of X is W[gj][gi]; a warp writes 32 consecutive floats.
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int gj = gj0 + i;
-                if (gj < O.m) {
-                  float* wp = O.w + (size_t)gj * O.n + gi;
-                  *wp = p.assign ? v[i] : *wp - p.lr * v[i];
-                }
-              }
+              for (int i = 0; i < 32; ++i)
+                *reinterpret_cast<float*>(Sh + sw128_off((uint32_t)i, (uint32_t)(rr >> 2)) + (rr & 3) * 4) =
+                    sg * v[i];
             }
+            fence_async_shared();
+            named_bar_sync(1, kEpiThreads);
+            if (et == 0) {
+              const CUtensorMap* wm = &p.wmaps[mat];
+              const int gi0 = tc.tm * kBM, gj0 = tc.tn * kBN + cc * 32;
+              if (!O.trans) {
+                if (p.assign) tma_store_2d(wm, S, gj0, gi0); else tma_reduce_add_2d(wm, S, gj0, gi0);
+              } else {
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  if (p.assign) tma_store_2d(wm, S + h * 4096, gi0 + 32 * h, gj0);
+                  else tma_reduce_add_2d(wm, S + h * 4096, gi0 + 32 * h, gj0);
+                }
+              }
+              tma_store_commit();
+              tma_store_wait_read1();          // the other staging buffer is free again
+            }
+            named_bar_sync(1, kEpiThreads);
+          } else if (final_w) {
+            // fp32 result slice (128 rows x 32 cols) through shared memory so that
+            // W is read and written in whole 128-byte rows.
+            const OutMat& O = p.out[mat];
+            float* S = reinterpret_cast<float*>(mtile + (cc & 1) * (kChunkBytes));
+            if (!O.trans) {
+              // S[row][quad ^ (row & 7)]: 8 float4 per row
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<float4*>(S + r * 32 + ((j ^ (r & 7)) << 2)) =
+                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            } else {
+              // S[col][row]: row c of S is a 128-float row of W
+#pragma unroll
+              for (int i = 0; i < 32; ++i) S[i * kBM + r] = v[i];
+            }
+            named_bar_sync(1, kEpiThreads);
+            store_w_slice(O, S, tc.tm * kBM, tc.tn * kBN + cc * 32, et, p.lr, p.assign);
           } else {
             // bf16 output tile (in place over the input tile), 128-byte swizzled for the TMA store
 #pragma unroll

@@ -79,7 +79,7 @@ struct Group {
   std::vector<ClassDesc> classes;
   std::vector<int> pro_tile_begin;
   int pro_tiles = 0;
-  size_t off_partials = 0, off_tickets = 0, off_scale = 0, off_tmaps = 0;
+  size_t off_partials = 0, off_tickets = 0, off_scale = 0, off_tmaps = 0, off_wmaps = 0;
   size_t data_bytes = 0;
   int sym_tiles = 0, upd_tiles = 0;
   std::vector<GemmClass> sym_cls, upd_cls;
@@ -99,8 +99,16 @@ struct Plan {
   size_t tmap_bytes = 0;
   void* ws = nullptr;                       // workspace the tensor maps point into
   void* tmaps = nullptr;                    // this plan's own device copy of its tensor maps
+  // Per group: fp32 tensor maps of the caller's output matrices, re-encoded
+  // when the caller passes other pointers; host copy in pinned memory.
+  std::vector<std::vector<const void*>> wmap_key;
+  std::vector<CUtensorMap*> wmap_host;
+  cudaEvent_t wmap_copied = nullptr;
   ~Plan() {
     if (tmaps) cudaFree(tmaps);
+    for (auto h : wmap_host)
+      if (h) cudaFreeHost(h);
+    if (wmap_copied) cudaEventDestroy(wmap_copied);
   }
 };
 
@@ -198,6 +206,8 @@ int build_layout(const int64_t* shapes, int n, Plan& plan) {
   for (auto& g : plan.groups) {
     g.off_tmaps = off;
     off = align_up(off + g.classes.size() * kTmapsPerClass * sizeof(CUtensorMap), 1024);
+    g.off_wmaps = off;
+    off = align_up(off + g.mats.size() * sizeof(CUtensorMap), 1024);
   }
   plan.tmap_bytes = off;
   plan.ws_bytes = data_max;
@@ -215,6 +225,21 @@ int encode_map(CUtensorMap* map, void* base, int cols, int rows, int batch, int 
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return MUON_OK;
+}
+
+// W (m x n fp32, row-major, n % 4 == 0, 16-byte aligned) as a 2-D tensor map
+// for the final epilogue: box 32 cols x 128 rows (X = W) or 32 x 32 (X = W^T).
+int encode_wmap(CUtensorMap* map, void* w, int m, int n, int trans) {
+  auto fn = encode_fn();
+  if (!fn) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {(cuuint64_t)n, (cuuint64_t)m};
+  cuuint64_t strides[1] = {(cuuint64_t)n * 4};
+  cuuint32_t box[2] = {32, trans ? 32u : 128u};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, w, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled (W) failed: " + std::to_string((int)r));
   return MUON_OK;
 }
 
@@ -325,6 +350,17 @@ int get_plan(Ctx& c, const int64_t* shapes, int n, Plan** out) {
     CUDA_TRY(cudaMemcpy((char*)p->tmaps + g.off_tmaps, maps.data(), maps.size() * sizeof(CUtensorMap),
                         cudaMemcpyHostToDevice));
   }
+  p->wmap_key.resize(p->groups.size());
+  p->wmap_host.assign(p->groups.size(), nullptr);
+  for (size_t gi = 0; gi < p->groups.size(); ++gi) {
+    if (cudaHostAlloc((void**)&p->wmap_host[gi], p->groups[gi].mats.size() * sizeof(CUtensorMap),
+                      cudaHostAllocDefault) != cudaSuccess) {
+      cudaGetLastError();
+      p->wmap_host[gi] = nullptr;
+      return fail(MUON_ERR_NOMEM, "pinned tensor-map staging allocation failed");
+    }
+  }
+  CUDA_TRY(cudaEventCreateWithFlags(&p->wmap_copied, cudaEventDisableTiming));
   c.plans.push_front(std::move(p));
   if (c.plans.size() > 4) {
     CUDA_TRY(cudaStreamSynchronize(c.stream));
@@ -385,7 +421,33 @@ int check_status(Ctx& c) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int run_group(Ctx& c, const Plan& plan, const Group& g, const StepIO& io) {
+// Encodes and uploads the output tensor maps of group gi if the caller's
+// output pointers differ from the ones encoded last time.
+int update_wmaps(Ctx& c, Plan& plan, size_t gi, const StepIO& io) {
+  const Group& g = plan.groups[gi];
+  std::vector<const void*> key(g.mats.size());
+  for (size_t i = 0; i < g.mats.size(); ++i) key[i] = io.W[g.mats[i].user];
+  if (key == plan.wmap_key[gi]) return MUON_OK;
+  CUDA_TRY(cudaEventSynchronize(plan.wmap_copied));       // the staging buffer is free
+  CUtensorMap* h = plan.wmap_host[gi];
+  std::memset(h, 0, g.mats.size() * sizeof(CUtensorMap));
+  for (size_t i = 0; i < g.mats.size(); ++i) {
+    const MatDesc& d = g.mats[i];
+    void* w = (void*)io.W[d.user];
+    if (d.n % 4 == 0 && aligned16(w)) {
+      int rc = encode_wmap(&h[i], w, d.m, d.n, d.trans);
+      if (rc) return rc;
+    }
+  }
+  CUDA_TRY(cudaMemcpyAsync((char*)plan.tmaps + g.off_wmaps, h, g.mats.size() * sizeof(CUtensorMap),
+                           cudaMemcpyHostToDevice, c.stream));
+  CUDA_TRY(cudaEventRecord(plan.wmap_copied, c.stream));
+  plan.wmap_key[gi] = key;
+  return MUON_OK;
+}
+
+int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
+  const Group& g = plan.groups[gidx];
   char* base = (char*)c.ws;
   float* scale = (float*)(base + g.off_scale);
   const CUtensorMap* tmaps = (const CUtensorMap*)((char*)plan.tmaps + g.off_tmaps);
@@ -434,6 +496,7 @@ int run_group(Ctx& c, const Plan& plan, const Group& g, const StepIO& io) {
         o.w = io.W[d.user];
         o.m = d.m; o.n = d.n; o.trans = d.trans;
         o.vec = (d.n % 4 == 0) && aligned16(o.w);
+        o.tma = o.vec;
       }
   };
 
@@ -454,9 +517,12 @@ int run_group(Ctx& c, const Plan& plan, const Group& g, const StepIO& io) {
                   [&] { apply_x0_kernel<<<dim3(64, nm), 256, 0, c.stream>>>(*aa); });
   }
 
+  int rc0 = update_wmaps(c, plan, gidx, io);
+  if (rc0) return rc0;
   auto ga = std::make_unique<GemmArgs>();
   std::memset(ga.get(), 0, sizeof(GemmArgs));
   ga->tmaps = tmaps;
+  ga->wmaps = (const CUtensorMap*)((char*)plan.tmaps + g.off_wmaps);
   ga->scale = scale;
   ga->status = c.status_d;
   ga->wait_limit_ns = g_wait_limit_ns;
@@ -516,8 +582,8 @@ int step_impl(const StepIO& io, const int64_t* shapes, int n, void* stream) {
   if ((rc = check_status(*c))) return rc;
   Plan* plan = nullptr;
   if ((rc = get_plan(*c, shapes, n, &plan))) return rc;
-  for (const auto& g : plan->groups)
-    if ((rc = run_group(*c, *plan, g, io))) return rc;
+  for (size_t gi = 0; gi < plan->groups.size(); ++gi)
+    if ((rc = run_group(*c, *plan, gi, io))) return rc;
   return MUON_OK;
 }
 
@@ -599,8 +665,8 @@ int muon_step_host(float* const* params, const float* const* grads, float* const
   if ((rc = get_plan(*c, shapes, n, &plan))) return rc;
   StepIO io{dW.data(), (const float* const*)dg.data(), db.data(), lr, mu, MUON_NS_A, MUON_NS_B, MUON_NS_C,
             MUON_NS_EPS, ns_steps, 1, 0};
-  for (const auto& g : plan->groups)
-    if ((rc = run_group(*c, *plan, g, io))) return rc;
+  for (size_t gi = 0; gi < plan->groups.size(); ++gi)
+    if ((rc = run_group(*c, *plan, gi, io))) return rc;
   for (int i = 0; i < n; ++i) {
     const size_t e = (size_t)(shapes[2 * i] * shapes[2 * i + 1]);
     CUDA_TRY(cudaMemcpyAsync(params[i], dW[i], e * 4, cudaMemcpyDeviceToHost, c->stream));
