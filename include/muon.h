@@ -106,6 +106,38 @@ int muon_orthogonalize(const float* const* G, float* const* O, const int64_t* sh
 int muon_step_host(float* const* params, const float* const* grads, float* const* momentum_bufs,
                    const int64_t* shapes, int n, float lr, float mu, int ns_steps, void* stream);
 
+/*
+ * muon_step without any device allocation.  (Not part of the method: the
+ * article has no counterpart; this is a deployment variant of muon_step.)
+ *
+ * For callers that cannot call cudaMalloc -- code running inside a custom
+ * allocator or a memory-pool callback, or a process whose device memory is
+ * budgeted up front so that a new allocation could fail or deadlock.  The
+ * caller passes the same inputs and outputs as to muon_step (device
+ * pointers, updated in place); all scratch (bf16 iterates, Gram and
+ * polynomial matrices, norm partials, tensor-map table, status word) lives
+ * in one static device array of 64 MiB that every GPU loading this library
+ * holds until the process exits.
+ *   - Limit: one call takes at most 320 matrices over at most 16 padded
+ *     shapes, and their scratch (the muon_workspace_size layout) must fit in
+ *     64 MiB minus a 64 KiB table, e.g. one GPT-2-124M layer (4 x 768x768,
+ *     768x3072, 3072x768).  Larger requests return MUON_ERR_UNSUPPORTED with
+ *     the required size in muon_last_error(); nothing is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; each call clears what must start at zero.  Calls that overlap
+ *     on the GPU (e.g. on two streams) race on it: serialise them.
+ *   - The tensor-map table is copied from pageable host memory, so the call
+ *     may wait for earlier work on `stream` before returning.
+ *   - A bounded wait that runs out inside its kernels stops them cleanly; it
+ *     is recorded in the array's status word but not returned here (use
+ *     muon_step where device-side error reporting is needed).
+ */
+int muon_step_noalloc(float* const* params, const float* const* grads, float* const* momentum_bufs,
+                      const int64_t* shapes, int n, float lr, float mu, int ns_steps, void* stream);
+
 /* Bytes of device workspace a call with these shapes uses (0 on bad input). */
 size_t muon_workspace_size(const int64_t* shapes, int n);
 

@@ -18,7 +18,7 @@ import os
 import re
 
 __all__ = [
-    "step", "orthogonalize", "step_host", "workspace_size", "sync_status", "last_error", "release",
+    "step", "orthogonalize", "step_host", "step_noalloc", "workspace_size", "sync_status", "last_error", "release",
     "profile_enable", "profile_read", "launch_count", "debug_set", "lib", "MuonError", "KINDS",
     "NS_A", "NS_B", "NS_C", "NS_STEPS", "NS_EPS", "LIB_PATH", "header_functions",
 ]
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
     L.muon_step_ex.restype = ctypes.c_int
     L.muon_step_host.argtypes = step_args + [_P]
     L.muon_step_host.restype = ctypes.c_int
+    L.muon_step_noalloc.argtypes = step_args + [_P]
+    L.muon_step_noalloc.restype = ctypes.c_int
     L.muon_orthogonalize.argtypes = [_PP, _PP, _I64P, ctypes.c_int, ctypes.c_int, _P]
     L.muon_orthogonalize.restype = ctypes.c_int
     L.muon_workspace_size.argtypes = [_I64P, ctypes.c_int]
@@ -168,6 +170,18 @@ def step_host(params, grads, bufs, lr: float, mu: float, ns_steps: int = NS_STEP
     rc = lib().muon_step_host(_ptrs([t.data_ptr() for t in params]), _ptrs([t.data_ptr() for t in grads]),
                               _ptrs([t.data_ptr() for t in bufs]), _shapes([t.shape for t in params]),
                               len(params), float(lr), float(mu), int(ns_steps), _stream(stream))
+    _check(rc)
+
+
+def step_noalloc(params, grads, bufs, lr: float, mu: float, ns_steps: int = NS_STEPS, stream=None):
+    """muon_step for callers that cannot allocate device memory: the library's
+    scratch is a fixed 64 MiB static device array instead of cudaMalloc'd
+    workspace (see include/muon.h for the limits)."""
+    for name, ts in (("params", params), ("grads", grads), ("bufs", bufs)):
+        _check_tensors(name, ts)
+    rc = lib().muon_step_noalloc(_ptrs([t.data_ptr() for t in params]), _ptrs([t.data_ptr() for t in grads]),
+                                 _ptrs([t.data_ptr() for t in bufs]), _shapes([t.shape for t in params]),
+                                 len(params), float(lr), float(mu), int(ns_steps), _stream(stream))
     _check(rc)
 
 

@@ -748,3 +748,192 @@ int muon_debug_set(int flags, int64_t wait_limit_ns) {
 }
 
 }  // extern "C"
+
+// ======================================================= no-allocation step ===
+// muon_step_noalloc: the same Muon step for callers that must not allocate
+// device memory -- for example code running inside a custom allocator or a
+// memory-pool callback, or a host whose device memory is budgeted up front so
+// that any cudaMalloc could fail or deadlock.  Its scratch (bf16 iterates,
+// Gram / polynomial matrices, norm partials, scales, tensor-map table and a
+// status word) lives in one file-scope device array of fixed size that every
+// GPU loading this library holds until the process exits.
+namespace {
+
+constexpr size_t kNoAllocBytes = size_t(64) << 20;      // 64 MiB of static scratch per device
+constexpr size_t kNoAllocTableBytes = size_t(64) << 10; // tensor maps + status word at the end
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+// Device address of g_noalloc_scratch, looked up once per device (with that
+// device current) by the first muon_step_noalloc call on it.
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+int noalloc_setup(int dev, void** out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(MUON_ERR_DEVICE, "device index out of range");
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(MUON_ERR_CUDA, std::string("cudaGetSymbolAddress(static scratch): ") + cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MUON_OK;
+}
+
+int noalloc_launch(cudaStream_t stream, char* base, const Plan& plan, const StepIO& io, int sm_count) {
+  const Group& g = plan.groups[0];
+  const size_t table_off = kNoAllocBytes - kNoAllocTableBytes;
+  int* status = (int*)(base + kNoAllocBytes - 256);
+  CUtensorMap* tmaps = (CUtensorMap*)(base + table_off);
+  CUtensorMap* wmaps = tmaps + g.classes.size() * kTmapsPerClass;
+  float* scale = (float*)(base + g.off_scale);
+  const int nm = (int)g.mats.size();
+
+  // Everything that must start at zero: the norm arrival counters and the status word.
+  CUDA_TRY(cudaMemsetAsync(base, 0, kTicketBytes, stream));
+  CUDA_TRY(cudaMemsetAsync(status, 0, 256, stream));
+
+  // Tensor maps of this call (scratch buffers and the caller's outputs), copied
+  // from host memory into the table at the end of the scratch.
+  std::vector<CUtensorMap> host(g.classes.size() * kTmapsPerClass + g.mats.size());
+  std::memset(host.data(), 0, host.size() * sizeof(CUtensorMap));
+  int rc;
+  for (size_t ci = 0; ci < g.classes.size(); ++ci) {
+    const ClassDesc& cd = g.classes[ci];
+    const int batch = (int)cd.mats.size();
+    CUtensorMap* m = &host[ci * kTmapsPerClass];
+    if ((rc = encode_map(&m[kTmX0], base + cd.off_x0, cd.lp, cd.kp, batch, 64, 128))) return rc;
+    if ((rc = encode_map(&m[kTmX1], base + cd.off_x1, cd.lp, cd.kp, batch, 64, 128))) return rc;
+    if ((rc = encode_map(&m[kTmX0mn], base + cd.off_x0, cd.lp, cd.kp, batch, 64, 64))) return rc;
+    if ((rc = encode_map(&m[kTmX1mn], base + cd.off_x1, cd.lp, cd.kp, batch, 64, 64))) return rc;
+    if ((rc = encode_map(&m[kTmA], base + cd.off_a, cd.kp, cd.kp, batch, 64, 128))) return rc;
+    if ((rc = encode_map(&m[kTmB], base + cd.off_b, cd.kp, cd.kp, batch, 64, 128))) return rc;
+  }
+  CUtensorMap* hw = &host[g.classes.size() * kTmapsPerClass];
+  for (size_t i = 0; i < g.mats.size(); ++i) {
+    const MatDesc& d = g.mats[i];
+    if (d.n % 4 == 0 && aligned16(io.W[d.user]))
+      if ((rc = encode_wmap(&hw[i], (void*)io.W[d.user], d.m, d.n, d.trans))) return rc;
+  }
+  CUDA_TRY(cudaMemcpyAsync(tmaps, host.data(), host.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice, stream));
+
+  // prologue: momentum, norm partials, bf16 iterate
+  auto pa = std::make_unique<ProArgs>();
+  std::memset(pa.get(), 0, sizeof(ProArgs));
+  pa->nmats = nm;
+  pa->total_tiles = g.pro_tiles;
+  pa->mu = io.mu;
+  pa->eps = io.eps;
+  pa->nesterov = io.nesterov;
+  pa->has_buf = 1;
+  pa->partials = (float*)(base + g.off_partials);
+  pa->tickets = (unsigned*)(base + g.off_tickets);
+  pa->scale = scale;
+  auto ga = std::make_unique<GemmArgs>();
+  std::memset(ga.get(), 0, sizeof(GemmArgs));
+  auto aa = std::make_unique<ApplyArgs>();
+  std::memset(aa.get(), 0, sizeof(ApplyArgs));
+  for (const auto& cd : g.classes)
+    for (size_t b = 0; b < cd.mats.size(); ++b) {
+      const int gi = cd.mats[b];
+      const MatDesc& d = g.mats[gi];
+      ProMat& pm = pa->mats[gi];
+      pm.g = io.g[d.user];
+      pm.buf = io.buf[d.user];
+      pm.x = (__nv_bfloat16*)(base + cd.off_x0 + b * (size_t)cd.kp * cd.lp * 2);
+      pm.m = d.m; pm.n = d.n; pm.kp = d.kp; pm.lp = d.lp;
+      pm.trans = d.trans;
+      pm.vec = (d.n % 4 == 0) && aligned16(pm.g) && aligned16(pm.buf);
+      pm.tile_begin = g.pro_tile_begin[gi];
+      pm.tiles_c = d.lp / kProCols;
+      pm.tiles = (d.kp / kProRows) * pm.tiles_c;
+      OutMat o;
+      o.w = io.W[d.user];
+      o.m = d.m; o.n = d.n; o.trans = d.trans;
+      o.vec = (d.n % 4 == 0) && aligned16(o.w);
+      o.tma = o.vec;
+      ga->out[gi] = o;
+      aa->out[gi] = o;
+      aa->x[gi] = pm.x;
+      aa->lp[gi] = cd.lp;
+    }
+  prologue_kernel<<<g.pro_tiles, kProThreads, 0, stream>>>(*pa);
+  CUDA_TRY(cudaGetLastError());
+  g_launches.fetch_add(1);
+
+  if (io.ns_steps == 0) {
+    aa->scale = scale;
+    aa->lr = io.lr;
+    aa->assign = 0;
+    aa->nmats = nm;
+    apply_x0_kernel<<<dim3(64, nm), 256, 0, stream>>>(*aa);
+    CUDA_TRY(cudaGetLastError());
+    g_launches.fetch_add(1);
+    return MUON_OK;
+  }
+  ga->tmaps = tmaps;
+  ga->wmaps = wmaps;
+  ga->scale = scale;
+  ga->status = status;
+  ga->wait_limit_ns = 2000000000ull;
+  ga->nclasses = (int)g.classes.size();
+  ga->a = io.a; ga->b = io.b; ga->c = io.c; ga->lr = io.lr;
+  ga->assign = 0;
+  for (int it = 0; it < io.ns_steps; ++it) {
+    for (int mode = kModeGram; mode <= kModeUpdate; ++mode) {
+      const bool sym = mode != kModeUpdate;
+      const auto& cls = sym ? g.sym_cls : g.upd_cls;
+      for (size_t ci = 0; ci < cls.size(); ++ci) {
+        ga->cls[ci] = cls[ci];
+        if (mode == kModePoly) ga->cls[ci].kblocks = cls[ci].kp / kBK;
+      }
+      ga->total_tiles = sym ? g.sym_tiles : g.upd_tiles;
+      ga->mode = mode;
+      ga->x_in = it & 1;
+      ga->first = it == 0;
+      ga->final_apply = (mode == kModeUpdate) && (it == io.ns_steps - 1);
+      ga->debug_flags = 0;
+      const int grid = std::min(ga->total_tiles, sm_count);
+      ns_gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(*ga);
+      CUDA_TRY(cudaGetLastError());
+      g_launches.fetch_add(1);
+    }
+  }
+  return MUON_OK;
+}
+
+}  // namespace
+
+extern "C" int muon_step_noalloc(float* const* params, const float* const* grads, float* const* momentum_bufs,
+                                 const int64_t* shapes, int n, float lr, float mu, int ns_steps, void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int rc = validate_common(shapes, n, ns_steps);
+  if (rc) return rc;
+  if ((rc = validate_ptrs((const void* const*)params, n, "params"))) return rc;
+  if ((rc = validate_ptrs((const void* const*)grads, n, "grads"))) return rc;
+  if ((rc = validate_ptrs((const void* const*)momentum_bufs, n, "momentum_bufs"))) return rc;
+  Plan plan;
+  if ((rc = build_layout(shapes, n, plan))) return rc;
+  if (plan.groups.size() != 1)
+    return fail(MUON_ERR_UNSUPPORTED, "muon_step_noalloc takes at most " + std::to_string(kMaxMats) +
+                                          " matrices of at most " + std::to_string(kMaxClasses) +
+                                          " padded shapes per call");
+  const size_t table = (plan.groups[0].classes.size() * kTmapsPerClass + plan.groups[0].mats.size()) *
+                       sizeof(CUtensorMap);
+  if (plan.ws_bytes > kNoAllocBytes - kNoAllocTableBytes || table > kNoAllocTableBytes - 256)
+    return fail(MUON_ERR_UNSUPPORTED, "muon_step_noalloc: these shapes need " + std::to_string(plan.ws_bytes) +
+                                          " bytes of scratch; the static scratch holds " +
+                                          std::to_string(kNoAllocBytes - kNoAllocTableBytes) +
+                                          " (split the matrices over several calls)");
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if ((rc = device_setup(dev))) return rc;
+  void* base = nullptr;
+  if ((rc = noalloc_setup(dev, &base))) return rc;
+  int sm_count = 148;
+  CUDA_TRY(cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev));
+  StepIO io{params, grads, momentum_bufs, lr, mu, MUON_NS_A, MUON_NS_B, MUON_NS_C, MUON_NS_EPS, ns_steps, 1, 0};
+  return noalloc_launch((cudaStream_t)stream, (char*)base, plan, io, sm_count);
+}
