@@ -19,28 +19,36 @@
 
 namespace muon {
 
-constexpr int kBM = 128;            // tile rows (TMEM lanes)
-constexpr int kBN = 128;            // tile cols (TMEM fp32 columns per accumulator)
+constexpr int kTile = 256;          // pair tile: 256 x 256 outputs per CTA pair
+constexpr int kBM = 128;            // rows of the pair tile held by one CTA (TMEM lanes)
+constexpr int kBN = 256;            // columns of the pair tile (TMEM fp32 columns per accumulator)
+constexpr int kBNh = 128;           // B-operand rows / columns loaded by one CTA (half of kBN)
 constexpr int kBK = 64;             // K per pipeline stage: one 128-byte swizzle row of bf16
 constexpr int kUmmaK = 16;          // K of one tcgen05.mma kind::f16
-constexpr int kStages = 4;
-constexpr int kGemmThreads = 192;   // warp 0 TMA, warp 1 MMA (+TMEM alloc), warps 2..5 epilogue
+constexpr int kStages = 5;
+constexpr int kGemmThreads = 224;   // warp 0 TMA, warp 1 MMA (+TMEM alloc), warp 2 epilogue DMA, warps 3..6 epilogue math
 constexpr int kEpiThreads = 128;
-constexpr int kTmemCols = 256;      // two 128-column fp32 accumulators
+constexpr int kEpiWarp0 = 3;        // first epilogue math warp
+constexpr int kTmemCols = 512;      // two 256-column fp32 accumulators
 constexpr int kMaxClasses = 16;
 constexpr int kMaxMats = 320;
-constexpr int kTmapsPerClass = 6;
+constexpr int kTmapsPerClass = 8;
 constexpr int kPad = 128;           // padding granule of the short and long sides
 
-enum TmapSlot : int { kTmX0 = 0, kTmX1 = 1, kTmX0mn = 2, kTmX1mn = 3, kTmA = 4, kTmB = 5 };
+enum TmapSlot : int {
+  kTmX0 = 0, kTmX1 = 1,             // iterates, 64 x 128 boxes (K-major operand rows, epilogue slices, stores)
+  kTmX0mn = 2, kTmX1mn = 3,         // iterates, 64 x 64 boxes (MN-major operand of the update)
+  kTmA = 4, kTmB = 5,               // Gram / polynomial matrices, 64 x 128 boxes
+  kTmAmn = 6, kTmBmn = 7            // Gram / polynomial matrices, 64 x 64 boxes (mirrored stores)
+};
 enum GemmMode : int { kModeGram = 0, kModePoly = 1, kModeUpdate = 2 };
 
 constexpr uint32_t kStageABytes = kBM * kBK * 2;     // 16 KB
-constexpr uint32_t kStageBBytes = kBN * kBK * 2;     // 16 KB
+constexpr uint32_t kStageBBytes = kBNh * kBK * 2;    // 16 KB
 constexpr uint32_t kStageBytes = kStageABytes + kStageBBytes;
-constexpr uint32_t kTileBytes = kBM * kBN * 2;       // 32 KB bf16 output / epilogue input tile
-constexpr uint32_t kChunkBytes = kBM * 64 * 2;       // 16 KB: 128 rows x 64 cols (one TMA box)
-constexpr uint32_t kSmemDataBytes = kStages * kStageBytes + 2 * kTileBytes;
+constexpr uint32_t kSliceBytes = kBM * 64 * 2;       // 16 KB: 128 rows x 64 cols bf16 (one TMA box)
+constexpr uint32_t kChunkBytes = kSliceBytes;
+constexpr uint32_t kSmemDataBytes = kStages * kStageBytes + 4 * kSliceBytes;
 constexpr uint32_t kSmemCtrlBytes = 256;
 constexpr uint32_t kGemmSmemBytes = kSmemDataBytes + kSmemCtrlBytes + 1024;  // + alignment slack
 
@@ -49,8 +57,8 @@ struct GemmClass {
   int batch;          // matrices of this shape class
   int kp, lp;         // padded short side (rows of X) and long side (cols of X)
   int mat_first;      // first matrix of the class in group order
-  int tiles_m;        // kp / 128
-  int tiles_n;        // UPDATE: lp / 128; GRAM / POLY: tiles_m
+  int tiles_m;        // ceil(kp / 256)
+  int tiles_n;        // UPDATE: ceil(lp / 256); GRAM / POLY: tiles_m
   int tiles_per_mat;  // GRAM / POLY: tiles_m (tiles_m + 1) / 2; UPDATE: tiles_m * tiles_n
   int tile_begin;     // first tile of the class in this launch
   int kblocks;        // GRAM: lp / 64; POLY, UPDATE: kp / 64
@@ -293,93 +301,104 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& p, int t, bool 
 // box stored with the 128-byte swizzle (the pattern TMA writes / reads).
 __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t u) { return r * 128u + ((u ^ (r & 7u)) << 4); }
 
-// Read-modify-write of one 128 x 32 slice of the final result into W (or
-// O), staged in shared memory by the epilogue.  X row gi0 + r, col gj0 + c maps
-// to W[gi][gj] (X = W) or W[gj][gi] (X = W^T).  Each warp touches whole rows.
-__device__ __forceinline__ void store_w_slice(const OutMat& O, const float* S, int gi0, int gj0, int et, float lr,
-                                              int assign) {
-  // all loads of the slice are issued before any store (8 in flight per thread)
-  float4 o[8], w[8];
-  float* wp[8];
-  bool ok[8], full[8];
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    int row, col, sidx;
-    if (!O.trans) {
-      const int rr = it * 16 + (et >> 3), q = et & 7;
-      row = gi0 + rr; col = gj0 + 4 * q;
-      sidx = rr * 32 + ((q ^ (rr & 7)) << 2);
-      ok[it] = row < O.m && col < O.n;
-    } else {
-      const int c = it * 4 + (et >> 5), q = et & 31;
-      row = gj0 + c; col = gi0 + 4 * q;          // W[row][col..col+3]
-      sidx = c * kBM + 4 * q;
-      ok[it] = row < O.m && col < O.n;
+// Read-modify-write of this warp's 32 rows of a 128 x 32 slice of the final
+// result into W (or O), for outputs whose rows are not 16-byte aligned.  The
+// slice is staged in shared memory by the same warp (rows 32q..32q+31); X row
+// gi0 + r, col gj0 + c maps to W[gi][gj] (X = W) or W[gj][gi] (X = W^T).  Every
+// access pattern touches whole 128-byte rows of W.
+__device__ __forceinline__ void store_w_slice_warp(const OutMat& O, const float* S, int gi0, int gj0, int q,
+                                                   int lane, float lr, int assign) {
+  if (!O.trans) {
+#pragma unroll 2
+    for (int it = 0; it < 8; ++it) {
+      const int rr = q * 32 + it * 4 + (lane >> 3), qd = lane & 7;
+      const int gi = gi0 + rr, gj = gj0 + 4 * qd;
+      if (gi >= O.m || gj >= O.n) continue;
+      const float4 o = *reinterpret_cast<const float4*>(S + rr * 32 + ((qd ^ (rr & 7)) << 2));
+      float* wp = O.w + (size_t)gi * O.n + gj;
+      const float ov[4] = {o.x, o.y, o.z, o.w};
+      for (int e = 0; e < 4 && gj + e < O.n; ++e) wp[e] = assign ? ov[e] : wp[e] - lr * ov[e];
     }
-    full[it] = O.vec && col + 3 < O.n;
-    wp[it] = O.w + (size_t)row * O.n + col;
-    o[it] = *reinterpret_cast<const float4*>(S + sidx);
-    w[it] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (ok[it] && full[it] && !assign) w[it] = *reinterpret_cast<const float4*>(wp[it]);
-  }
-  const float sg = assign ? -1.f : lr;
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    if (!ok[it]) continue;
-    if (full[it]) {
-      float4 r4 = w[it];
-      r4.x -= sg * o[it].x; r4.y -= sg * o[it].y; r4.z -= sg * o[it].z; r4.w -= sg * o[it].w;
-      *reinterpret_cast<float4*>(wp[it]) = r4;
-    } else {
-      const float ov[4] = {o[it].x, o[it].y, o[it].z, o[it].w};
-      const int col = (int)((wp[it] - O.w) % O.n);
-      for (int e = 0; e < 4 && col + e < O.n; ++e) wp[it][e] = assign ? ov[e] : wp[it][e] - lr * ov[e];
+  } else {
+    const int wcol = gi0 + q * 32 + lane;           // W column = X row
+#pragma unroll 4
+    for (int c = 0; c < 32; ++c) {
+      const int wrow = gj0 + c;                      // W row = X column
+      if (wrow >= O.m || wcol >= O.n) continue;
+      const float o = S[c * kBM + q * 32 + lane];
+      float* wp = O.w + (size_t)wrow * O.n + wcol;
+      *wp = assign ? o : *wp - lr * o;
     }
   }
 }
 
 struct __align__(8) GemmCtrl {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t tmem_full[2];
-  uint64_t tmem_empty[2];
-  uint64_t dfull;
-  uint64_t dempty;
+  uint64_t full[kStages];     // even CTA: both CTAs' operand bytes of a stage have landed
+  uint64_t empty[kStages];    // the pair MMAs reading a stage are done (both CTAs)
+  uint64_t tmem_full[2];      // an accumulator is ready (both CTAs)
+  uint64_t tmem_empty[2];     // even CTA: all 8 epilogue math warps of the pair drained an accumulator
+  uint64_t in_full[2];        // DMA -> math: slice buffer set ready (input slice landed, or just free)
+  uint64_t out_full[2];       // math -> DMA: slice staged (and input slice consumed)
+  uint64_t stg_full[2];       // math -> DMA: fp32 result chunk staged (final update)
+  uint64_t stg_free[2];       // DMA -> math: fp32 staging buffer free again
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
+// One persistent launch per Newton-Schulz phase.  A cluster of two CTAs (one
+// per SM) computes 256 x 256 output tiles with tcgen05.mma.cta_group::2: each
+// CTA loads its 128 rows of A and its 128 rows (or columns) of B per stage, the
+// even CTA issues the MMAs over both CTAs' shared memory, and each CTA's TMEM
+// holds its 128 rows x 256 fp32 columns (two accumulators, double-buffered).
+// Roles per CTA: warp 0 TMA producer; warp 1 MMA issuer (even CTA) and TMEM
+// allocator; warp 2 epilogue DMA (loads the epilogue's input slices, issues the
+// TMA stores / add-reductions of its output slices and recycles their
+// buffers); warps 3..6 epilogue math (per 64-column slice: tcgen05.ld -> fp32
+// math -> bf16 -> 128B-swizzled smem).  The math warps hand slices to the DMA
+// warp through mbarriers and never wait on TMA latency themselves.
 __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ GemmArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  uint8_t* dtile = smem + kStages * kStageBytes;       // epilogue input tile / output staging
-  uint8_t* mtile = dtile + kTileBytes;                 // mirrored (transposed) output staging
-  GemmCtrl* ctl = reinterpret_cast<GemmCtrl*>(mtile + kTileBytes);
+  uint8_t* dbuf = smem + kStages * kStageBytes;        // 2 x 16 KB: epilogue input / output slices
+  uint8_t* mbuf = dbuf + 2 * kSliceBytes;              // 2 x 16 KB: mirrored output / fp32 staging
+  GemmCtrl* ctl = reinterpret_cast<GemmCtrl*>(mbuf + 2 * kSliceBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();             // 0: issues the MMAs of the pair
+  const int cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
   const bool sym = p.mode != kModeUpdate;
   const bool has_d = p.mode != kModeGram;
+  const bool final_w = p.mode == kModeUpdate && p.final_apply;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&ctl->tmem_full[s], 1); mbar_init(&ctl->tmem_empty[s], kEpiThreads); }
-    mbar_init(&ctl->dfull, 1);
-    mbar_init(&ctl->dempty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ctl->tmem_full[s], 1);
+      mbar_init(&ctl->tmem_empty[s], 8);
+      mbar_init(&ctl->in_full[s], 1);
+      mbar_init(&ctl->out_full[s], 4);
+      mbar_init(&ctl->stg_full[s], 4);
+      mbar_init(&ctl->stg_free[s], 1);
+    }
     mbar_init(&ctl->drain, 1);
     ctl->abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem_base, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();                                  // barriers of both CTAs initialised
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
-  WaitCtx wc{&ctl->abort_flag, p.status, p.wait_limit_ns};
+  WaitCtx wc{&ctl->abort_flag, p.status, p.wait_limit_ns, mapa_shared(&ctl->abort_flag, rank ^ 1u)};
+  bool aborted = false;
+  // tiles of this cluster and their 64-column slices, in processing order
+  const int my_tiles = cid < p.total_tiles ? (p.total_tiles - cid + ncl - 1) / ncl : 0;
+  const int my_slices = 4 * my_tiles;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -392,12 +411,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         }
       int stage = 0;
       uint32_t phase = 0;
-      int pending[kStages];            // parity of the last issued, not yet landed, fill (-1: none)
-      for (int s = 0; s < kStages; ++s) pending[s] = -1;
-      int dpending = -1;
       bool ok = true;
       int it = 0;
-      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x, ++it) {
+      for (int t = cid; t < p.total_tiles && ok; t += ncl, ++it) {
         const TileCoord tc = decode_tile(p, t, sym);
         const GemmClass& C = p.cls[tc.cls];
         const CUtensorMap* tA;
@@ -405,56 +421,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         if (p.mode == kModeGram) { tA = &p.tmaps[C.tmap_base + (p.x_in ? kTmX1 : kTmX0)]; tB = tA; }
         else if (p.mode == kModePoly) { tA = &p.tmaps[C.tmap_base + kTmA]; tB = tA; }
         else { tA = &p.tmaps[C.tmap_base + kTmB]; tB = &p.tmaps[C.tmap_base + (p.x_in ? kTmX1mn : kTmX0mn)]; }
+        const int arow = tc.tm * kTile + (int)rank * kBM;     // this CTA's A rows
+        const int bidx = tc.tn * kTile + (int)rank * kBNh;    // this CTA's B rows (or columns)
         for (int kb = 0; kb < C.kblocks; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, wc, kDevTimeoutEmpty)) { ok = false; break; }
           uint8_t* sa = stage_base + stage * kStageBytes;
           uint8_t* sb = sa + kStageABytes;
+          const uint32_t full_lead = mapa_shared(&ctl->full[stage], 0);
           const bool inject_skip = (p.debug_flags & 1) && it == 0 && kb == 0;
           if (!inject_skip) {
-            mbar_arrive_expect_tx(&ctl->full[stage], kStageBytes);
-            tma_load_3d(sa, tA, &ctl->full[stage], kb * kBK, tc.tm * kBM, tc.b);
+            if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], 2 * kStageBytes);
+            tma_load_3d_pair(sa, tA, full_lead, kb * kBK, arow, tc.b);
             if (p.mode == kModeUpdate) {
-              // B operand = X rows [kb*64, +64) x cols [tn*128, +128), MN-major: two 64-col boxes
-              tma_load_3d(sb, tB, &ctl->full[stage], tc.tn * kBN, kb * kBK, tc.b);
-              tma_load_3d(sb + kStageBBytes / 2, tB, &ctl->full[stage], tc.tn * kBN + 64, kb * kBK, tc.b);
+              // B = X rows [kb*64, +64) x this CTA's 128 columns, MN-major: two 64-col boxes
+              tma_load_3d_pair(sb, tB, full_lead, bidx, kb * kBK, tc.b);
+              tma_load_3d_pair(sb + kStageBBytes / 2, tB, full_lead, bidx + 64, kb * kBK, tc.b);
             } else {
-              tma_load_3d(sb, tB, &ctl->full[stage], kb * kBK, tc.tn * kBN, tc.b);
+              tma_load_3d_pair(sb, tB, full_lead, kb * kBK, bidx, tc.b);
             }
-            pending[stage] = (int)phase;
           }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
-        if (has_d) {
-          if (!mbar_wait(&ctl->dempty, (uint32_t)((it & 1) ^ 1), wc, kDevTimeoutEpi)) { ok = false; break; }
-          const CUtensorMap* tD = (p.mode == kModePoly) ? &p.tmaps[C.tmap_base + kTmA]
-                                                        : &p.tmaps[C.tmap_base + (p.x_in ? kTmX1 : kTmX0)];
-          mbar_arrive_expect_tx(&ctl->dfull, kTileBytes);
-          tma_load_3d(dtile, tD, &ctl->dfull, tc.tn * kBN, tc.tm * kBM, tc.b);
-          tma_load_3d(dtile + kChunkBytes, tD, &ctl->dfull, tc.tn * kBN + 64, tc.tm * kBM, tc.b);
-          dpending = it & 1;
-        }
       }
-      // Never leave the CTA with copies in flight into its shared memory.
-      for (int s = 0; s < kStages; ++s)
-        if (pending[s] >= 0) mbar_wait(&ctl->full[s], (uint32_t)pending[s], wc, kDevTimeoutDrain);
-      if (dpending >= 0) mbar_wait(&ctl->dfull, (uint32_t)dpending, wc, kDevTimeoutDrain);
+      aborted = !ok;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0, p.mode == kModeUpdate ? 1 : 0);
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN, 0, p.mode == kModeUpdate ? 1 : 0);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
       bool issued_any = false;
-      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x, ++it) {
+      for (int t = cid; t < p.total_tiles && ok; t += ncl, ++it) {
         const TileCoord tc = decode_tile(p, t, sym);
         const GemmClass& C = p.cls[tc.cls];
         const int acc = it & 1;
         const uint32_t acc_phase = (uint32_t)((it >> 1) & 1);
-        if (!mbar_wait(&ctl->tmem_empty[acc], acc_phase ^ 1u, wc, kDevTimeoutAccum)) { ok = false; break; }
+        if (!mbar_wait_cluster(&ctl->tmem_empty[acc], acc_phase ^ 1u, wc, kDevTimeoutAccum)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
         for (int kb = 0; kb < C.kblocks; ++kb) {
@@ -468,192 +473,258 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             const uint64_t bdesc = (p.mode == kModeUpdate)
                                        ? smem_desc_sw128(sb + kk * (kUmmaK * 128), kStageBBytes / 2, 1024)
                                        : smem_desc_sw128(sb + kk * (kUmmaK * 2), 16, 1024);
-            tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           issued_any = true;
-          tc_commit(&ctl->empty[stage]);
+          tc_commit_pair(mapa_shared(&ctl->empty[stage], 0));
+          tc_commit_pair(mapa_shared(&ctl->empty[stage], 1));
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tc_commit(&ctl->tmem_full[acc]);
+        tc_commit_pair(mapa_shared(&ctl->tmem_full[acc], 0));
+        tc_commit_pair(mapa_shared(&ctl->tmem_full[acc], 1));
       }
       if (issued_any) {                 // all MMAs done before TMEM is released
-        tc_commit(&ctl->drain);
+        tc_commit_pair(mapa_shared(&ctl->drain, 0));
         mbar_wait(&ctl->drain, 0, wc, kDevTimeoutDrain);
       }
+      aborted = !ok;
     }
-  } else {
-    // --------------------------------------------------------- epilogue
-    const int et = threadIdx.x - 64;              // 0..127
-    const int q = warp & 3;                       // TMEM lane quarter this warp may access
-    const int r = q * 32 + lane;                  // tile row owned by this thread
-    const float alpha_first = 1.0f;
-    if (et == 0) {
+  } else if (warp == 2) {
+    // ----------------------------------------------------- epilogue DMA
+    if (lane == 0) {
       for (int c = 0; c < p.nclasses; ++c)
         for (int k = 0; k < kTmapsPerClass; ++k) tmap_acquire(&p.tmaps[p.cls[c].tmap_base + k]);
-      if (p.mode == kModeUpdate && p.final_apply)
+      if (final_w)
         for (int c = 0; c < p.nclasses; ++c)
           for (int b = 0; b < p.cls[c].batch; ++b)
             if (p.out[p.cls[c].mat_first + b].tma) tmap_acquire(&p.wmaps[p.cls[c].mat_first + b]);
+      int pend[2] = {-1, -1};                      // parity of an input load not yet seen landed
+      // Make slice gs's buffer set ready: load its input slice, or just hand it over.
+      auto prepare = [&](int gs) {
+        if (gs >= my_slices) return;
+        const int b = gs & 1;
+        if (has_d) {
+          const int t = cid + (gs >> 2) * ncl, h = gs & 3;
+          const TileCoord tc = decode_tile(p, t, sym);
+          const GemmClass& C = p.cls[tc.cls];
+          const CUtensorMap* tD = (p.mode == kModePoly) ? &p.tmaps[C.tmap_base + kTmA]
+                                                        : &p.tmaps[C.tmap_base + (p.x_in ? kTmX1 : kTmX0)];
+          mbar_arrive_expect_tx(&ctl->in_full[b], kSliceBytes);
+          tma_load_3d(dbuf + b * kSliceBytes, tD, &ctl->in_full[b], tc.tn * kTile + 64 * h,
+                      tc.tm * kTile + (int)rank * kBM, tc.b);
+          pend[b] = (gs >> 1) & 1;
+        } else {
+          mbar_arrive(&ctl->in_full[b]);
+        }
+      };
+      prepare(0);
+      prepare(1);
+      bool ok = true;
+      int gc = 0;                                  // fp32 chunk counter (final update)
+      for (int gs = 0; gs < my_slices && ok; ++gs) {
+        const int b = gs & 1;
+        const uint32_t ph = (uint32_t)((gs >> 1) & 1);
+        const int t = cid + (gs >> 2) * ncl, h = gs & 3;
+        const TileCoord tc = decode_tile(p, t, sym);
+        const GemmClass& C = p.cls[tc.cls];
+        const int row0 = tc.tm * kTile + (int)rank * kBM;
+        if (final_w) {
+          const int mat = C.mat_first + tc.b;
+          const OutMat& O = p.out[mat];
+          for (int sub = 0; sub < 2 && ok; ++sub, ++gc) {
+            const int s = gc & 1;
+            if (!mbar_wait(&ctl->stg_full[s], (uint32_t)((gc >> 1) & 1), wc, kDevTimeoutEpi)) { ok = false; break; }
+            if (O.tma) {
+              const uint8_t* S = mbuf + s * kSliceBytes;
+              const CUtensorMap* wm = &p.wmaps[mat];
+              const int gj0 = tc.tn * kTile + 64 * h + 32 * sub;
+              if (!O.trans) {
+                if (row0 < O.m && gj0 < O.n) {
+                  if (p.assign) tma_store_2d(wm, S, gj0, row0); else tma_reduce_add_2d(wm, S, gj0, row0);
+                }
+              } else if (gj0 < O.m) {
+                for (int hq = 0; hq < 4; ++hq) {
+                  if (row0 + 32 * hq >= O.n) continue;
+                  if (p.assign) tma_store_2d(wm, S + hq * 4096, row0 + 32 * hq, gj0);
+                  else tma_reduce_add_2d(wm, S + hq * 4096, row0 + 32 * hq, gj0);
+                }
+              }
+              tma_store_commit();
+              tma_store_wait_read0();
+            }
+            mbar_arrive(&ctl->stg_free[s]);
+          }
+          if (!ok) break;
+        }
+        if (!mbar_wait(&ctl->out_full[b], ph, wc, kDevTimeoutEpi)) { ok = false; break; }
+        if (has_d) pend[b] = -1;                   // the math warps saw this slice's input land
+        if (!final_w) {
+          const CUtensorMap* tO;
+          const CUtensorMap* tM;
+          if (p.mode == kModeGram) { tO = &p.tmaps[C.tmap_base + kTmA]; tM = &p.tmaps[C.tmap_base + kTmAmn]; }
+          else if (p.mode == kModePoly) { tO = &p.tmaps[C.tmap_base + kTmB]; tM = &p.tmaps[C.tmap_base + kTmBmn]; }
+          else { tO = &p.tmaps[C.tmap_base + (p.x_in ? kTmX0 : kTmX1)]; tM = tO; }
+          // stores start inside the tensor only (a pair tile can overhang the
+          // 128-padded edge by half; the overhang is never stored)
+          const int ocols = sym ? C.kp : C.lp;
+          const int x0 = tc.tn * kTile + 64 * h;
+          const bool mirror = sym && tc.tm != tc.tn;
+          if (row0 < C.kp && x0 < ocols) tma_store_3d(tO, dbuf + b * kSliceBytes, x0, row0, tc.b);
+          if (mirror && x0 < C.kp) {
+            if (row0 < C.kp) tma_store_3d(tM, mbuf + b * kSliceBytes, row0, x0, tc.b);
+            if (row0 + 64 < C.kp) tma_store_3d(tM, mbuf + b * kSliceBytes + kSliceBytes / 2, row0 + 64, x0, tc.b);
+          }
+          tma_store_commit();
+          tma_store_wait_read0();                  // buffers b readable again
+        }
+        prepare(gs + 2);
+      }
+      tma_store_wait_all0();
+      for (int b = 0; b < 2; ++b)
+        if (pend[b] >= 0) mbar_wait(&ctl->in_full[b], (uint32_t)pend[b], wc, kDevTimeoutDrain);
+      aborted = !ok;
     }
-    int it = 0;
+  } else {
+    // ---------------------------------------------------- epilogue math
+    const int q = warp & 3;                       // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;                  // tile row owned by this thread
+    int it = 0, gs = 0, gc = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
+    for (int t = cid; t < p.total_tiles && ok; t += ncl, ++it) {
       const TileCoord tc = decode_tile(p, t, sym);
       const GemmClass& C = p.cls[tc.cls];
       const int mat = C.mat_first + tc.b;
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)((it >> 1) & 1);
-      if (ok) ok = mbar_wait(&ctl->tmem_full[acc], acc_phase, wc, kDevTimeoutAccum);
+      ok = __all_sync(0xffffffffu, mbar_wait(&ctl->tmem_full[acc], acc_phase, wc, kDevTimeoutAccum));
+      if (!ok) break;
       tc_fence_after();
-      if (ok && has_d) ok = mbar_wait(&ctl->dfull, (uint32_t)(it & 1), wc, kDevTimeoutEpi);
-      // one outcome for all 128 epilogue threads: the branch below holds named
-      // barriers and warp-collective tcgen05.ld
-      ok = named_bar_and(1, kEpiThreads, ok);
-      const float s = p.first ? p.scale[mat] : alpha_first;
+      const float s = p.first ? p.scale[mat] : 1.0f;
       const bool mirror = sym && tc.tm != tc.tn;
-      const bool final_w = p.mode == kModeUpdate && p.final_apply;
-      if (ok) {
-        const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
+      const int row0 = tc.tm * kTile + (int)rank * kBM;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
 #pragma unroll 1
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          float v[32];
-          tmem_ld_32x32b_x32(tbase + (uint32_t)(cc * 32), v);
-          const int h = cc >> 1;                          // 64-column chunk
-          uint8_t* drow = dtile + h * kChunkBytes;
-          if (p.mode == kModeGram) {
-            const float alpha = s * s;
+      for (int h = 0; h < 4 && ok; ++h, ++gs) {
+        const int b = gs & 1;
+        uint8_t* dslice = dbuf + b * kSliceBytes;
+        uint8_t* mslice = mbuf + b * kSliceBytes;
+        ok = __all_sync(0xffffffffu, mbar_wait(&ctl->in_full[b], (uint32_t)((gs >> 1) & 1), wc, kDevTimeoutEpi));
+        if (!ok) break;
+        float v[64];
+        tmem_ld_32x32b_x64(tbase + (uint32_t)(h * 64), v);
+        if (h == 3) {                               // accumulator fully read: hand it back to the MMA
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(mapa_shared(&ctl->tmem_empty[acc], 0));
+        }
+        if (p.mode == kModeGram) {
+          const float alpha = s * s;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= alpha;
-          } else {
-            // epilogue input (A for POLY, X for UPDATE): 4 units of 8 bf16
-            const float wd = (p.mode == kModePoly) ? p.b : p.a * s;
-            const float wa = (p.mode == kModePoly) ? p.c : s;
+          for (int i = 0; i < 64; ++i) v[i] *= alpha;
+        } else {
+          const float wd = (p.mode == kModePoly) ? p.b : p.a * s;
+          const float wa = (p.mode == kModePoly) ? p.c : s;
 #pragma unroll
-            for (int uu = 0; uu < 4; ++uu) {
-              const uint32_t u = (uint32_t)((cc & 1) * 4 + uu);
-              uint4 raw = *reinterpret_cast<const uint4*>(drow + sw128_off((uint32_t)r, u));
-              const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&raw);
+          for (int u = 0; u < 8; ++u) {
+            uint4 raw = *reinterpret_cast<const uint4*>(dslice + sw128_off((uint32_t)r, (uint32_t)u));
+            const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                float2 f = __bfloat1622float2(hv[e]);
-                v[uu * 8 + 2 * e] = fmaf(wa, v[uu * 8 + 2 * e], wd * f.x);
-                v[uu * 8 + 2 * e + 1] = fmaf(wa, v[uu * 8 + 2 * e + 1], wd * f.y);
-              }
+            for (int e = 0; e < 4; ++e) {
+              float2 f = __bfloat1622float2(hv[e]);
+              v[u * 8 + 2 * e] = fmaf(wa, v[u * 8 + 2 * e], wd * f.x);
+              v[u * 8 + 2 * e + 1] = fmaf(wa, v[u * 8 + 2 * e + 1], wd * f.y);
             }
           }
-          if (final_w && p.out[mat].tma) {
-            // -lr*O (or O) for a 128 x 32 slice, staged 128-byte swizzled; TMA adds
-            // it to W in L2 (or stores it), so W never passes through the SM.
-            const OutMat& O = p.out[mat];
-            const float sg = p.assign ? 1.f : -p.lr;
-            uint8_t* S = mtile + (cc & 1) * kChunkBytes;
-            if (!O.trans) {
+        }
+        if (final_w) {
+          const OutMat& O = p.out[mat];
 #pragma unroll
-              for (int j = 0; j < 8; ++j)
-                *reinterpret_cast<float4*>(S + sw128_off((uint32_t)r, (uint32_t)j)) =
-                    make_float4(sg * v[4 * j], sg * v[4 * j + 1], sg * v[4 * j + 2], sg * v[4 * j + 3]);
-            } else {
-              // box h = r / 32 holds W rows gj0..gj0+31 x W cols gi0+32h..+31
-              uint8_t* Sh = S + (r >> 5) * 4096;
-              const int rr = r & 31;
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                *reinterpret_cast<float*>(Sh + sw128_off((uint32_t)i, (uint32_t)(rr >> 2)) + (rr & 3) * 4) =
-                    sg * v[i];
-            }
-            fence_async_shared();
-            named_bar_sync(1, kEpiThreads);
-            if (et == 0) {
-              const CUtensorMap* wm = &p.wmaps[mat];
-              const int gi0 = tc.tm * kBM, gj0 = tc.tn * kBN + cc * 32;
+          for (int sub = 0; sub < 2; ++sub, ++gc) {
+            const int sidx = gc & 1;
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(&ctl->stg_free[sidx], (uint32_t)(((gc >> 1) & 1) ^ 1), wc, kDevTimeoutEpi));
+            if (!ok) break;
+            uint8_t* S = mbuf + sidx * kSliceBytes;
+            const float* vv = v + 32 * sub;
+            if (O.tma) {
+              // -lr*O (or O), 128-byte swizzled; the DMA warp adds it to W in L2
+              const float sg = p.assign ? 1.f : -p.lr;
               if (!O.trans) {
-                if (p.assign) tma_store_2d(wm, S, gj0, gi0); else tma_reduce_add_2d(wm, S, gj0, gi0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  *reinterpret_cast<float4*>(S + sw128_off((uint32_t)r, (uint32_t)j)) =
+                      make_float4(sg * vv[4 * j], sg * vv[4 * j + 1], sg * vv[4 * j + 2], sg * vv[4 * j + 3]);
+              } else {
+                // box r / 32 holds W rows gj0..gj0+31 x W cols row0+32*(r/32)..+31
+                uint8_t* Sh = S + (r >> 5) * 4096;
+                const int rr = r & 31;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  *reinterpret_cast<float*>(Sh + sw128_off((uint32_t)i, (uint32_t)(rr >> 2)) + (rr & 3) * 4) =
+                      sg * vv[i];
+              }
+              fence_async_shared();
+            } else {
+              // rows not 16-byte aligned: the math warps update W themselves,
+              // in whole 128-byte rows through the staging buffer
+              float* Sf = reinterpret_cast<float*>(S);
+              if (!O.trans) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  *reinterpret_cast<float4*>(Sf + r * 32 + ((j ^ (r & 7)) << 2)) =
+                      make_float4(vv[4 * j], vv[4 * j + 1], vv[4 * j + 2], vv[4 * j + 3]);
               } else {
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                  if (p.assign) tma_store_2d(wm, S + h * 4096, gi0 + 32 * h, gj0);
-                  else tma_reduce_add_2d(wm, S + h * 4096, gi0 + 32 * h, gj0);
-                }
+                for (int i = 0; i < 32; ++i) Sf[i * kBM + r] = vv[i];
               }
-              tma_store_commit();
-              tma_store_wait_read1();          // the other staging buffer is free again
+              __syncwarp();
+              store_w_slice_warp(O, Sf, row0, tc.tn * kTile + 64 * h + 32 * sub, q, lane, p.lr, p.assign);
             }
-            named_bar_sync(1, kEpiThreads);
-          } else if (final_w) {
-            // fp32 result slice (128 rows x 32 cols) through shared memory so that
-            // W is read and written in whole 128-byte rows.
-            const OutMat& O = p.out[mat];
-            float* S = reinterpret_cast<float*>(mtile + (cc & 1) * (kChunkBytes));
-            if (!O.trans) {
-              // S[row][quad ^ (row & 7)]: 8 float4 per row
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->stg_full[sidx]);
+          }
+          if (!ok) break;
+        } else {
+          // bf16 output (in place over the input slice), 128-byte swizzled for the TMA store
 #pragma unroll
-              for (int j = 0; j < 8; ++j)
-                *reinterpret_cast<float4*>(S + r * 32 + ((j ^ (r & 7)) << 2)) =
-                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            } else {
-              // S[col][row]: row c of S is a 128-float row of W
+          for (int u = 0; u < 8; ++u) {
+            uint4 o;
+            o.x = pack_bf16x2(v[u * 8 + 0], v[u * 8 + 1]);
+            o.y = pack_bf16x2(v[u * 8 + 2], v[u * 8 + 3]);
+            o.z = pack_bf16x2(v[u * 8 + 4], v[u * 8 + 5]);
+            o.w = pack_bf16x2(v[u * 8 + 6], v[u * 8 + 7]);
+            *reinterpret_cast<uint4*>(dslice + sw128_off((uint32_t)r, (uint32_t)u)) = o;
+          }
+          if (mirror) {
+            // transposed copy: mirror box (r / 64) holds rows c (64 columns of
+            // this slice) x columns r (64 rows of this CTA)
+            uint8_t* mbox = mslice + (r >> 6) * (kSliceBytes / 2);
+            const uint32_t mu = (uint32_t)((r & 63) >> 3);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) S[i * kBM + r] = v[i];
-            }
-            named_bar_sync(1, kEpiThreads);
-            store_w_slice(O, S, tc.tm * kBM, tc.tn * kBN + cc * 32, et, p.lr, p.assign);
-          } else {
-            // bf16 output tile (in place over the input tile), 128-byte swizzled for the TMA store
-#pragma unroll
-            for (int uu = 0; uu < 4; ++uu) {
-              const uint32_t u = (uint32_t)((cc & 1) * 4 + uu);
-              uint4 o;
-              o.x = pack_bf16x2(v[uu * 8 + 0], v[uu * 8 + 1]);
-              o.y = pack_bf16x2(v[uu * 8 + 2], v[uu * 8 + 3]);
-              o.z = pack_bf16x2(v[uu * 8 + 4], v[uu * 8 + 5]);
-              o.w = pack_bf16x2(v[uu * 8 + 6], v[uu * 8 + 7]);
-              *reinterpret_cast<uint4*>(drow + sw128_off((uint32_t)r, u)) = o;
-            }
-            if (mirror) {
-              // transposed copy: row c of the mirror tile holds column c of this tile
-              uint8_t* mchunk = mtile + (r >> 6) * kChunkBytes;
-              const uint32_t mu = (uint32_t)((r & 63) >> 3);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const uint32_t crow = (uint32_t)(cc * 32 + i);
-                __nv_bfloat16* dst =
-                    reinterpret_cast<__nv_bfloat16*>(mchunk + sw128_off(crow, mu)) + (r & 7);
-                *dst = __float2bfloat16_rn(v[i]);
-              }
+            for (int i = 0; i < 64; ++i) {
+              __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(mbox + sw128_off((uint32_t)i, mu)) + (r & 7);
+              *dst = __float2bfloat16_rn(v[i]);
             }
           }
+          fence_async_shared();
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->out_full[b]);
       }
-      tc_fence_before();
-      mbar_arrive(&ctl->tmem_empty[acc]);
-      fence_async_shared();
-      named_bar_sync(1, kEpiThreads);
-      if (et == 0 && ok && !final_w) {
-        const CUtensorMap* tO;
-        if (p.mode == kModeGram) tO = &p.tmaps[C.tmap_base + kTmA];
-        else if (p.mode == kModePoly) tO = &p.tmaps[C.tmap_base + kTmB];
-        else tO = &p.tmaps[C.tmap_base + (p.x_in ? kTmX0 : kTmX1)];
-        tma_store_3d(tO, dtile, tc.tn * kBN, tc.tm * kBM, tc.b);
-        tma_store_3d(tO, dtile + kChunkBytes, tc.tn * kBN + 64, tc.tm * kBM, tc.b);
-        if (mirror) {
-          tma_store_3d(tO, mtile, tc.tm * kBM, tc.tn * kBN, tc.b);
-          tma_store_3d(tO, mtile + kChunkBytes, tc.tm * kBM + 64, tc.tn * kBN, tc.b);
-        }
-        tma_store_commit();
-        tma_store_wait_read0();
-      }
-      named_bar_sync(1, kEpiThreads);
-      if (et == 0 && has_d) mbar_arrive(&ctl->dempty);
     }
-    if (et == 0) tma_store_wait_all0();
+    aborted = !ok;
   }
 
-  __syncthreads();
+  // On the abort path, give copies that a CTA issued towards its shared memory
+  // time to land before either CTA of the pair leaves (bounded).
+  if (aborted || *reinterpret_cast<volatile int*>(&ctl->abort_flag)) sleep_ns_bounded(200000);
+  tc_fence_before();
+  cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 

@@ -184,9 +184,9 @@ int build_layout(const int64_t* shapes, int n, Plan& plan) {
       s.batch = u.batch = (int)c.mats.size();
       s.kp = u.kp = c.kp; s.lp = u.lp = c.lp;
       s.mat_first = u.mat_first = first;
-      s.tiles_m = u.tiles_m = c.kp / kBM;
+      s.tiles_m = u.tiles_m = (c.kp + kTile - 1) / kTile;
       s.tiles_n = s.tiles_m;
-      u.tiles_n = c.lp / kBN;
+      u.tiles_n = (c.lp + kTile - 1) / kTile;
       s.tiles_per_mat = s.tiles_m * (s.tiles_m + 1) / 2;
       u.tiles_per_mat = u.tiles_m * u.tiles_n;
       s.tile_begin = sym; u.tile_begin = upd;
@@ -226,6 +226,39 @@ int encode_map(CUtensorMap* map, void* base, int cols, int rows, int batch, int 
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
   return MUON_OK;
+}
+
+// The 8 tensor maps of one shape class (see TmapSlot) over its buffers at `base`.
+int encode_class_maps(CUtensorMap* m, char* base, const ClassDesc& cd) {
+  const int batch = (int)cd.mats.size();
+  int rc;
+  if ((rc = encode_map(&m[kTmX0], base + cd.off_x0, cd.lp, cd.kp, batch, 64, 128))) return rc;
+  if ((rc = encode_map(&m[kTmX1], base + cd.off_x1, cd.lp, cd.kp, batch, 64, 128))) return rc;
+  if ((rc = encode_map(&m[kTmX0mn], base + cd.off_x0, cd.lp, cd.kp, batch, 64, 64))) return rc;
+  if ((rc = encode_map(&m[kTmX1mn], base + cd.off_x1, cd.lp, cd.kp, batch, 64, 64))) return rc;
+  if ((rc = encode_map(&m[kTmA], base + cd.off_a, cd.kp, cd.kp, batch, 64, 128))) return rc;
+  if ((rc = encode_map(&m[kTmB], base + cd.off_b, cd.kp, cd.kp, batch, 64, 128))) return rc;
+  if ((rc = encode_map(&m[kTmAmn], base + cd.off_a, cd.kp, cd.kp, batch, 64, 64))) return rc;
+  if ((rc = encode_map(&m[kTmBmn], base + cd.off_b, cd.kp, cd.kp, batch, 64, 64))) return rc;
+  return MUON_OK;
+}
+
+// One NS-phase launch: persistent clusters of two CTAs (one CTA per SM).
+cudaError_t launch_gemm(cudaStream_t stream, const GemmArgs& args, int sm_count) {
+  const int pairs = std::max(1, std::min(args.total_tiles, sm_count / 2));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = kGemmSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, ns_gemm_kernel, args);
 }
 
 // W (m x n fp32, row-major, n % 4 == 0, 16-byte aligned) as a 2-D tensor map
@@ -337,15 +370,7 @@ int get_plan(Ctx& c, const int64_t* shapes, int n, Plan** out) {
   for (auto& g : p->groups) {
     std::vector<CUtensorMap> maps(g.classes.size() * kTmapsPerClass);
     for (size_t ci = 0; ci < g.classes.size(); ++ci) {
-      const ClassDesc& cd = g.classes[ci];
-      const int batch = (int)cd.mats.size();
-      CUtensorMap* m = &maps[ci * kTmapsPerClass];
-      if ((rc = encode_map(&m[kTmX0], base + cd.off_x0, cd.lp, cd.kp, batch, 64, 128))) return rc;
-      if ((rc = encode_map(&m[kTmX1], base + cd.off_x1, cd.lp, cd.kp, batch, 64, 128))) return rc;
-      if ((rc = encode_map(&m[kTmX0mn], base + cd.off_x0, cd.lp, cd.kp, batch, 64, 64))) return rc;
-      if ((rc = encode_map(&m[kTmX1mn], base + cd.off_x1, cd.lp, cd.kp, batch, 64, 64))) return rc;
-      if ((rc = encode_map(&m[kTmA], base + cd.off_a, cd.kp, cd.kp, batch, 64, 128))) return rc;
-      if ((rc = encode_map(&m[kTmB], base + cd.off_b, cd.kp, cd.kp, batch, 64, 128))) return rc;
+      if ((rc = encode_class_maps(&maps[ci * kTmapsPerClass], base, g.classes[ci]))) return rc;
     }
     CUDA_TRY(cudaMemcpy((char*)p->tmaps + g.off_tmaps, maps.data(), maps.size() * sizeof(CUtensorMap),
                         cudaMemcpyHostToDevice));
@@ -546,13 +571,10 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
       ga->final_apply = (mode == kModeUpdate) && (it == io.ns_steps - 1);
       ga->debug_flags = 0;
       if (g_debug_flags & 1) { ga->debug_flags = 1; g_debug_flags &= ~1; }
-      const int grid = std::min(ga->total_tiles, c.sm_count);
       const int kind = mode == kModeGram ? MUON_KIND_GRAM
                        : mode == kModePoly ? MUON_KIND_POLY
                        : (ga->final_apply ? MUON_KIND_UPDATE_APPLY : MUON_KIND_UPDATE);
-      int rc = launch(c, kind, [&] {
-        ns_gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, c.stream>>>(*ga);
-      });
+      int rc = launch(c, kind, [&] { launch_gemm(c.stream, *ga, c.sm_count); });
       if (rc) return rc;
     }
   }
@@ -801,15 +823,7 @@ int noalloc_launch(cudaStream_t stream, char* base, const Plan& plan, const Step
   std::memset(host.data(), 0, host.size() * sizeof(CUtensorMap));
   int rc;
   for (size_t ci = 0; ci < g.classes.size(); ++ci) {
-    const ClassDesc& cd = g.classes[ci];
-    const int batch = (int)cd.mats.size();
-    CUtensorMap* m = &host[ci * kTmapsPerClass];
-    if ((rc = encode_map(&m[kTmX0], base + cd.off_x0, cd.lp, cd.kp, batch, 64, 128))) return rc;
-    if ((rc = encode_map(&m[kTmX1], base + cd.off_x1, cd.lp, cd.kp, batch, 64, 128))) return rc;
-    if ((rc = encode_map(&m[kTmX0mn], base + cd.off_x0, cd.lp, cd.kp, batch, 64, 64))) return rc;
-    if ((rc = encode_map(&m[kTmX1mn], base + cd.off_x1, cd.lp, cd.kp, batch, 64, 64))) return rc;
-    if ((rc = encode_map(&m[kTmA], base + cd.off_a, cd.kp, cd.kp, batch, 64, 128))) return rc;
-    if ((rc = encode_map(&m[kTmB], base + cd.off_b, cd.kp, cd.kp, batch, 64, 128))) return rc;
+    if ((rc = encode_class_maps(&host[ci * kTmapsPerClass], base, g.classes[ci]))) return rc;
   }
   CUtensorMap* hw = &host[g.classes.size() * kTmapsPerClass];
   for (size_t i = 0; i < g.mats.size(); ++i) {
@@ -895,9 +909,7 @@ int noalloc_launch(cudaStream_t stream, char* base, const Plan& plan, const Step
       ga->first = it == 0;
       ga->final_apply = (mode == kModeUpdate) && (it == io.ns_steps - 1);
       ga->debug_flags = 0;
-      const int grid = std::min(ga->total_tiles, sm_count);
-      ns_gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(*ga);
-      CUDA_TRY(cudaGetLastError());
+      CUDA_TRY(launch_gemm(stream, *ga, sm_count));
       g_launches.fetch_add(1);
     }
   }
