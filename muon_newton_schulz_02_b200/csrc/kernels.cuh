@@ -337,8 +337,8 @@ struct __align__(8) GemmCtrl {
   uint64_t empty[kStages];    // the pair MMAs reading a stage are done (both CTAs)
   uint64_t tmem_full[2];      // an accumulator is ready (both CTAs)
   uint64_t tmem_empty[2];     // even CTA: all 8 epilogue math warps of the pair drained an accumulator
-  uint64_t in_full[2];        // DMA -> math: slice buffer set ready (input slice landed, or just free)
-  uint64_t out_full[2];       // math -> DMA: slice staged (and input slice consumed)
+  uint64_t in_full[4];        // DMA -> math: slice buffer set ready (input slice landed, or just free)
+  uint64_t out_full[4];       // math -> DMA: slice staged (and input slice consumed)
   uint64_t stg_full[2];       // math -> DMA: fp32 result chunk staged (final update)
   uint64_t stg_free[2];       // DMA -> math: fp32 staging buffer free again
   uint64_t drain;
@@ -357,6 +357,7 @@ struct __align__(8) GemmCtrl {
 // buffers); warps 3..6 epilogue math (per 64-column slice: tcgen05.ld -> fp32
 // math -> bf16 -> 128B-swizzled smem).  The math warps hand slices to the DMA
 // warp through mbarriers and never wait on TMA latency themselves.
+template <int kMode, bool kFinal>
 __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ GemmArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -368,19 +369,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();             // 0: issues the MMAs of the pair
   const int cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
-  const bool sym = p.mode != kModeUpdate;
-  const bool has_d = p.mode != kModeGram;
-  const bool final_w = p.mode == kModeUpdate && p.final_apply;
+  constexpr bool sym = kMode != kModeUpdate;
+  constexpr bool has_d = kMode != kModeGram;
+  constexpr bool final_w = kMode == kModeUpdate && kFinal;
+  // Slice buffers: the update (no mirrored output, no fp32 staging) uses all four
+  // 16 KB buffers for input/output slices, with two output stores in flight;
+  // the other modes use two, plus two for mirrored output or fp32 staging.
+  constexpr int nbuf = (kMode == kModeUpdate && !kFinal) ? 4 : 2;
+  auto slice_buf = [&](int b) { return b < 2 ? dbuf + b * kSliceBytes : mbuf + (b - 2) * kSliceBytes; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl->tmem_full[s], 1);
       mbar_init(&ctl->tmem_empty[s], 8);
-      mbar_init(&ctl->in_full[s], 1);
-      mbar_init(&ctl->out_full[s], 4);
       mbar_init(&ctl->stg_full[s], 4);
       mbar_init(&ctl->stg_free[s], 1);
+    }
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(&ctl->in_full[s], 1);
+      mbar_init(&ctl->out_full[s], 4);
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort_flag = 0;
@@ -418,8 +426,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         const GemmClass& C = p.cls[tc.cls];
         const CUtensorMap* tA;
         const CUtensorMap* tB;
-        if (p.mode == kModeGram) { tA = &p.tmaps[C.tmap_base + (p.x_in ? kTmX1 : kTmX0)]; tB = tA; }
-        else if (p.mode == kModePoly) { tA = &p.tmaps[C.tmap_base + kTmA]; tB = tA; }
+        if (kMode == kModeGram) { tA = &p.tmaps[C.tmap_base + (p.x_in ? kTmX1 : kTmX0)]; tB = tA; }
+        else if (kMode == kModePoly) { tA = &p.tmaps[C.tmap_base + kTmA]; tB = tA; }
         else { tA = &p.tmaps[C.tmap_base + kTmB]; tB = &p.tmaps[C.tmap_base + (p.x_in ? kTmX1mn : kTmX0mn)]; }
         const int arow = tc.tm * kTile + (int)rank * kBM;     // this CTA's A rows
         const int bidx = tc.tn * kTile + (int)rank * kBNh;    // this CTA's B rows (or columns)
@@ -432,7 +440,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           if (!inject_skip) {
             if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], 2 * kStageBytes);
             tma_load_3d_pair(sa, tA, full_lead, kb * kBK, arow, tc.b);
-            if (p.mode == kModeUpdate) {
+            if (kMode == kModeUpdate) {
               // B = X rows [kb*64, +64) x this CTA's 128 columns, MN-major: two 64-col boxes
               tma_load_3d_pair(sb, tB, full_lead, bidx, kb * kBK, tc.b);
               tma_load_3d_pair(sb + kStageBBytes / 2, tB, full_lead, bidx + 64, kb * kBK, tc.b);
@@ -448,7 +456,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN, 0, p.mode == kModeUpdate ? 1 : 0);
+      const uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN, 0, kMode == kModeUpdate ? 1 : 0);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -470,7 +478,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
             const uint64_t adesc = smem_desc_sw128(sa + kk * (kUmmaK * 2), 16, 1024);
-            const uint64_t bdesc = (p.mode == kModeUpdate)
+            const uint64_t bdesc = (kMode == kModeUpdate)
                                        ? smem_desc_sw128(sb + kk * (kUmmaK * 128), kStageBBytes / 2, 1024)
                                        : smem_desc_sw128(sb + kk * (kUmmaK * 2), 16, 1024);
             tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
@@ -499,32 +507,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         for (int c = 0; c < p.nclasses; ++c)
           for (int b = 0; b < p.cls[c].batch; ++b)
             if (p.out[p.cls[c].mat_first + b].tma) tmap_acquire(&p.wmaps[p.cls[c].mat_first + b]);
-      int pend[2] = {-1, -1};                      // parity of an input load not yet seen landed
+      int pend[4] = {-1, -1, -1, -1};              // parity of an input load not yet seen landed
       // Make slice gs's buffer set ready: load its input slice, or just hand it over.
       auto prepare = [&](int gs) {
-        if (gs >= my_slices) return;
-        const int b = gs & 1;
+        if (gs < 0 || gs >= my_slices) return;
+        const int b = gs % nbuf;
         if (has_d) {
           const int t = cid + (gs >> 2) * ncl, h = gs & 3;
           const TileCoord tc = decode_tile(p, t, sym);
           const GemmClass& C = p.cls[tc.cls];
-          const CUtensorMap* tD = (p.mode == kModePoly) ? &p.tmaps[C.tmap_base + kTmA]
+          const CUtensorMap* tD = (kMode == kModePoly) ? &p.tmaps[C.tmap_base + kTmA]
                                                         : &p.tmaps[C.tmap_base + (p.x_in ? kTmX1 : kTmX0)];
           mbar_arrive_expect_tx(&ctl->in_full[b], kSliceBytes);
-          tma_load_3d(dbuf + b * kSliceBytes, tD, &ctl->in_full[b], tc.tn * kTile + 64 * h,
+          tma_load_3d(slice_buf(b), tD, &ctl->in_full[b], tc.tn * kTile + 64 * h,
                       tc.tm * kTile + (int)rank * kBM, tc.b);
-          pend[b] = (gs >> 1) & 1;
+          pend[b] = (gs / nbuf) & 1;
         } else {
           mbar_arrive(&ctl->in_full[b]);
         }
       };
-      prepare(0);
-      prepare(1);
+      for (int g0 = 0; g0 < nbuf; ++g0) prepare(g0);
       bool ok = true;
       int gc = 0;                                  // fp32 chunk counter (final update)
       for (int gs = 0; gs < my_slices && ok; ++gs) {
-        const int b = gs & 1;
-        const uint32_t ph = (uint32_t)((gs >> 1) & 1);
+        const int b = gs % nbuf;
+        const uint32_t ph = (uint32_t)((gs / nbuf) & 1);
         const int t = cid + (gs >> 2) * ncl, h = gs & 3;
         const TileCoord tc = decode_tile(p, t, sym);
         const GemmClass& C = p.cls[tc.cls];
@@ -562,26 +569,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         if (!final_w) {
           const CUtensorMap* tO;
           const CUtensorMap* tM;
-          if (p.mode == kModeGram) { tO = &p.tmaps[C.tmap_base + kTmA]; tM = &p.tmaps[C.tmap_base + kTmAmn]; }
-          else if (p.mode == kModePoly) { tO = &p.tmaps[C.tmap_base + kTmB]; tM = &p.tmaps[C.tmap_base + kTmBmn]; }
+          if (kMode == kModeGram) { tO = &p.tmaps[C.tmap_base + kTmA]; tM = &p.tmaps[C.tmap_base + kTmAmn]; }
+          else if (kMode == kModePoly) { tO = &p.tmaps[C.tmap_base + kTmB]; tM = &p.tmaps[C.tmap_base + kTmBmn]; }
           else { tO = &p.tmaps[C.tmap_base + (p.x_in ? kTmX0 : kTmX1)]; tM = tO; }
           // stores start inside the tensor only (a pair tile can overhang the
           // 128-padded edge by half; the overhang is never stored)
           const int ocols = sym ? C.kp : C.lp;
           const int x0 = tc.tn * kTile + 64 * h;
           const bool mirror = sym && tc.tm != tc.tn;
-          if (row0 < C.kp && x0 < ocols) tma_store_3d(tO, dbuf + b * kSliceBytes, x0, row0, tc.b);
+          if (row0 < C.kp && x0 < ocols) tma_store_3d(tO, slice_buf(b), x0, row0, tc.b);
           if (mirror && x0 < C.kp) {
             if (row0 < C.kp) tma_store_3d(tM, mbuf + b * kSliceBytes, row0, x0, tc.b);
             if (row0 + 64 < C.kp) tma_store_3d(tM, mbuf + b * kSliceBytes + kSliceBytes / 2, row0 + 64, x0, tc.b);
           }
           tma_store_commit();
+          if constexpr (nbuf == 4) {
+            tma_store_wait_read1();                // the previous slice's buffer is free again
+            if (gs >= 1) prepare(gs - 1 + nbuf);   // slices 0..3 were armed before the loop
+            continue;
+          }
           tma_store_wait_read0();                  // buffers b readable again
         }
-        prepare(gs + 2);
+        prepare(gs + nbuf);
       }
       tma_store_wait_all0();
-      for (int b = 0; b < 2; ++b)
+      for (int b = 0; b < nbuf; ++b)
         if (pend[b] >= 0) mbar_wait(&ctl->in_full[b], (uint32_t)pend[b], wc, kDevTimeoutDrain);
       aborted = !ok;
     }
@@ -606,10 +618,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
 #pragma unroll 1
       for (int h = 0; h < 4 && ok; ++h, ++gs) {
-        const int b = gs & 1;
-        uint8_t* dslice = dbuf + b * kSliceBytes;
-        uint8_t* mslice = mbuf + b * kSliceBytes;
-        ok = __all_sync(0xffffffffu, mbar_wait(&ctl->in_full[b], (uint32_t)((gs >> 1) & 1), wc, kDevTimeoutEpi));
+        const int b = gs % nbuf;
+        uint8_t* dslice = slice_buf(b);
+        uint8_t* mslice = mbuf + b * kSliceBytes;   // mirror (GRAM / POLY only: b < 2)
+        ok = __all_sync(0xffffffffu, mbar_wait(&ctl->in_full[b], (uint32_t)((gs / nbuf) & 1), wc, kDevTimeoutEpi));
         if (!ok) break;
         float v[64];
         tmem_ld_32x32b_x64(tbase + (uint32_t)(h * 64), v);
@@ -618,13 +630,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(mapa_shared(&ctl->tmem_empty[acc], 0));
         }
-        if (p.mode == kModeGram) {
+        if (kMode == kModeGram) {
           const float alpha = s * s;
 #pragma unroll
           for (int i = 0; i < 64; ++i) v[i] *= alpha;
         } else {
-          const float wd = (p.mode == kModePoly) ? p.b : p.a * s;
-          const float wa = (p.mode == kModePoly) ? p.c : s;
+          const float wd = (kMode == kModePoly) ? p.b : p.a * s;
+          const float wa = (kMode == kModePoly) ? p.c : s;
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             uint4 raw = *reinterpret_cast<const uint4*>(dslice + sw128_off((uint32_t)r, (uint32_t)u));

@@ -258,7 +258,13 @@ cudaError_t launch_gemm(cudaStream_t stream, const GemmArgs& args, int sm_count)
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ns_gemm_kernel, args);
+  switch (args.mode) {
+    case kModeGram: return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false>, args);
+    case kModePoly: return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModePoly, false>, args);
+    default:
+      return args.final_apply ? cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeUpdate, true>, args)
+                              : cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeUpdate, false>, args);
+  }
 }
 
 // W (m x n fp32, row-major, n % 4 == 0, 16-byte aligned) as a 2-D tensor map
@@ -304,7 +310,14 @@ int device_setup(int dev) {
   if (prop.major != 10 || prop.minor != 0)
     return fail(MUON_ERR_DEVICE, "this library is built for sm_100a (B200); device is sm_" +
                                      std::to_string(prop.major) + std::to_string(prop.minor));
-  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kGemmSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModePoly, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kGemmSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeUpdate, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kGemmSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeUpdate, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kGemmSmemBytes));
   g_dev_ready[dev] = true;
   return MUON_OK;
 }
