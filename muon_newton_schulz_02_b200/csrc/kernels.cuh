@@ -6,8 +6,8 @@
 //                     X0 = bf16(G), stored short-side-major (k x l, padded).
 //   ns_gemm_kernel    one persistent tcgen05 GEMM launch per NS phase over all
 //                     matrices of a group:
-//                       GRAM    A = s^2 * X X^T            (upper tiles, mirrored)
-//                       POLY    B = b*A + c*(A A)          (upper tiles, mirrored)
+//                       GRAM    A = s^2 * X X^T            (upper-triangle 256-blocks only)
+//                       POLY    B = b*A + c*(A A)          (upper-triangle 256-blocks only)
 //                       UPDATE  X' = a*s*X + s*(B X)       (last step: W -= lr*X')
 //                     s = 1/(||G||_F+eps) on the first iteration, 1 afterwards,
 //                     so the listing's normalisation is folded into epilogues.
@@ -39,7 +39,7 @@ enum TmapSlot : int {
   kTmX0 = 0, kTmX1 = 1,             // iterates, 64 x 128 boxes (K-major operand rows, epilogue slices, stores)
   kTmX0mn = 2, kTmX1mn = 3,         // iterates, 64 x 64 boxes (MN-major operand of the update)
   kTmA = 4, kTmB = 5,               // Gram / polynomial matrices, 64 x 128 boxes
-  kTmAmn = 6, kTmBmn = 7            // Gram / polynomial matrices, 64 x 64 boxes (mirrored stores)
+  kTmAmn = 6, kTmBmn = 7            // Gram / polynomial matrices, 64 x 64 boxes (transposed operand reads)
 };
 enum GemmMode : int { kModeGram = 0, kModePoly = 1, kModeUpdate = 2 };
 
@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   uint8_t* dbuf = smem + kStages * kStageBytes;        // 2 x 16 KB: epilogue input / output slices
-  uint8_t* mbuf = dbuf + 2 * kSliceBytes;              // 2 x 16 KB: mirrored output / fp32 staging
+  uint8_t* mbuf = dbuf + 2 * kSliceBytes;              // 2 x 16 KB: slice buffers 2, 3 / fp32 staging
   GemmCtrl* ctl = reinterpret_cast<GemmCtrl*>(mbuf + 2 * kSliceBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -372,10 +372,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   constexpr bool sym = kMode != kModeUpdate;
   constexpr bool has_d = kMode != kModeGram;
   constexpr bool final_w = kMode == kModeUpdate && kFinal;
-  // Slice buffers: the update (no mirrored output, no fp32 staging) uses all four
-  // 16 KB buffers for input/output slices, with two output stores in flight;
-  // the other modes use two, plus two for mirrored output or fp32 staging.
-  constexpr int nbuf = (kMode == kModeUpdate && !kFinal) ? 4 : 2;
+  // Slice buffers: every phase but the final update uses all four 16 KB buffers
+  // for input/output slices, with two output stores in flight; the final update
+  // uses two, plus two for fp32 staging of the weight update.
+  constexpr int nbuf = kFinal ? 2 : 4;
   auto slice_buf = [&](int b) { return b < 2 ? dbuf + b * kSliceBytes : mbuf + (b - 2) * kSliceBytes; };
 
   if (threadIdx.x == 0) {
@@ -431,6 +431,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         else { tA = &p.tmaps[C.tmap_base + kTmB]; tB = &p.tmaps[C.tmap_base + (p.x_in ? kTmX1mn : kTmX0mn)]; }
         const int arow = tc.tm * kTile + (int)rank * kBM;     // this CTA's A rows
         const int bidx = tc.tn * kTile + (int)rank * kBNh;    // this CTA's B rows (or columns)
+        // The Gram and polynomial matrices hold only their upper-triangle 256-blocks:
+        // an operand block below the diagonal is read through its stored transpose.
+        const CUtensorMap* tAt = (kMode == kModePoly) ? &p.tmaps[C.tmap_base + kTmAmn]
+                                                      : &p.tmaps[C.tmap_base + kTmBmn];
         for (int kb = 0; kb < C.kblocks; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, wc, kDevTimeoutEmpty)) { ok = false; break; }
           uint8_t* sa = stage_base + stage * kStageBytes;
@@ -439,11 +443,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           const bool inject_skip = (p.debug_flags & 1) && it == 0 && kb == 0;
           if (!inject_skip) {
             if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], 2 * kStageBytes);
-            tma_load_3d_pair(sa, tA, full_lead, kb * kBK, arow, tc.b);
-            if (kMode == kModeUpdate) {
-              // B = X rows [kb*64, +64) x this CTA's 128 columns, MN-major: two 64-col boxes
-              tma_load_3d_pair(sb, tB, full_lead, bidx, kb * kBK, tc.b);
-              tma_load_3d_pair(sb + kStageBBytes / 2, tB, full_lead, bidx + 64, kb * kBK, tc.b);
+            if (kMode != kModeGram && tc.tm > (kb >> 2)) {
+              // A rows below the diagonal block: columns [arow, +128) of rows [kb*64, +64), MN-major
+              tma_load_3d_pair(sa, tAt, full_lead, arow, kb * kBK, tc.b);
+              tma_load_3d_pair(sa + kStageABytes / 2, tAt, full_lead, arow + 64, kb * kBK, tc.b);
+            } else {
+              tma_load_3d_pair(sa, tA, full_lead, kb * kBK, arow, tc.b);
+            }
+            if (kMode == kModeUpdate || (kMode == kModePoly && tc.tn > (kb >> 2))) {
+              // B = rows [kb*64, +64) x this CTA's 128 columns, MN-major: two 64-col boxes
+              const CUtensorMap* tBm = (kMode == kModeUpdate) ? tB : tAt;
+              tma_load_3d_pair(sb, tBm, full_lead, bidx, kb * kBK, tc.b);
+              tma_load_3d_pair(sb + kStageBBytes / 2, tBm, full_lead, bidx + 64, kb * kBK, tc.b);
             } else {
               tma_load_3d_pair(sb, tB, full_lead, kb * kBK, bidx, tc.b);
             }
@@ -456,7 +467,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN, 0, kMode == kModeUpdate ? 1 : 0);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -475,12 +485,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * kStageBytes);
           const uint32_t sb = sa + kStageABytes;
+          // same choice as the producer: operand blocks below the diagonal arrive MN-major
+          const uint32_t a_mn = (kMode != kModeGram && tc.tm > (kb >> 2)) ? 1u : 0u;
+          const uint32_t b_mn = (kMode == kModeUpdate || (kMode == kModePoly && tc.tn > (kb >> 2))) ? 1u : 0u;
+          const uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN, a_mn, b_mn);
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(sa + kk * (kUmmaK * 2), 16, 1024);
-            const uint64_t bdesc = (kMode == kModeUpdate)
-                                       ? smem_desc_sw128(sb + kk * (kUmmaK * 128), kStageBBytes / 2, 1024)
-                                       : smem_desc_sw128(sb + kk * (kUmmaK * 2), 16, 1024);
+            const uint64_t adesc = a_mn ? smem_desc_sw128(sa + kk * (kUmmaK * 128), kStageABytes / 2, 1024)
+                                        : smem_desc_sw128(sa + kk * (kUmmaK * 2), 16, 1024);
+            const uint64_t bdesc = b_mn ? smem_desc_sw128(sb + kk * (kUmmaK * 128), kStageBBytes / 2, 1024)
+                                        : smem_desc_sw128(sb + kk * (kUmmaK * 2), 16, 1024);
             tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           issued_any = true;
@@ -568,20 +582,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         if (has_d) pend[b] = -1;                   // the math warps saw this slice's input land
         if (!final_w) {
           const CUtensorMap* tO;
-          const CUtensorMap* tM;
-          if (kMode == kModeGram) { tO = &p.tmaps[C.tmap_base + kTmA]; tM = &p.tmaps[C.tmap_base + kTmAmn]; }
-          else if (kMode == kModePoly) { tO = &p.tmaps[C.tmap_base + kTmB]; tM = &p.tmaps[C.tmap_base + kTmBmn]; }
-          else { tO = &p.tmaps[C.tmap_base + (p.x_in ? kTmX0 : kTmX1)]; tM = tO; }
+          if (kMode == kModeGram) tO = &p.tmaps[C.tmap_base + kTmA];
+          else if (kMode == kModePoly) tO = &p.tmaps[C.tmap_base + kTmB];
+          else tO = &p.tmaps[C.tmap_base + (p.x_in ? kTmX0 : kTmX1)];
           // stores start inside the tensor only (a pair tile can overhang the
           // 128-padded edge by half; the overhang is never stored)
           const int ocols = sym ? C.kp : C.lp;
           const int x0 = tc.tn * kTile + 64 * h;
-          const bool mirror = sym && tc.tm != tc.tn;
           if (row0 < C.kp && x0 < ocols) tma_store_3d(tO, slice_buf(b), x0, row0, tc.b);
-          if (mirror && x0 < C.kp) {
-            if (row0 < C.kp) tma_store_3d(tM, mbuf + b * kSliceBytes, row0, x0, tc.b);
-            if (row0 + 64 < C.kp) tma_store_3d(tM, mbuf + b * kSliceBytes + kSliceBytes / 2, row0 + 64, x0, tc.b);
-          }
           tma_store_commit();
           if constexpr (nbuf == 4) {
             tma_store_wait_read1();                // the previous slice's buffer is free again
@@ -613,14 +621,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       if (!ok) break;
       tc_fence_after();
       const float s = p.first ? p.scale[mat] : 1.0f;
-      const bool mirror = sym && tc.tm != tc.tn;
       const int row0 = tc.tm * kTile + (int)rank * kBM;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
 #pragma unroll 1
       for (int h = 0; h < 4 && ok; ++h, ++gs) {
         const int b = gs % nbuf;
         uint8_t* dslice = slice_buf(b);
-        uint8_t* mslice = mbuf + b * kSliceBytes;   // mirror (GRAM / POLY only: b < 2)
         ok = __all_sync(0xffffffffu, mbar_wait(&ctl->in_full[b], (uint32_t)((gs / nbuf) & 1), wc, kDevTimeoutEpi));
         if (!ok) break;
         float v[64];
@@ -707,17 +713,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             o.z = pack_bf16x2(v[u * 8 + 4], v[u * 8 + 5]);
             o.w = pack_bf16x2(v[u * 8 + 6], v[u * 8 + 7]);
             *reinterpret_cast<uint4*>(dslice + sw128_off((uint32_t)r, (uint32_t)u)) = o;
-          }
-          if (mirror) {
-            // transposed copy: mirror box (r / 64) holds rows c (64 columns of
-            // this slice) x columns r (64 rows of this CTA)
-            uint8_t* mbox = mslice + (r >> 6) * (kSliceBytes / 2);
-            const uint32_t mu = (uint32_t)((r & 63) >> 3);
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-              __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(mbox + sw128_off((uint32_t)i, mu)) + (r & 7);
-              *dst = __float2bfloat16_rn(v[i]);
-            }
           }
           fence_async_shared();
         }
