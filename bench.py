@@ -227,7 +227,8 @@ def workload_config(w, args):
     return {"workload": w.name, "matrices": w.n_matrices, "shapes": shapes, "ns_steps": 5,
             "mu": w.mu, "lr": w.lr, "nesterov": True, "grad_sets": args.grad_sets,
             "l2": f"inputs larger than L2: W, g, buf are {w.n_elements * 12 / 1e9:.2f} GB per step",
-            "parallelism": f"independent replicas x{args.gpus}"}
+            "parallelism": (f"matrices sharded over {args.gpus} ranks + all_gather" if args.sharded
+                            else f"independent replicas x{args.gpus}")}
 
 
 def run_ours(args):
@@ -258,8 +259,13 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize(dev)
 
+    from muon_newton_schulz_02_b200 import distributed as mdist
+
     def one_step(s):
-        muon.step(W, gsets[s % args.grad_sets], bufs, lr=w.lr, mu=w.mu, stream=stream)
+        if args.sharded and world > 1:
+            mdist.sharded_step(W, gsets[s % args.grad_sets], bufs, lr=w.lr, mu=w.mu)
+        else:
+            muon.step(W, gsets[s % args.grad_sets], bufs, lr=w.lr, mu=w.mu, stream=stream)
 
     for s in range(args.warmup):
         one_step(s)
@@ -309,13 +315,11 @@ def run_ours(args):
         ms_prof = p0.elapsed_time(p1)
     if muon.sync_status(stream) != 0:
         raise RuntimeError("device status after timing: " + muon.last_error())
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = mdist.max_over_ranks(ms, device=dev)
 
     flops_step = ns_flops(w.shapes)
-    value = flops_step * args.steps * world / (ms_max / 1e3) / 1e12
+    jobs = 1 if args.sharded else world          # sharded: one model split over the ranks
+    value = flops_step * args.steps * jobs / (ms_max / 1e3) / 1e12
 
     peaks, peak_src = load_peaks()
     fk = flops_by_kind(w.shapes)
@@ -327,8 +331,12 @@ def run_ours(args):
             kinds[k] = {"launches": cnt, "ms_total": tms, "us_per_launch": tms / cnt * 1e3,
                         "share_of_step": tms / ms_prof}
     roofline = None
+    # algorithmic work of this rank's own GEMM launches
+    own_flops = flops_step
+    if args.sharded and world > 1:
+        own_flops = ns_flops([w.shapes[i] for i in mdist.partition(w.shapes, world)[rank]])
     if gemm_launches and args.kernel_events:
-        gemm_flops_per_launch = flops_step * args.steps / gemm_launches
+        gemm_flops_per_launch = own_flops * args.steps / gemm_launches
         achieved = gemm_flops_per_launch / (gemm_ms / gemm_launches / 1e3) / 1e12
         peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
         roofline = {"bound": "tensor", "kernel": "ns_gemm_kernel", "achieved": achieved, "peak": peak,
@@ -359,11 +367,7 @@ def run_ours(args):
         t0 = time.perf_counter()
         for s in range(k2):
             muon.step_host(Wh, gh[s % 2], bh, lr=w.lr, mu=w.mu, stream=stream)
-        el = time.perf_counter() - t0
-        te = torch.tensor([el], device=dev, dtype=torch.float64)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        el = float(te.item())
+        el = mdist.max_over_ranks(time.perf_counter() - t0, device=dev)
         e2e = {"value": flops_step * k2 * world / el / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": 12 * w.n_elements, "d2h_bytes_per_step": 8 * w.n_elements,
                "ms_per_step": el / k2 * 1e3, "steps": k2,
@@ -382,7 +386,7 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "strong" if args.sharded else "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) gradients, N(0,0.02) weights, zero-initialised momentum; "
                 "GPT-2-124M hidden-matrix shapes)",
         "config": workload_config(w, args),
@@ -413,7 +417,9 @@ def main():
     ap.add_argument("--ref-total", type=float, default=90.0, help="seconds of CPU oracle work (--impl reference)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-events", type=int, default=1, help="per-launch CUDA events in the timed region")
+    ap.add_argument("--kernel-events", type=int, default=1, help="per-launch CUDA events in a second timed pass")
+    ap.add_argument("--sharded", action="store_true",
+                    help="split one model's matrices over the ranks (all_gather exchange) instead of replicas")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -1,0 +1,94 @@
+"""Data-parallel Muon step over several ranks (one process per GPU).
+
+In data-parallel training every rank holds the same weights and, after the
+gradient all-reduce, the same gradients (the speedrun context of the
+Modded-NanoGPT article trains on 8 GPUs launched with --nproc_per_node).  The
+Muon update of each weight matrix is independent of the others, so the ranks
+split the matrices: rank r runs the step (momentum, NS5, apply) on the
+matrices it owns, then one all_gather gives every rank every updated matrix.
+Each rank keeps the momentum buffers of the matrices it owns; the buffers of
+other ranks' matrices are left untouched.
+
+Nothing here loads another GPU's memory directly: the exchange is a NCCL (or,
+on the CPU, gloo) all_gather of a packed fp32 buffer.
+"""
+
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+
+def step_flops(rows: int, cols: int, ns_steps: int = 5) -> float:
+    """Algorithmic NS5 flops of one matrix (symmetry of X X^T and A A used)."""
+    k, l = min(rows, cols), max(rows, cols)
+    return float(ns_steps * (k * (k + 1) * l + k * k * (k + 1) + 2 * k * k * l))
+
+
+def partition(shapes, world: int, ns_steps: int = 5):
+    """Greedy longest-processing-time split: matrices by decreasing flops, each
+    to the rank with the least work so far (ties: lowest rank).  Deterministic,
+    so every rank computes the same split.  Returns a list of index lists."""
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    order = sorted(range(len(shapes)), key=lambda i: (-step_flops(*shapes[i], ns_steps), i))
+    load = [0.0] * world
+    owned = [[] for _ in range(world)]
+    for i in order:
+        r = min(range(world), key=lambda q: (load[q], q))
+        owned[r].append(i)
+        load[r] += step_flops(*shapes[i], ns_steps)
+    return [sorted(o) for o in owned]
+
+
+def _default_local_step(params, grads, bufs, lr, mu, ns_steps):
+    from . import step
+    step(params, grads, bufs, lr=lr, mu=mu, ns_steps=ns_steps)
+
+
+def sharded_step(params, grads, bufs, lr: float, mu: float, ns_steps: int = 5, group=None, local_step=None):
+    """One Muon step split across the ranks of `group` (default: the world).
+
+    params / grads / bufs: the full, identical lists on every rank (same
+    device type on all ranks: CUDA with NCCL, CPU with gloo).  On return every
+    rank holds every updated matrix.  `local_step(params, grads, bufs, lr, mu,
+    ns_steps)` updates a sub-list in place; the default is the CUDA step."""
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    local_step = local_step or _default_local_step
+    shapes = [tuple(p.shape) for p in params]
+    owned = partition(shapes, world, ns_steps)
+    mine = owned[rank]
+    if mine:
+        local_step([params[i] for i in mine], [grads[i] for i in mine], [bufs[i] for i in mine], lr, mu, ns_steps)
+    if world == 1:
+        return owned
+    sizes = [sum(params[i].numel() for i in o) for o in owned]
+    chunk = max(sizes)
+    dev = params[0].device
+    send = torch.zeros(chunk, dtype=torch.float32, device=dev)
+    off = 0
+    for i in mine:
+        n = params[i].numel()
+        send[off:off + n].copy_(params[i].reshape(-1))
+        off += n
+    recv = [torch.empty(chunk, dtype=torch.float32, device=dev) for _ in range(world)]
+    dist.all_gather(recv, send, group=group)
+    for r in range(world):
+        if r == rank:
+            continue
+        off = 0
+        for i in owned[r]:
+            n = params[i].numel()
+            params[i].reshape(-1).copy_(recv[r][off:off + n])
+            off += n
+    return owned
+
+
+def max_over_ranks(value: float, group=None, device=None) -> float:
+    """The maximum of a per-rank scalar (timings are reported as the slowest rank)."""
+    if not dist.is_initialized() or dist.get_world_size(group) == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
