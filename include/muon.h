@@ -160,7 +160,8 @@ void muon_release(void);
 #define MUON_KIND_UPDATE 3
 #define MUON_KIND_UPDATE_APPLY 4
 #define MUON_KIND_APPLY_X0 5
-#define MUON_NUM_KINDS 6
+#define MUON_KIND_SMALL 6        /* fused single-CTA step of small matrices */
+#define MUON_NUM_KINDS 7
 
 /* 1: bracket every kernel launch with CUDA events on its stream; 0: stop. */
 int muon_profile_enable(int enable);

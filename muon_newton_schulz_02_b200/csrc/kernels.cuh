@@ -735,6 +735,382 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   }
 }
 
+// ================================================ small matrices, fused ===
+// The whole step of one small matrix (short side k <= 128, long side l <= 512)
+// in one CTA: momentum and norm while X0 is written into shared memory, then
+// every quintic iteration with X, A and B resident in shared memory and the
+// accumulators in TMEM, then the apply.  One launch covers every small matrix
+// of a call (one CTA each).  X is stored as 128-row x 64-column chunks with
+// the 128-byte swizzle: read K-major by the Gram product and MN-major (LBO =
+// chunk stride) by the update, so it is never transposed.
+constexpr int kSmallThreads = 128;
+constexpr int kSmallMaxK = 128;
+constexpr int kSmallMaxL = 512;
+constexpr uint32_t kSmallChunk = 128 * 64 * 2;                       // 16 KB
+constexpr uint32_t kSmallSmem = (kSmallMaxL / 64 + 2 + 2) * kSmallChunk + 256 + 1024;
+
+struct SmallMat {
+  const float* g;
+  float* buf;
+  float* w;           // W (step) or O (orthogonalize), m x n
+  int m, n, trans, vec;
+  int lp;             // long side padded to 64
+};
+
+struct SmallArgs {
+  int nmats, ns_steps, nesterov, has_buf, assign;
+  float mu, eps, a, b, c, lr;
+  int* status;
+  unsigned long long wait_limit_ns;
+  SmallMat mats[kMaxMats];
+};
+
+// smem byte offset of element (row r, col c) in a chunked 128B-swizzled buffer
+__device__ __forceinline__ uint32_t chunk_off(uint32_t r, uint32_t c) {
+  return (c >> 6) * kSmallChunk + r * 128u + ((((c & 63u) >> 3) ^ (r & 7u)) << 4) + (c & 7u) * 2u;
+}
+
+__global__ void __launch_bounds__(kSmallThreads, 1) ns_small_kernel(const __grid_constant__ SmallArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Xs = smem;                                        // 8 chunks
+  uint8_t* As = Xs + (kSmallMaxL / 64) * kSmallChunk;        // 2 chunks
+  uint8_t* Bs = As + 2 * kSmallChunk;                        // 2 chunks
+  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(Bs + 2 * kSmallChunk);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(abort_flag + 1);     // 4 warp partials
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const SmallMat& M = p.mats[blockIdx.x];
+  const int lp = M.lp, k = M.trans ? M.n : M.m;
+  (void)k;
+
+  if (tid == 0) {
+    mbar_init(mma_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+
+  // ---- momentum, norm, X0 (bf16) into shared memory; zero padding included.
+  // Each thread issues all loads of a batch before any store (one CTA per SM
+  // has few warps to hide memory latency with).
+  const float* __restrict__ gp = M.g;
+  float* __restrict__ bp = M.buf;
+  float ss = 0.f;
+  auto load4 = [&](size_t off, int col, int ncols, float (&gv)[4], float (&bv)[4]) {
+    if (M.vec && col + 3 < ncols) {
+      const float4 g4 = __ldg(reinterpret_cast<const float4*>(gp + off));
+      gv[0] = g4.x; gv[1] = g4.y; gv[2] = g4.z; gv[3] = g4.w;
+      if (p.has_buf) {
+        const float4 b4 = *reinterpret_cast<const float4*>(bp + off);
+        bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (col + q < ncols) {
+          gv[q] = gp[off + q];
+          if (p.has_buf) bv[q] = bp[off + q];
+        }
+      }
+    }
+  };
+  auto store4 = [&](size_t off, int col, int ncols, const float (&bv)[4]) {
+    if (!p.has_buf) return;
+    if (M.vec && col + 3 < ncols) {
+      *reinterpret_cast<float4*>(bp + off) = make_float4(bv[0], bv[1], bv[2], bv[3]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (col + q < ncols) bp[off + q] = bv[q];
+    }
+  };
+  if (!M.trans) {
+    // X[i][j] = G[i][j]: a batch is 2 rows x up to 4 steps of 128 columns
+    for (int i0 = warp; i0 < kSmallMaxK; i0 += 8) {
+      float gv[2][4][4], bv[2][4][4];
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+        for (int cs = 0; cs < 4; ++cs) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) { gv[rr][cs][q] = 0.f; bv[rr][cs][q] = 0.f; }
+          const int i = i0 + 4 * rr, j = cs * 128 + 4 * lane;
+          if (i < M.m && j < M.n) load4((size_t)i * M.n + j, j, M.n, gv[rr][cs], bv[rr][cs]);
+        }
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+        for (int cs = 0; cs < 4; ++cs) {
+          const int i = i0 + 4 * rr, j = cs * 128 + 4 * lane;
+          if (j >= lp) continue;
+          float G[4] = {0.f, 0.f, 0.f, 0.f};
+          if (i < M.m && j < M.n) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (j + q < M.n) G[q] = nesterov_g(gv[rr][cs][q], bv[rr][cs][q], p.mu, p.nesterov, p.has_buf);
+            store4((size_t)i * M.n + j, j, M.n, bv[rr][cs]);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) ss = fmaf(G[q], G[q], ss);
+          *reinterpret_cast<uint2*>(Xs + chunk_off((uint32_t)i, (uint32_t)j)) =
+              make_uint2(pack_bf16x2(G[0], G[1]), pack_bf16x2(G[2], G[3]));
+        }
+    }
+  } else {
+    // X[j][i] = G[i][j]: a warp reads rows i of G (n <= 128 columns), 8 rows per batch
+    for (int i0 = warp; i0 < lp; i0 += 32) {
+      float gv[8][4], bv[8][4];
+      const int j = 4 * lane;                                 // X rows j..j+3
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) { gv[t][q] = 0.f; bv[t][q] = 0.f; }
+        const int i = i0 + 4 * t;
+        if (i < M.m && j < M.n) load4((size_t)i * M.n + j, j, M.n, gv[t], bv[t]);
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int i = i0 + 4 * t;
+        if (i >= lp) continue;
+        float G[4] = {0.f, 0.f, 0.f, 0.f};
+        if (i < M.m && j < M.n) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (j + q < M.n) G[q] = nesterov_g(gv[t][q], bv[t][q], p.mu, p.nesterov, p.has_buf);
+          store4((size_t)i * M.n + j, j, M.n, bv[t]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          ss = fmaf(G[q], G[q], ss);
+          *reinterpret_cast<__nv_bfloat16*>(Xs + chunk_off((uint32_t)(j + q), (uint32_t)i)) =
+              __float2bfloat16_rn(G[q]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) red[warp] = ss;
+  fence_async_shared();                                      // X0 visible to the tensor core
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const float scale = 1.0f / ((float)sqrt((double)red[0] + (double)red[1] + (double)red[2] + (double)red[3]) + p.eps);
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's 32 lanes
+  const int r = warp * 32 + lane;                            // row of X / A / B owned by this thread
+  WaitCtx wc{abort_flag, p.status, p.wait_limit_ns, 0u};
+  bool ok = true;
+  uint32_t phase = 0;
+
+  auto wait_mma = [&]() {
+    bool got = ok && mbar_wait(mma_bar, phase, wc, kDevTimeoutAccum);
+    phase ^= 1u;
+    ok = __syncthreads_and(got) != 0;
+    tc_fence_after();
+  };
+  auto publish_smem = [&]() {                                // generic writes -> next MMAs
+    fence_async_shared();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  };
+
+  // W -= lr * O (or O = result) for X columns cc*32 .. +31 of this thread's row
+  // r: staged in the A buffer (free at that point), then read-modified-written
+  // in whole 128-byte rows with all loads of a thread in flight at once
+  auto apply_chunk = [&](int cc, const float* v) {
+        float* S = reinterpret_cast<float*>(As);
+        if (!M.trans) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4*>(S + r * 32 + ((j ^ (r & 7)) << 2)) =
+                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) S[q * 128 + r] = v[q];
+        }
+        __syncthreads();
+        float4 o[8], w4[8];
+        float* wp[8];
+        bool okw[8], full[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int idx = tid + kSmallThreads * t;
+          int wi, wj;
+          if (!M.trans) {
+            const int row = idx >> 3, qd = idx & 7;
+            wi = row; wj = cc * 32 + 4 * qd;
+            o[t] = *reinterpret_cast<const float4*>(S + row * 32 + ((qd ^ (row & 7)) << 2));
+          } else {
+            const int c = idx >> 5, qd = idx & 31;
+            wi = cc * 32 + c; wj = 4 * qd;
+            o[t] = *reinterpret_cast<const float4*>(S + c * 128 + 4 * qd);
+          }
+          okw[t] = wi < M.m && wj < M.n;
+          full[t] = M.vec && wj + 3 < M.n;
+          wp[t] = M.w + (size_t)wi * M.n + wj;
+          w4[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (okw[t] && full[t] && !p.assign) w4[t] = *reinterpret_cast<const float4*>(wp[t]);
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (!okw[t]) continue;
+          if (full[t]) {
+            float4 r4 = w4[t];
+            if (p.assign) r4 = o[t];
+            else { r4.x -= p.lr * o[t].x; r4.y -= p.lr * o[t].y; r4.z -= p.lr * o[t].z; r4.w -= p.lr * o[t].w; }
+            *reinterpret_cast<float4*>(wp[t]) = r4;
+          } else {
+            const float ov[4] = {o[t].x, o[t].y, o[t].z, o[t].w};
+            const int wj = (int)((wp[t] - M.w) % M.n);
+            for (int e = 0; e < 4 && wj + e < M.n; ++e) wp[t][e] = p.assign ? ov[e] : wp[t][e] - p.lr * ov[e];
+          }
+        }
+        __syncthreads();
+  };
+
+  for (int it = 0; it < p.ns_steps && ok; ++it) {
+    const float s = it == 0 ? scale : 1.0f;
+    const bool last = it == p.ns_steps - 1;
+    // A = s^2 X X^T : M = N = 128, K = lp
+    if (tid == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+      for (int kk = 0; kk < lp / 16; ++kk) {
+        const uint32_t a = smem_u32(Xs) + (kk >> 2) * kSmallChunk + (kk & 3) * 32;
+        const uint64_t d = smem_desc_sw128(a, 16, 1024);
+        tc_mma_bf16(tmem, d, d, idesc, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(mma_bar);
+    }
+    wait_mma();
+    if (!ok) break;
+#pragma unroll 1
+    for (int c64 = 0; c64 < 2; ++c64) {
+      float v[64];
+      tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v);
+#pragma unroll
+      for (int q = 0; q < 64; q += 8) {
+        uint4 o;
+        o.x = pack_bf16x2(s * s * v[q], s * s * v[q + 1]);
+        o.y = pack_bf16x2(s * s * v[q + 2], s * s * v[q + 3]);
+        o.z = pack_bf16x2(s * s * v[q + 4], s * s * v[q + 5]);
+        o.w = pack_bf16x2(s * s * v[q + 6], s * s * v[q + 7]);
+        *reinterpret_cast<uint4*>(As + chunk_off((uint32_t)r, (uint32_t)(c64 * 64 + q))) = o;
+      }
+    }
+    publish_smem();
+    // B = b A + c A A : M = N = K = 128 (A symmetric: both operands K-major rows of A)
+    if (tid == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t a = smem_u32(As) + (kk >> 2) * kSmallChunk + (kk & 3) * 32;
+        const uint64_t d = smem_desc_sw128(a, 16, 1024);
+        tc_mma_bf16(tmem, d, d, idesc, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(mma_bar);
+    }
+    wait_mma();
+    if (!ok) break;
+#pragma unroll 1
+    for (int c64 = 0; c64 < 2; ++c64) {
+      float v[64];
+      tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v);
+#pragma unroll
+      for (int q = 0; q < 64; q += 8) {
+        const uint4 araw = *reinterpret_cast<const uint4*>(As + chunk_off((uint32_t)r, (uint32_t)(c64 * 64 + q)));
+        const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&araw);
+        float o8[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(ah[e]);
+          o8[2 * e] = fmaf(p.c, v[q + 2 * e], p.b * f.x);
+          o8[2 * e + 1] = fmaf(p.c, v[q + 2 * e + 1], p.b * f.y);
+        }
+        *reinterpret_cast<uint4*>(Bs + chunk_off((uint32_t)r, (uint32_t)(c64 * 64 + q))) =
+            make_uint4(pack_bf16x2(o8[0], o8[1]), pack_bf16x2(o8[2], o8[3]), pack_bf16x2(o8[4], o8[5]),
+                       pack_bf16x2(o8[6], o8[7]));
+      }
+    }
+    publish_smem();
+    // X' = a s X + s B X : M = 128, N = lp (<= 256 per instruction), K = 128; X read MN-major
+    if (tid == 0) {
+      for (int n0 = 0; n0 < lp; n0 += 256) {
+        const int nn = min(256, lp - n0);
+        const uint32_t idesc = idesc_bf16_f32(128, (uint32_t)nn, 0, 1);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t a = smem_u32(Bs) + (kk >> 2) * kSmallChunk + (kk & 3) * 32;
+          const uint32_t b = smem_u32(Xs) + (n0 >> 6) * kSmallChunk + kk * (16 * 128);
+          tc_mma_bf16(tmem + (uint32_t)n0, smem_desc_sw128(a, 16, 1024), smem_desc_sw128(b, kSmallChunk, 1024),
+                      idesc, kk > 0 ? 1u : 0u);
+        }
+      }
+      tc_commit(mma_bar);
+    }
+    wait_mma();
+    if (!ok) break;
+#pragma unroll 1
+    for (int c64 = 0; c64 < lp / 64; ++c64) {
+     float v64[64];
+     tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v64);
+#pragma unroll
+     for (int half = 0; half < 2; ++half) {
+      const int cc = 2 * c64 + half;
+      float* v = v64 + 32 * half;
+#pragma unroll
+      for (int q = 0; q < 32; q += 8) {
+        const uint32_t xo = chunk_off((uint32_t)r, (uint32_t)(cc * 32 + q));
+        const uint4 xraw = *reinterpret_cast<const uint4*>(Xs + xo);
+        const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xraw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(xh[e]);
+          v[q + 2 * e] = fmaf(s, v[q + 2 * e], p.a * s * f.x);
+          v[q + 2 * e + 1] = fmaf(s, v[q + 2 * e + 1], p.a * s * f.y);
+        }
+        if (!last)
+          *reinterpret_cast<uint4*>(Xs + xo) =
+              make_uint4(pack_bf16x2(v[q], v[q + 1]), pack_bf16x2(v[q + 2], v[q + 3]),
+                         pack_bf16x2(v[q + 4], v[q + 5]), pack_bf16x2(v[q + 6], v[q + 7]));
+      }
+      if (last) apply_chunk(cc, v);
+     }
+    }
+    if (!last) publish_smem();
+  }
+  if (p.ns_steps == 0 && ok) {
+    // O = s * X0 (the listing with an empty loop)
+#pragma unroll 1
+    for (int cc = 0; cc < lp / 32; ++cc) {
+      float v[32];
+#pragma unroll
+      for (int q = 0; q < 32; q += 8) {
+        const uint4 xraw = *reinterpret_cast<const uint4*>(Xs + chunk_off((uint32_t)r, (uint32_t)(cc * 32 + q)));
+        const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xraw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(xh[e]);
+          v[q + 2 * e] = scale * f.x;
+          v[q + 2 * e + 1] = scale * f.y;
+        }
+      }
+      apply_chunk(cc, v);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // ======================================================= ns_steps == 0 ===
 __global__ void apply_x0_kernel(const __grid_constant__ ApplyArgs p) {
   const int mi = blockIdx.y;

@@ -95,6 +95,7 @@ static_assert(kMaxMats * 4 <= kTicketBytes, "ticket region too small");
 struct Plan {
   std::vector<int64_t> shapes;
   std::vector<Group> groups;
+  std::vector<MatDesc> small;               // matrices of the fused single-CTA kernel (no workspace)
   size_t ws_bytes = 0;
   size_t tmap_bytes = 0;
   void* ws = nullptr;                       // workspace the tensor maps point into
@@ -131,6 +132,15 @@ int build_layout(const int64_t* shapes, int n, Plan& plan) {
     if (d.kp > 16384) return fail(MUON_ERR_SHAPE, "short side above 16384 is not supported");
     d.user = i;
     all[i] = d;
+  }
+  // short side <= 128 and long side <= 512: fused single-CTA kernel, no workspace
+  {
+    std::vector<MatDesc> big;
+    for (const auto& d : all) {
+      if (d.k <= kSmallMaxK && round_up(d.l, 64) <= kSmallMaxL) plan.small.push_back(d);
+      else big.push_back(d);
+    }
+    all.swap(big);
   }
   // greedy grouping in caller order, respecting kMaxMats and kMaxClasses
   std::vector<std::vector<MatDesc>> raw;
@@ -310,6 +320,7 @@ int device_setup(int dev) {
   if (prop.major != 10 || prop.minor != 0)
     return fail(MUON_ERR_DEVICE, "this library is built for sm_100a (B200); device is sm_" +
                                      std::to_string(prop.major) + std::to_string(prop.minor));
+  CUDA_TRY(cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallSmem));
   CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kGemmSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModePoly, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -371,11 +382,11 @@ int get_plan(Ctx& c, const int64_t* shapes, int n, Plan** out) {
   auto p = std::make_unique<Plan>();
   int rc = build_layout(shapes, n, *p);
   if (rc) return rc;
-  rc = ensure_workspace(c, p->ws_bytes);
+  rc = ensure_workspace(c, std::max<size_t>(p->ws_bytes, kTicketBytes));
   if (rc) return rc;
   p->ws = c.ws;
   char* base = (char*)c.ws;
-  if (cudaMalloc(&p->tmaps, p->tmap_bytes) != cudaSuccess) {
+  if (p->tmap_bytes && cudaMalloc(&p->tmaps, p->tmap_bytes) != cudaSuccess) {
     cudaGetLastError();
     p->tmaps = nullptr;
     return fail(MUON_ERR_NOMEM, "tensor-map table allocation failed");
@@ -594,6 +605,43 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
   return MUON_OK;
 }
 
+// One launch of the fused kernel per kMaxMats small matrices (one CTA each).
+int run_small(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& small, const StepIO& io, int* status) {
+  for (size_t base = 0; base < small.size(); base += kMaxMats) {
+    const int nm = (int)std::min<size_t>(kMaxMats, small.size() - base);
+    auto sa = std::make_unique<SmallArgs>();
+    std::memset(sa.get(), 0, sizeof(SmallArgs));
+    sa->nmats = nm;
+    sa->ns_steps = io.ns_steps;
+    sa->nesterov = io.nesterov;
+    sa->has_buf = io.buf != nullptr;
+    sa->assign = io.assign;
+    sa->mu = io.mu; sa->eps = io.eps; sa->a = io.a; sa->b = io.b; sa->c = io.c; sa->lr = io.lr;
+    sa->status = status;
+    sa->wait_limit_ns = g_wait_limit_ns;
+    for (int i = 0; i < nm; ++i) {
+      const MatDesc& d = small[base + i];
+      SmallMat& m = sa->mats[i];
+      m.g = io.g[d.user];
+      m.buf = io.buf ? io.buf[d.user] : nullptr;
+      m.w = io.W[d.user];
+      m.m = d.m; m.n = d.n; m.trans = d.trans;
+      m.vec = (d.n % 4 == 0) && aligned16(m.g) && aligned16(m.w) && (!m.buf || aligned16(m.buf));
+      m.lp = round_up(d.l, 64);
+    }
+    auto go = [&] { ns_small_kernel<<<nm, kSmallThreads, kSmallSmem, stream>>>(*sa); };
+    if (c) {
+      int rc = launch(*c, MUON_KIND_SMALL, go);
+      if (rc) return rc;
+    } else {
+      go();
+      CUDA_TRY(cudaGetLastError());
+      g_launches.fetch_add(1);
+    }
+  }
+  return MUON_OK;
+}
+
 int validate_common(const int64_t* shapes, int n, int ns_steps) {
   if (!shapes) return fail(MUON_ERR_INVALID_ARG, "shapes is null");
   if (n <= 0) return fail(MUON_ERR_INVALID_ARG, "n must be > 0");
@@ -617,6 +665,7 @@ int step_impl(const StepIO& io, const int64_t* shapes, int n, void* stream) {
   if ((rc = check_status(*c))) return rc;
   Plan* plan = nullptr;
   if ((rc = get_plan(*c, shapes, n, &plan))) return rc;
+  if (!plan->small.empty() && (rc = run_small(c, c->stream, plan->small, io, c->status_d))) return rc;
   for (size_t gi = 0; gi < plan->groups.size(); ++gi)
     if ((rc = run_group(*c, *plan, gi, io))) return rc;
   return MUON_OK;
@@ -700,6 +749,7 @@ int muon_step_host(float* const* params, const float* const* grads, float* const
   if ((rc = get_plan(*c, shapes, n, &plan))) return rc;
   StepIO io{dW.data(), (const float* const*)dg.data(), db.data(), lr, mu, MUON_NS_A, MUON_NS_B, MUON_NS_C,
             MUON_NS_EPS, ns_steps, 1, 0};
+  if (!plan->small.empty() && (rc = run_small(c, c->stream, plan->small, io, c->status_d))) return rc;
   for (size_t gi = 0; gi < plan->groups.size(); ++gi)
     if ((rc = run_group(*c, *plan, gi, io))) return rc;
   for (int i = 0; i < n; ++i) {
@@ -717,7 +767,7 @@ size_t muon_workspace_size(const int64_t* shapes, int n) {
     if (shapes[i] <= 0) return 0;
   Plan p;
   if (build_layout(shapes, n, p)) return 0;
-  return p.ws_bytes;
+  return std::max<size_t>(p.ws_bytes, kTicketBytes);
 }
 
 int muon_sync_status(void* stream) {
@@ -941,12 +991,13 @@ extern "C" int muon_step_noalloc(float* const* params, const float* const* grads
   if ((rc = validate_ptrs((const void* const*)momentum_bufs, n, "momentum_bufs"))) return rc;
   Plan plan;
   if ((rc = build_layout(shapes, n, plan))) return rc;
-  if (plan.groups.size() != 1)
+  if (plan.groups.size() > 1)
     return fail(MUON_ERR_UNSUPPORTED, "muon_step_noalloc takes at most " + std::to_string(kMaxMats) +
                                           " matrices of at most " + std::to_string(kMaxClasses) +
                                           " padded shapes per call");
-  const size_t table = (plan.groups[0].classes.size() * kTmapsPerClass + plan.groups[0].mats.size()) *
-                       sizeof(CUtensorMap);
+  const size_t table = plan.groups.empty() ? 0
+                       : (plan.groups[0].classes.size() * kTmapsPerClass + plan.groups[0].mats.size()) *
+                             sizeof(CUtensorMap);
   if (plan.ws_bytes > kNoAllocBytes - kNoAllocTableBytes || table > kNoAllocTableBytes - 256)
     return fail(MUON_ERR_UNSUPPORTED, "muon_step_noalloc: these shapes need " + std::to_string(plan.ws_bytes) +
                                           " bytes of scratch; the static scratch holds " +
@@ -960,5 +1011,11 @@ extern "C" int muon_step_noalloc(float* const* params, const float* const* grads
   int sm_count = 148;
   CUDA_TRY(cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev));
   StepIO io{params, grads, momentum_bufs, lr, mu, MUON_NS_A, MUON_NS_B, MUON_NS_C, MUON_NS_EPS, ns_steps, 1, 0};
+  int* status = (int*)((char*)base + kNoAllocBytes - 256);
+  if (!plan.small.empty()) {
+    CUDA_TRY(cudaMemsetAsync(status, 0, 256, (cudaStream_t)stream));
+    if ((rc = run_small(nullptr, (cudaStream_t)stream, plan.small, io, status))) return rc;
+  }
+  if (plan.groups.empty()) return MUON_OK;
   return noalloc_launch((cudaStream_t)stream, (char*)base, plan, io, sm_count);
 }

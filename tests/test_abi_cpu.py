@@ -68,7 +68,11 @@ def _expect_ws(shapes):
     classes = {}
     for r, c in shapes:
         k, l = min(r, c), max(r, c)
+        if k <= 128 and up(l, 64) <= 512:
+            continue                      # fused single-CTA kernel: no workspace
         classes.setdefault((up(k, 128), up(l, 128)), []).append((r, c))
+    if not classes:
+        return 4096
     off = 4096
     tiles = 0
     for (kp, lp), mats in classes.items():
@@ -78,7 +82,7 @@ def _expect_ws(shapes):
         off = up(off + b * kp * kp * 2, 1024)
         off = up(off + b * kp * kp * 2, 1024)
         tiles += b * (kp // 64) * (lp // 128)
-    n = len(shapes)
+    n = sum(len(v) for v in classes.values())
     off = up(off + tiles * 4, 1024)
     off = up(off + n * 4, 1024)
     return off
@@ -88,6 +92,7 @@ def _expect_ws(shapes):
     [(128, 512)],
     [(768, 768)] * 4 + [(768, 3072), (3072, 768)],
     [(1, 1), (127, 129), (129, 127), (1000, 300)],
+    [(128, 640), (129, 512), (256, 256), (64, 64)],
 ])
 def test_workspace_size_matches_layout(L, shapes):
     assert _ws(shapes) == _expect_ws(shapes)
@@ -100,8 +105,8 @@ def test_workspace_size_rejects_bad_input(L):
 
 def test_many_matrices_split_into_groups(L):
     # more matrices than one launch holds: groups share the data region
-    shapes = [(64, 64)] * 700
-    one_group = _expect_ws([(64, 64)] * 320)
+    shapes = [(192, 192)] * 700
+    one_group = _expect_ws([(192, 192)] * 320)
     got = _ws(shapes)
     assert got == one_group
 

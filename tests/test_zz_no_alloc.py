@@ -57,13 +57,19 @@ def test_noalloc_matches_muon_step_on_two_calls_in_a_row():
             assert relF(bb[i].cpu().numpy(), ba[i].cpu().numpy()) <= REL_BUF, (call, i)
 
 
+def _refused(shapes):
+    # real device buffers, so that nothing could fault even if a call were accepted
+    dev = torch.device("cuda:0")
+    ts = [torch.zeros(*s, device=dev) for s in shapes]
+    ptrs = (ctypes.c_void_p * len(ts))(*[ctypes.c_void_p(t.data_ptr()) for t in ts])
+    sh = (ctypes.c_int64 * (2 * len(shapes)))(*[v for s in shapes for v in s])
+    rc = muon.lib().muon_step_noalloc(ptrs, ptrs, ptrs, sh, len(shapes), 0.02, 0.95, 5,
+                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    return rc
+
+
 def test_noalloc_rejects_requests_beyond_its_scratch():
-    L = muon.lib()
-    p = (ctypes.c_void_p * 1)(ctypes.c_void_p(16))
-    sh = (ctypes.c_int64 * 2)(4096, 4096)             # needs 4 x 32 MiB of iterates and matrices
-    assert L.muon_step_noalloc(p, p, p, sh, 1, 0.02, 0.95, 5, None) == -7
+    assert _refused([(4096, 4096)]) == -7             # needs 4 x 32 MiB of iterates and matrices
     assert "static scratch" in muon.last_error()
-    many = 400
-    pp = (ctypes.c_void_p * many)(*[ctypes.c_void_p(16)] * many)
-    shm = (ctypes.c_int64 * (2 * many))(*([64, 64] * many))
-    assert L.muon_step_noalloc(pp, pp, pp, shm, many, 0.02, 0.95, 5, None) == -7
+    assert _refused([(192, 192)] * 400) == -7         # more matrices than one call takes
