@@ -1,0 +1,76 @@
+"""Precision budget of the bf16 Newton-Schulz iteration, and of fp8 operands.
+
+An emulation on the CPU (torch dtype casts) of the rounding the GPU path
+performs: bf16 GEMM operands, fp32 accumulation, one bf16 rounding per GEMM
+output (fused epilogues).  Its error against the fp64 oracle matches what the
+GPU measures on the same shapes (about 1e-2), so it can rank alternatives
+before any kernel is written:
+
+* fp8 (e4m3 / e5m2) operands in every iteration are far outside the 3e-2 bar;
+* e4m3 operands in only the first two iterations stay inside it, because the
+  later quintic iterations absorb the early perturbation.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import muon_oracle as orc
+
+A_, B_, C_ = orc.NS_A, orc.NS_B, orc.NS_C
+
+
+def q_bf16(x):
+    return x.to(torch.bfloat16).to(torch.float32)
+
+
+def q_fp8(x, fmt=torch.float8_e4m3fn, maxv=448.0):
+    s = x.abs().max().clamp(min=1e-30) / maxv
+    return (x / s).to(fmt).to(torch.float32) * s
+
+
+def ns_emulated(G, fp8_iters=(), fmt=torch.float8_e4m3fn, maxv=448.0, steps=5):
+    X = torch.tensor(G, dtype=torch.float32)
+    X = X / (X.norm() + 1e-7)
+    t = X.shape[0] > X.shape[1]
+    if t:
+        X = X.T
+    X = q_bf16(X)
+    for i in range(steps):
+        qop = (lambda x: q_fp8(x, fmt, maxv)) if i in fp8_iters else q_bf16
+        Xo = qop(X)
+        A = q_bf16(Xo @ Xo.T)
+        Ao = qop(A)
+        B = q_bf16(B_ * A + C_ * (Ao @ Ao))
+        Xn = A_ * X + qop(B) @ Xo
+        X = Xn if i == steps - 1 else q_bf16(Xn)
+    return (X.T if t else X).double().numpy()
+
+
+def _rel(O, ref):
+    return float(np.linalg.norm(O - ref) / np.linalg.norm(ref))
+
+
+@pytest.fixture(scope="module")
+def case():
+    G = np.random.default_rng(0).standard_normal((384, 768)) * 0.02
+    return G, orc.zeroth_power_via_newtonschulz5(G)
+
+
+def test_bf16_fused_epilogue_error_is_about_one_percent(case):
+    G, ref = case
+    assert 5e-3 < _rel(ns_emulated(G), ref) < 2e-2
+
+
+def test_fp8_operands_everywhere_break_the_tolerance(case):
+    G, ref = case
+    assert _rel(ns_emulated(G, fp8_iters=range(5)), ref) > 0.1
+    assert _rel(ns_emulated(G, fp8_iters=range(5), fmt=torch.float8_e5m2, maxv=57344.0), ref) > 0.1
+
+
+def test_fp8_operands_in_first_two_iterations_stay_inside(case):
+    G, ref = case
+    bf16 = _rel(ns_emulated(G), ref)
+    mixed = _rel(ns_emulated(G, fp8_iters=(0, 1)), ref)
+    assert mixed < 3e-2 and abs(mixed - bf16) < 5e-3
+    assert _rel(ns_emulated(G, fp8_iters=(0, 1, 2, 3)), ref) > 3e-2
