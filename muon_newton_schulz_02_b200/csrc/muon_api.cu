@@ -308,6 +308,8 @@ struct Ctx {
   std::vector<ProfRec> prof;
   std::vector<cudaEvent_t> event_pool;
   int sm_count = 148;
+  cudaStream_t h2d = nullptr, d2h = nullptr;       // copy streams of muon_step_host
+  std::vector<cudaEvent_t> host_events;            // per-chunk ordering events of muon_step_host
 };
 
 std::map<std::pair<int, void*>, std::unique_ptr<Ctx>> g_ctx;
@@ -411,9 +413,9 @@ int get_plan(Ctx& c, const int64_t* shapes, int n, Plan** out) {
   }
   CUDA_TRY(cudaEventCreateWithFlags(&p->wmap_copied, cudaEventDisableTiming));
   c.plans.push_front(std::move(p));
-  if (c.plans.size() > 4) {
+  if (c.plans.size() > 16) {
     CUDA_TRY(cudaStreamSynchronize(c.stream));
-    while (c.plans.size() > 4) c.plans.pop_back();
+    while (c.plans.size() > 16) c.plans.pop_back();
   }
   *out = c.plans.front().get();
   return MUON_OK;
@@ -718,6 +720,7 @@ int muon_step_host(float* const* params, const float* const* grads, float* const
   if ((rc = validate_ptrs((const void* const*)momentum_bufs, n, "momentum_bufs"))) return rc;
   Ctx* c = nullptr;
   if ((rc = get_ctx(stream, &c))) return rc;
+  if ((rc = check_status(*c))) return rc;
   size_t total = 0;
   for (int i = 0; i < n; ++i) total += align_up((size_t)(shapes[2 * i] * shapes[2 * i + 1]), 64);
   const size_t need = 3 * total * sizeof(float);
@@ -732,31 +735,68 @@ int muon_step_host(float* const* params, const float* const* grads, float* const
     }
     c->stage_cap = need;
   }
+  if (!c->h2d) CUDA_TRY(cudaStreamCreateWithFlags(&c->h2d, cudaStreamNonBlocking));
+  if (!c->d2h) CUDA_TRY(cudaStreamCreateWithFlags(&c->d2h, cudaStreamNonBlocking));
   std::vector<float*> dW(n), dg(n), db(n);
-  size_t off = 0;
-  for (int i = 0; i < n; ++i) {
-    const size_t e = (size_t)(shapes[2 * i] * shapes[2 * i + 1]);
-    dW[i] = c->stage + off;
-    dg[i] = c->stage + total + off;
-    db[i] = c->stage + 2 * total + off;
-    off += align_up(e, 64);
-    CUDA_TRY(cudaMemcpyAsync(dW[i], params[i], e * 4, cudaMemcpyHostToDevice, c->stream));
-    CUDA_TRY(cudaMemcpyAsync(dg[i], grads[i], e * 4, cudaMemcpyHostToDevice, c->stream));
-    CUDA_TRY(cudaMemcpyAsync(db[i], momentum_bufs[i], e * 4, cudaMemcpyHostToDevice, c->stream));
+  {
+    size_t off = 0;
+    for (int i = 0; i < n; ++i) {
+      dW[i] = c->stage + off;
+      dg[i] = c->stage + total + off;
+      db[i] = c->stage + 2 * total + off;
+      off += align_up((size_t)(shapes[2 * i] * shapes[2 * i + 1]), 64);
+    }
   }
-  if ((rc = check_status(*c))) return rc;
-  Plan* plan = nullptr;
-  if ((rc = get_plan(*c, shapes, n, &plan))) return rc;
-  StepIO io{dW.data(), (const float* const*)dg.data(), db.data(), lr, mu, MUON_NS_A, MUON_NS_B, MUON_NS_C,
-            MUON_NS_EPS, ns_steps, 1, 0};
-  if (!plan->small.empty() && (rc = run_small(c, c->stream, plan->small, io, c->status_d))) return rc;
-  for (size_t gi = 0; gi < plan->groups.size(); ++gi)
-    if ((rc = run_group(*c, *plan, gi, io))) return rc;
-  for (int i = 0; i < n; ++i) {
-    const size_t e = (size_t)(shapes[2 * i] * shapes[2 * i + 1]);
-    CUDA_TRY(cudaMemcpyAsync(params[i], dW[i], e * 4, cudaMemcpyDeviceToHost, c->stream));
-    CUDA_TRY(cudaMemcpyAsync(momentum_bufs[i], db[i], e * 4, cudaMemcpyDeviceToHost, c->stream));
+  // Chunks of consecutive matrices: copies in (stream h2d), the step (caller's
+  // stream) and copies out (stream d2h) of different chunks overlap.
+  const size_t chunk_bytes = std::max<size_t>(size_t(64) << 20, need / 8);
+  std::vector<std::pair<int, int>> chunks;
+  for (int i = 0; i < n;) {
+    int j = i;
+    size_t bytes = 0;
+    while (j < n && (j == i || bytes + 12 * (size_t)(shapes[2 * j] * shapes[2 * j + 1]) <= chunk_bytes)) {
+      bytes += 12 * (size_t)(shapes[2 * j] * shapes[2 * j + 1]);
+      ++j;
+    }
+    chunks.push_back({i, j});
+    i = j;
   }
+  while (c->host_events.size() < 2 * chunks.size()) {
+    cudaEvent_t e;
+    CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    c->host_events.push_back(e);
+  }
+  // the step of a chunk must not start before earlier work on the caller's stream
+  cudaEvent_t* ev = c->host_events.data();
+  CUDA_TRY(cudaEventRecord(ev[0], c->stream));
+  CUDA_TRY(cudaStreamWaitEvent(c->h2d, ev[0], 0));
+  for (size_t ci = 0; ci < chunks.size(); ++ci) {
+    const int i0 = chunks[ci].first, i1 = chunks[ci].second;
+    for (int i = i0; i < i1; ++i) {
+      const size_t e = (size_t)(shapes[2 * i] * shapes[2 * i + 1]);
+      CUDA_TRY(cudaMemcpyAsync(dW[i], params[i], e * 4, cudaMemcpyHostToDevice, c->h2d));
+      CUDA_TRY(cudaMemcpyAsync(dg[i], grads[i], e * 4, cudaMemcpyHostToDevice, c->h2d));
+      CUDA_TRY(cudaMemcpyAsync(db[i], momentum_bufs[i], e * 4, cudaMemcpyHostToDevice, c->h2d));
+    }
+    CUDA_TRY(cudaEventRecord(ev[2 * ci], c->h2d));
+    CUDA_TRY(cudaStreamWaitEvent(c->stream, ev[2 * ci], 0));
+    Plan* plan = nullptr;
+    if ((rc = get_plan(*c, shapes + 2 * i0, i1 - i0, &plan))) return rc;
+    // StepIO indexes by the caller's matrix index within this chunk
+    StepIO io{dW.data() + i0, (const float* const*)dg.data() + i0, db.data() + i0, lr, mu, MUON_NS_A, MUON_NS_B,
+              MUON_NS_C, MUON_NS_EPS, ns_steps, 1, 0};
+    if (!plan->small.empty() && (rc = run_small(c, c->stream, plan->small, io, c->status_d))) return rc;
+    for (size_t gi = 0; gi < plan->groups.size(); ++gi)
+      if ((rc = run_group(*c, *plan, gi, io))) return rc;
+    CUDA_TRY(cudaEventRecord(ev[2 * ci + 1], c->stream));
+    CUDA_TRY(cudaStreamWaitEvent(c->d2h, ev[2 * ci + 1], 0));
+    for (int i = i0; i < i1; ++i) {
+      const size_t e = (size_t)(shapes[2 * i] * shapes[2 * i + 1]);
+      CUDA_TRY(cudaMemcpyAsync(params[i], dW[i], e * 4, cudaMemcpyDeviceToHost, c->d2h));
+      CUDA_TRY(cudaMemcpyAsync(momentum_bufs[i], db[i], e * 4, cudaMemcpyDeviceToHost, c->d2h));
+    }
+  }
+  CUDA_TRY(cudaStreamSynchronize(c->d2h));
   CUDA_TRY(cudaStreamSynchronize(c->stream));
   return check_status(*c);
 }
@@ -794,6 +834,9 @@ void muon_release(void) {
     if (c.status_h) cudaFreeHost(c.status_h);
     for (auto& r : c.prof) { cudaEventDestroy(r.a); cudaEventDestroy(r.b); }
     for (auto e : c.event_pool) cudaEventDestroy(e);
+    for (auto e : c.host_events) cudaEventDestroy(e);
+    if (c.h2d) cudaStreamDestroy(c.h2d);
+    if (c.d2h) cudaStreamDestroy(c.d2h);
   }
   g_ctx.clear();
   cudaSetDevice(cur);
