@@ -140,6 +140,8 @@ __global__ void __launch_bounds__(kProThreads) prologue_kernel(const __grid_cons
   __shared__ unsigned last_flag;
   __shared__ double dred[kProThreads / 32];
 
+  griddep_launch_dependents();
+  griddep_wait();
   const int t = blockIdx.x;
   const int mi = find_mat(p, t);
   const ProMat& M = p.mats[mi];
@@ -404,6 +406,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   const uint32_t tmem_base = ctl->tmem_base;
   WaitCtx wc{&ctl->abort_flag, p.status, p.wait_limit_ns, mapa_shared(&ctl->abort_flag, rank ^ 1u)};
   bool aborted = false;
+  // set-up above overlaps the previous launch; its outputs are read only below
+  griddep_launch_dependents();
+  griddep_wait();
   // tiles of this cluster and their 64-column slices, in processing order
   const int my_tiles = cid < p.total_tiles ? (p.total_tiles - cid + ncl - 1) / ncl : 0;
   const int my_slices = 4 * my_tiles;
@@ -795,6 +800,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_small_kernel(const __grid
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  griddep_launch_dependents();
+  griddep_wait();
 
   // ---- momentum, norm, X0 (bf16) into shared memory; zero padding included.
   // Each thread issues all loads of a batch before any store (one CTA per SM
@@ -1113,6 +1120,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_small_kernel(const __grid
 
 // ======================================================= ns_steps == 0 ===
 __global__ void apply_x0_kernel(const __grid_constant__ ApplyArgs p) {
+  griddep_wait();
   const int mi = blockIdx.y;
   if (mi >= p.nmats) return;
   const OutMat& O = p.out[mi];

@@ -253,6 +253,25 @@ int encode_class_maps(CUtensorMap* m, char* base, const ClassDesc& cd) {
   return MUON_OK;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous launch on the stream drains; it calls griddepcontrol.wait
+// before touching anything the previous launch wrote.
+template <class Args>
+cudaError_t launch_pdl(void (*kernel)(Args), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       const Args& args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args);
+}
+
 // One NS-phase launch: persistent clusters of two CTAs (one CTA per SM).
 cudaError_t launch_gemm(cudaStream_t stream, const GemmArgs& args, int sm_count) {
   const int pairs = std::max(1, std::min(args.total_tiles, sm_count / 2));
@@ -261,13 +280,15 @@ cudaError_t launch_gemm(cudaStream_t stream, const GemmArgs& args, int sm_count)
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = kGemmSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   switch (args.mode) {
     case kModeGram: return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false>, args);
     case kModePoly: return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModePoly, false>, args);
@@ -534,7 +555,7 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
       }
     }
     int rc = launch(c, MUON_KIND_PROLOGUE,
-                    [&] { prologue_kernel<<<g.pro_tiles, kProThreads, 0, c.stream>>>(*pa); });
+                    [&] { launch_pdl(prologue_kernel, dim3(g.pro_tiles), dim3(kProThreads), 0, c.stream, *pa); });
     if (rc) return rc;
   }
 
@@ -565,7 +586,7 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
         aa->lp[cd.mats[b]] = cd.lp;
       }
     return launch(c, MUON_KIND_APPLY_X0,
-                  [&] { apply_x0_kernel<<<dim3(64, nm), 256, 0, c.stream>>>(*aa); });
+                  [&] { launch_pdl(apply_x0_kernel, dim3(64, nm), dim3(256), 0, c.stream, *aa); });
   }
 
   int rc0 = update_wmaps(c, plan, gidx, io);
@@ -631,7 +652,7 @@ int run_small(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& small, co
       m.vec = (d.n % 4 == 0) && aligned16(m.g) && aligned16(m.w) && (!m.buf || aligned16(m.buf));
       m.lp = round_up(d.l, 64);
     }
-    auto go = [&] { ns_small_kernel<<<nm, kSmallThreads, kSmallSmem, stream>>>(*sa); };
+    auto go = [&] { launch_pdl(ns_small_kernel, dim3(nm), dim3(kSmallThreads), kSmallSmem, stream, *sa); };
     if (c) {
       int rc = launch(*c, MUON_KIND_SMALL, go);
       if (rc) return rc;
@@ -979,8 +1000,7 @@ int noalloc_launch(cudaStream_t stream, char* base, const Plan& plan, const Step
       aa->x[gi] = pm.x;
       aa->lp[gi] = cd.lp;
     }
-  prologue_kernel<<<g.pro_tiles, kProThreads, 0, stream>>>(*pa);
-  CUDA_TRY(cudaGetLastError());
+  CUDA_TRY(launch_pdl(prologue_kernel, dim3(g.pro_tiles), dim3(kProThreads), 0, stream, *pa));
   g_launches.fetch_add(1);
 
   if (io.ns_steps == 0) {
@@ -988,8 +1008,7 @@ int noalloc_launch(cudaStream_t stream, char* base, const Plan& plan, const Step
     aa->lr = io.lr;
     aa->assign = 0;
     aa->nmats = nm;
-    apply_x0_kernel<<<dim3(64, nm), 256, 0, stream>>>(*aa);
-    CUDA_TRY(cudaGetLastError());
+    CUDA_TRY(launch_pdl(apply_x0_kernel, dim3(64, nm), dim3(256), 0, stream, *aa));
     g_launches.fetch_add(1);
     return MUON_OK;
   }

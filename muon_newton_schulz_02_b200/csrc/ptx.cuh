@@ -146,6 +146,15 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bo
   return r != 0;
 }
 
+// ------------------------------------------- programmatic dependent launch ---
+// Wait until the grids this launch depends on have completed and their memory
+// is visible (no-op when the launch has no programmatic dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next launch on the stream to be scheduled before this grid ends.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------ cluster (CTA pair) ---
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
