@@ -11,6 +11,10 @@
 //                       UPDATE  X' = a*s*X + s*(B X)       (last step: W -= lr*X')
 //                     s = 1/(||G||_F+eps) on the first iteration, 1 afterwards,
 //                     so the listing's normalisation is folded into epilogues.
+//                     (256 x 256 output tiles per cluster of two CTAs,
+//                     tcgen05.mma.cta_group::2; a template per phase.)
+//   ns_small_kernel   the whole step of a small matrix (short side <= 128,
+//                     long side <= 512) in one CTA, everything on chip.
 //   apply_x0_kernel   ns_steps == 0: W -= lr * s * X0.
 #pragma once
 
@@ -47,7 +51,6 @@ constexpr uint32_t kStageABytes = kBM * kBK * 2;     // 16 KB
 constexpr uint32_t kStageBBytes = kBNh * kBK * 2;    // 16 KB
 constexpr uint32_t kStageBytes = kStageABytes + kStageBBytes;
 constexpr uint32_t kSliceBytes = kBM * 64 * 2;       // 16 KB: 128 rows x 64 cols bf16 (one TMA box)
-constexpr uint32_t kChunkBytes = kSliceBytes;
 constexpr uint32_t kSmemDataBytes = kStages * kStageBytes + 4 * kSliceBytes;
 constexpr uint32_t kSmemCtrlBytes = 256;
 constexpr uint32_t kGemmSmemBytes = kSmemDataBytes + kSmemCtrlBytes + 1024;  // + alignment slack

@@ -7,6 +7,8 @@
 // box shape.  A step is then 1 + 3*ns_steps kernel launches on the caller's
 // stream: the fused momentum/norm/cast prologue, then per NS iteration one
 // persistent tcgen05 GEMM launch per phase over all matrices of the group.
+// Small matrices (short side <= 128, long side <= 512) need no workspace:
+// one launch of the fused single-CTA kernel runs their whole step.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>

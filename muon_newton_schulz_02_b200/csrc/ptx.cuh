@@ -125,27 +125,6 @@ __device__ __forceinline__ void sleep_ns_bounded(uint64_t ns) {
   while (globaltimer_ns() - t0 < ns) __nanosleep(1000);
 }
 
-// Named barrier among a subset of warps (ids 1..15; 0 is __syncthreads).
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// Named barrier that also returns the AND of `pred` over the participating
-// threads, so a group can agree on one outcome before branching around
-// further barriers.
-__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "barrier.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-
 // ------------------------------------------- programmatic dependent launch ---
 // Wait until the grids this launch depends on have completed and their memory
 // is visible (no-op when the launch has no programmatic dependency).

@@ -1,0 +1,45 @@
+"""bench.py prints one JSON line with the keys its consumers read: checked for
+the reference arm (the CPU oracle, no GPU needed) and for the GPU arm."""
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+BASE_KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+             "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"}
+
+
+def _run(args, timeout):
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT, capture_output=True,
+                         text=True, timeout=timeout)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1, out.stdout
+    return json.loads(lines[0])
+
+
+def test_reference_arm_line():
+    d = _run(["--impl", "reference", "--steps", "2", "--warmup", "3", "--ref-total", "3"], 600)
+    assert BASE_KEYS <= set(d)
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
+    assert d["config"]["workload"] == "gpt2_124m"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+@pytest.mark.gpu
+def test_gpu_arm_line():
+    d = _run(["--steps", "20", "--warmup", "3", "--grad-sets", "2", "--e2e-steps", "2", "--ref-budget", "1"], 900)
+    assert BASE_KEYS | {"roofline", "gpu_launches", "clocks", "kernels"} <= set(d)
+    assert d["n_gpus"] == 1 and d["scaling"] == "weak" and d["higher_is_better"] is True
+    r = d["roofline"]
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and 0 < r["frac"] < 1.5
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
+    assert d["gpu_launches"] == 20 * 16                 # prologue + 3 launches x 5 iterations per step
+    assert d["e2e"]["h2d_bytes_per_step"] > 0 and d["e2e"]["d2h_bytes_per_step"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle"
+    assert set(d["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
