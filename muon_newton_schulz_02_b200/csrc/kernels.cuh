@@ -449,8 +449,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           uint8_t* sb = sa + kStageABytes;
           const uint32_t full_lead = mapa_shared(&ctl->full[stage], 0);
           const bool inject_skip = (p.debug_flags & 1) && it == 0 && kb == 0;
+          // on a diagonal tile of the symmetric phases a CTA's A rows are its B
+          // rows: load them once, the MMA reads both operands from the A buffer
+          const bool same_ab = sym && tc.tm == tc.tn;
           if (!inject_skip) {
-            if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], 2 * kStageBytes);
+            if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], same_ab ? 2 * kStageABytes : 2 * kStageBytes);
             if (kMode != kModeGram && tc.tm > (kb >> 2)) {
               // A rows below the diagonal block: columns [arow, +128) of rows [kb*64, +64), MN-major
               tma_load_3d_pair(sa, tAt, full_lead, arow, kb * kBK, tc.b);
@@ -458,7 +461,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             } else {
               tma_load_3d_pair(sa, tA, full_lead, kb * kBK, arow, tc.b);
             }
-            if (kMode == kModeUpdate || (kMode == kModePoly && tc.tn > (kb >> 2))) {
+            if (same_ab) {
+              // nothing: B is the A block just loaded
+            } else if (kMode == kModeUpdate || (kMode == kModePoly && tc.tn > (kb >> 2))) {
               // B = rows [kb*64, +64) x this CTA's 128 columns, MN-major: two 64-col boxes
               const CUtensorMap* tBm = (kMode == kModeUpdate) ? tB : tAt;
               tma_load_3d_pair(sb, tBm, full_lead, bidx, kb * kBK, tc.b);
@@ -492,10 +497,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           if (!mbar_wait(&ctl->full[stage], phase, wc, kDevTimeoutFull)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * kStageBytes);
-          const uint32_t sb = sa + kStageABytes;
-          // same choice as the producer: operand blocks below the diagonal arrive MN-major
+          // same choices as the producer: diagonal tiles of the symmetric phases
+          // share one operand buffer, blocks below the diagonal arrive MN-major
+          const bool same_ab = sym && tc.tm == tc.tn;
+          const uint32_t sb = same_ab ? sa : sa + kStageABytes;
           const uint32_t a_mn = (kMode != kModeGram && tc.tm > (kb >> 2)) ? 1u : 0u;
-          const uint32_t b_mn = (kMode == kModeUpdate || (kMode == kModePoly && tc.tn > (kb >> 2))) ? 1u : 0u;
+          const uint32_t b_mn = same_ab ? a_mn
+                                : (kMode == kModeUpdate || (kMode == kModePoly && tc.tn > (kb >> 2))) ? 1u : 0u;
           const uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN, a_mn, b_mn);
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
