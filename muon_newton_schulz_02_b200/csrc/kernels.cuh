@@ -559,6 +559,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       for (int g0 = 0; g0 < nbuf; ++g0) prepare(g0);
       bool ok = true;
       int gc = 0;                                  // fp32 chunk counter (final update)
+      int stg_pend = -1;                           // staging buffer an add-reduction may still read
       for (int gs = 0; gs < my_slices && ok; ++gs) {
         const int b = gs % nbuf;
         const uint32_t ph = (uint32_t)((gs / nbuf) & 1);
@@ -588,9 +589,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
                 }
               }
               tma_store_commit();
-              tma_store_wait_read0();
+              tma_store_wait_read1();              // the previous chunk's staging buffer was read
+              if (stg_pend >= 0) mbar_arrive(&ctl->stg_free[stg_pend]);
+              stg_pend = s;
+            } else {
+              if (stg_pend >= 0) { tma_store_wait_read0(); mbar_arrive(&ctl->stg_free[stg_pend]); }
+              stg_pend = -1;
+              mbar_arrive(&ctl->stg_free[s]);
             }
-            mbar_arrive(&ctl->stg_free[s]);
           }
           if (!ok) break;
         }
@@ -617,6 +623,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         prepare(gs + nbuf);
       }
       tma_store_wait_all0();
+      if (stg_pend >= 0) mbar_arrive(&ctl->stg_free[stg_pend]);
       for (int b = 0; b < nbuf; ++b)
         if (pend[b] >= 0) mbar_wait(&ctl->in_full[b], (uint32_t)pend[b], wc, kDevTimeoutDrain);
       aborted = !ok;
