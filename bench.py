@@ -227,7 +227,8 @@ def workload_config(w, args):
     return {"workload": w.name, "matrices": w.n_matrices, "shapes": shapes, "ns_steps": 5,
             "mu": w.mu, "lr": w.lr, "nesterov": True, "grad_sets": args.grad_sets,
             "l2": f"inputs larger than L2: W, g, buf are {w.n_elements * 12 / 1e9:.2f} GB per step",
-            "parallelism": (f"matrices sharded over {args.gpus} ranks + all_gather" if args.sharded
+            "parallelism": (f"matrices sharded over {args.gpus} ranks + all_gather in {args.buckets} run(s)"
+                            if args.sharded
                             else f"independent replicas x{args.gpus}")}
 
 
@@ -263,7 +264,7 @@ def run_ours(args):
 
     def one_step(s):
         if args.sharded and world > 1:
-            mdist.sharded_step(W, gsets[s % args.grad_sets], bufs, lr=w.lr, mu=w.mu)
+            mdist.sharded_step(W, gsets[s % args.grad_sets], bufs, lr=w.lr, mu=w.mu, nbuckets=args.buckets)
         else:
             muon.step(W, gsets[s % args.grad_sets], bufs, lr=w.lr, mu=w.mu, stream=stream)
 
@@ -420,6 +421,8 @@ def main():
     ap.add_argument("--kernel-events", type=int, default=1, help="per-launch CUDA events in a second timed pass")
     ap.add_argument("--sharded", action="store_true",
                     help="split one model's matrices over the ranks (all_gather exchange) instead of replicas")
+    ap.add_argument("--buckets", type=int, default=2,
+                    help="with --sharded: runs per rank whose all_gather overlaps the next run's step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -46,42 +46,73 @@ def _default_local_step(params, grads, bufs, lr, mu, ns_steps):
     step(params, grads, bufs, lr=lr, mu=mu, ns_steps=ns_steps)
 
 
-def sharded_step(params, grads, bufs, lr: float, mu: float, ns_steps: int = 5, group=None, local_step=None):
+def buckets_of(owned, nbuckets: int):
+    """Split every rank's owned indices into `nbuckets` contiguous runs (the
+    same count on every rank; a run may be empty)."""
+    if nbuckets < 1:
+        raise ValueError("nbuckets must be >= 1")
+    out = []
+    for o in owned:
+        q, r = divmod(len(o), nbuckets)
+        runs, pos = [], 0
+        for j in range(nbuckets):
+            n = q + (1 if j < r else 0)
+            runs.append(o[pos:pos + n])
+            pos += n
+        out.append(runs)
+    return out
+
+
+def sharded_step(params, grads, bufs, lr: float, mu: float, ns_steps: int = 5, group=None, local_step=None,
+                 nbuckets: int = 1):
     """One Muon step split across the ranks of `group` (default: the world).
 
     params / grads / bufs: the full, identical lists on every rank (same
     device type on all ranks: CUDA with NCCL, CPU with gloo).  On return every
     rank holds every updated matrix.  `local_step(params, grads, bufs, lr, mu,
-    ns_steps)` updates a sub-list in place; the default is the CUDA step."""
+    ns_steps)` updates a sub-list in place; the default is the CUDA step.
+
+    With nbuckets > 1 each rank's matrices are stepped in that many runs, and
+    the all_gather of a finished run is issued asynchronously, so it overlaps
+    the step of the next run (every rank issues the same collectives in the
+    same order: run j of all ranks goes in the j-th all_gather)."""
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     local_step = local_step or _default_local_step
     shapes = [tuple(p.shape) for p in params]
     owned = partition(shapes, world, ns_steps)
-    mine = owned[rank]
-    if mine:
-        local_step([params[i] for i in mine], [grads[i] for i in mine], [bufs[i] for i in mine], lr, mu, ns_steps)
-    if world == 1:
-        return owned
-    sizes = [sum(params[i].numel() for i in o) for o in owned]
-    chunk = max(sizes)
+    runs = buckets_of(owned, nbuckets)
     dev = params[0].device
-    send = torch.zeros(chunk, dtype=torch.float32, device=dev)
-    off = 0
-    for i in mine:
-        n = params[i].numel()
-        send[off:off + n].copy_(params[i].reshape(-1))
-        off += n
-    recv = [torch.empty(chunk, dtype=torch.float32, device=dev) for _ in range(world)]
-    dist.all_gather(recv, send, group=group)
-    for r in range(world):
-        if r == rank:
+    pending = []
+    for j in range(nbuckets):
+        mine = runs[rank][j]
+        if mine:
+            local_step([params[i] for i in mine], [grads[i] for i in mine], [bufs[i] for i in mine], lr, mu, ns_steps)
+        if world == 1:
             continue
+        chunk = max(sum(params[i].numel() for i in runs[r][j]) for r in range(world))
+        if chunk == 0:
+            continue                                    # identical on every rank: nobody has a run j
+        send = torch.zeros(chunk, dtype=torch.float32, device=dev)
         off = 0
-        for i in owned[r]:
+        for i in mine:
             n = params[i].numel()
-            params[i].reshape(-1).copy_(recv[r][off:off + n])
+            send[off:off + n].copy_(params[i].reshape(-1))
             off += n
+        recv = [torch.empty(chunk, dtype=torch.float32, device=dev) for _ in range(world)]
+        work = dist.all_gather(recv, send, group=group, async_op=nbuckets > 1)
+        pending.append((j, recv, work))
+    for j, recv, work in pending:
+        if work is not None:
+            work.wait()
+        for r in range(world):
+            if r == rank:
+                continue
+            off = 0
+            for i in runs[r][j]:
+                n = params[i].numel()
+                params[i].reshape(-1).copy_(recv[r][off:off + n])
+                off += n
     return owned
 
 

@@ -1,7 +1,8 @@
 """Multi-rank host logic on the CPU with the gloo backend (world size 2 and 3):
 the flop-balanced partition, the sharded step's exchange (every rank ends with
-every updated matrix, equal to a single-process step), and the max-over-ranks
-timing reduction.  The per-rank compute is injected: here the CPU oracle stands
+every updated matrix, equal to a single-process step; in one all_gather or in
+several asynchronous ones overlapping the step), and the max-over-ranks timing
+reduction.  The per-rank compute is injected: here the CPU oracle stands
 in for the CUDA step, which needs a GPU."""
 
 import os
@@ -51,26 +52,37 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, shapes, q):
+def _worker(rank, world, port, shapes, q, nbuckets=1):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         W, g, b = _inputs(shapes=shapes)
-        owned = mdist.sharded_step(W, g, b, lr=0.02, mu=0.95, local_step=_oracle_local_step)
+        owned = mdist.sharded_step(W, g, b, lr=0.02, mu=0.95, local_step=_oracle_local_step, nbuckets=nbuckets)
         t = mdist.max_over_ranks(float(rank) + 0.5)
         q.put((rank, [w.numpy() for w in W], [x.numpy() for x in b], owned, t))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_sharded_step_matches_single_process(world):
+def test_buckets_split_each_rank_into_runs():
+    owned = mdist.partition(SHAPES, 3)
+    for nb in (1, 2, 4, 7):
+        runs = mdist.buckets_of(owned, nb)
+        for o, rr in zip(owned, runs):
+            assert len(rr) == nb and [i for run in rr for i in run] == o
+            assert max(map(len, rr)) - min(map(len, rr)) <= 1
+    with pytest.raises(ValueError):
+        mdist.buckets_of(owned, 0)
+
+
+@pytest.mark.parametrize("world,nbuckets", [(2, 1), (3, 1), (2, 3), (3, 4)])
+def test_sharded_step_matches_single_process(world, nbuckets):
     shapes = SHAPES[4:]                                  # keep the CPU oracle quick
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, shapes, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, shapes, q, nbuckets)) for r in range(world)]
     for p in procs:
         p.start()
     results = [q.get(timeout=300) for _ in range(world)]
