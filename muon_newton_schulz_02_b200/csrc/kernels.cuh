@@ -7,10 +7,12 @@
 //   ns_gemm_kernel    one persistent tcgen05 GEMM launch per NS phase over all
 //                     matrices of a group:
 //                       GRAM    A = s^2 * X X^T            (upper-triangle 256-blocks only)
-//                       POLY    B = b*A + c*(A A)          (upper-triangle 256-blocks only)
-//                       UPDATE  X' = a*s*X + s*(B X)       (last step: W -= lr*X')
+//                       POLY    B' = a*I + b*A + c*(A A)   (upper-triangle 256-blocks only)
+//                       UPDATE  X' = s*(B' X)              (last step: W -= lr*X')
 //                     s = 1/(||G||_F+eps) on the first iteration, 1 afterwards,
-//                     so the listing's normalisation is folded into epilogues.
+//                     so the listing's normalisation is folded into epilogues;
+//                     a*X + B X = (a*I + B) X, so the a*X term rides on the
+//                     diagonal of B' and the update reads no second copy of X.
 //                     (256 x 256 output tiles per cluster of two CTAs,
 //                     tcgen05.mma.cta_group::2; a template per phase.)
 //   ns_small_kernel   the whole step of a small matrix (short side <= 128,
@@ -375,7 +377,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   const uint32_t rank = cluster_ctarank();             // 0: issues the MMAs of the pair
   const int cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
   constexpr bool sym = kMode != kModeUpdate;
-  constexpr bool has_d = kMode != kModeGram;
+  constexpr bool has_d = kMode == kModePoly;           // the epilogue reads an input tile (A)
   constexpr bool final_w = kMode == kModeUpdate && kFinal;
   // Slice buffers: every phase but the final update uses all four 16 KB buffers
   // for input/output slices, with two output stores in flight; the final update
@@ -546,8 +548,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           const int t = cid + (gs >> 2) * ncl, h = gs & 3;
           const TileCoord tc = decode_tile(p, t, sym);
           const GemmClass& C = p.cls[tc.cls];
-          const CUtensorMap* tD = (kMode == kModePoly) ? &p.tmaps[C.tmap_base + kTmA]
-                                                        : &p.tmaps[C.tmap_base + (p.x_in ? kTmX1 : kTmX0)];
+          const CUtensorMap* tD = &p.tmaps[C.tmap_base + kTmA];
           mbar_arrive_expect_tx(&ctl->in_full[b], kSliceBytes);
           tma_load_3d(slice_buf(b), tD, &ctl->in_full[b], tc.tn * kTile + 64 * h,
                       tc.tm * kTile + (int)rank * kBM, tc.b);
@@ -659,13 +660,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(mapa_shared(&ctl->tmem_empty[acc], 0));
         }
-        if (kMode == kModeGram) {
-          const float alpha = s * s;
+        if (kMode != kModePoly) {
+          // Gram: s^2 X X^T.  Update: s (aI + B) X = a s X + s B X, the aI term
+          // carried on the diagonal of the polynomial phase's output.
+          const float alpha = kMode == kModeGram ? s * s : s;
 #pragma unroll
           for (int i = 0; i < 64; ++i) v[i] *= alpha;
         } else {
-          const float wd = (kMode == kModePoly) ? p.b : p.a * s;
-          const float wa = (kMode == kModePoly) ? p.c : s;
+          // b A + c A A
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             uint4 raw = *reinterpret_cast<const uint4*>(dslice + sw128_off((uint32_t)r, (uint32_t)u));
@@ -673,8 +675,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               float2 f = __bfloat1622float2(hv[e]);
-              v[u * 8 + 2 * e] = fmaf(wa, v[u * 8 + 2 * e], wd * f.x);
-              v[u * 8 + 2 * e + 1] = fmaf(wa, v[u * 8 + 2 * e + 1], wd * f.y);
+              v[u * 8 + 2 * e] = fmaf(p.c, v[u * 8 + 2 * e], p.b * f.x);
+              v[u * 8 + 2 * e + 1] = fmaf(p.c, v[u * 8 + 2 * e + 1], p.b * f.y);
+            }
+          }
+          // + a on the diagonal: on a diagonal tile, a warp's 32 rows meet the
+          // slice's columns at 32 consecutive columns starting at dbase, lane by lane
+          const int dbase = (int)rank * kBM + q * 32 - 64 * h;
+          if (tc.tm == tc.tn && (dbase == 0 || dbase == 32)) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j == lane) {
+                if (dbase == 0) v[j] += p.a; else v[32 + j] += p.a;
+              }
             }
           }
         }
