@@ -54,7 +54,12 @@ constexpr uint32_t kStageBBytes = kBNh * kBK * 2;    // 16 KB
 constexpr uint32_t kStageBytes = kStageABytes + kStageBBytes;
 constexpr uint32_t kSliceBytes = kBM * 64 * 2;       // 16 KB: 128 rows x 64 cols bf16 (one TMA box)
 constexpr uint32_t kSmemDataBytes = kStages * kStageBytes + 4 * kSliceBytes;
-constexpr uint32_t kSmemCtrlBytes = 256;
+constexpr uint32_t kSmemCtrlBytes = 512;
+// Final update: fp32 staging ring for the W add-reductions (the two slice
+// buffers plus the two the other phases use for slices 2 and 3), and how many
+// add-reductions stay in flight behind the newest one.
+constexpr int kStgBufs = 4;
+constexpr int kStgLag = 1;
 constexpr uint32_t kGemmSmemBytes = kSmemDataBytes + kSmemCtrlBytes + 1024;  // + alignment slack
 
 // ------------------------------------------------------------ arguments ---
@@ -346,12 +351,15 @@ struct __align__(8) GemmCtrl {
   uint64_t tmem_empty[2];     // even CTA: all 8 epilogue math warps of the pair drained an accumulator
   uint64_t in_full[4];        // DMA -> math: slice buffer set ready (input slice landed, or just free)
   uint64_t out_full[4];       // math -> DMA: slice staged (and input slice consumed)
-  uint64_t stg_full[2];       // math -> DMA: fp32 result chunk staged (final update)
-  uint64_t stg_free[2];       // DMA -> math: fp32 staging buffer free again
+  uint64_t stg_full[kStgBufs];  // math -> DMA: fp32 result chunk staged (final update)
+  uint64_t stg_free[kStgBufs];  // DMA -> math: fp32 staging buffer free again
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
+static_assert(sizeof(GemmCtrl) <= kSmemCtrlBytes, "GemmCtrl does not fit its shared-memory slot");
+static_assert(kGemmSmemBytes <= 232448, "more dynamic shared memory than a CTA may have");
+static_assert(kStgLag >= 1 && kStgLag < kStgBufs, "staging ring");
 
 // One persistent launch per Newton-Schulz phase.  A cluster of two CTAs (one
 // per SM) computes 256 x 256 output tiles with tcgen05.mma.cta_group::2: each
@@ -384,12 +392,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   // uses two, plus two for fp32 staging of the weight update.
   constexpr int nbuf = kFinal ? 2 : 4;
   auto slice_buf = [&](int b) { return b < 2 ? dbuf + b * kSliceBytes : mbuf + (b - 2) * kSliceBytes; };
+  // fp32 staging buffers of the final update (its epilogue reads no input slices)
+  auto stg_buf = [&](int i) { return i < 2 ? mbuf + i * kSliceBytes : dbuf + (i - 2) * kSliceBytes; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl->tmem_full[s], 1);
       mbar_init(&ctl->tmem_empty[s], 8);
+    }
+    for (int s = 0; s < kStgBufs; ++s) {
       mbar_init(&ctl->stg_full[s], 4);
       mbar_init(&ctl->stg_free[s], 1);
     }
@@ -560,7 +572,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       for (int g0 = 0; g0 < nbuf; ++g0) prepare(g0);
       bool ok = true;
       int gc = 0;                                  // fp32 chunk counter (final update)
-      int stg_pend = -1;                           // staging buffer an add-reduction may still read
+      int stg_freed = 0;                           // chunks whose staging buffer was handed back
+      auto release_stg = [&](int upto) {           // hand back the buffers of chunks < upto, in order
+        for (; stg_freed < upto; ++stg_freed) mbar_arrive(&ctl->stg_free[stg_freed % kStgBufs]);
+      };
       for (int gs = 0; gs < my_slices && ok; ++gs) {
         const int b = gs % nbuf;
         const uint32_t ph = (uint32_t)((gs / nbuf) & 1);
@@ -572,10 +587,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           const int mat = C.mat_first + tc.b;
           const OutMat& O = p.out[mat];
           for (int sub = 0; sub < 2 && ok; ++sub, ++gc) {
-            const int s = gc & 1;
-            if (!mbar_wait(&ctl->stg_full[s], (uint32_t)((gc >> 1) & 1), wc, kDevTimeoutEpi)) { ok = false; break; }
+            const int s = gc % kStgBufs;
+            if (!mbar_wait(&ctl->stg_full[s], (uint32_t)((gc / kStgBufs) & 1), wc, kDevTimeoutEpi)) { ok = false; break; }
             if (O.tma) {
-              const uint8_t* S = mbuf + s * kSliceBytes;
+              const uint8_t* S = stg_buf(s);
               const CUtensorMap* wm = &p.wmaps[mat];
               const int gj0 = tc.tn * kTile + 64 * h + 32 * sub;
               if (!O.trans) {
@@ -589,14 +604,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
                   else tma_reduce_add_2d(wm, S + hq * 4096, row0 + 32 * hq, gj0);
                 }
               }
-              tma_store_commit();
-              tma_store_wait_read1();              // the previous chunk's staging buffer was read
-              if (stg_pend >= 0) mbar_arrive(&ctl->stg_free[stg_pend]);
-              stg_pend = s;
+              tma_store_commit();                  // one bulk group per chunk
+              tma_store_wait_read<kStgLag>();      // chunks up to gc - kStgLag have been read
+              release_stg(gc + 1 - kStgLag);
             } else {
-              if (stg_pend >= 0) { tma_store_wait_read0(); mbar_arrive(&ctl->stg_free[stg_pend]); }
-              stg_pend = -1;
-              mbar_arrive(&ctl->stg_free[s]);
+              tma_store_wait_read0();
+              release_stg(gc + 1);
             }
           }
           if (!ok) break;
@@ -624,7 +637,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         prepare(gs + nbuf);
       }
       tma_store_wait_all0();
-      if (stg_pend >= 0) mbar_arrive(&ctl->stg_free[stg_pend]);
+      release_stg(gc);
       for (int b = 0; b < nbuf; ++b)
         if (pend[b] >= 0) mbar_wait(&ctl->in_full[b], (uint32_t)pend[b], wc, kDevTimeoutDrain);
       aborted = !ok;
@@ -695,11 +708,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           const OutMat& O = p.out[mat];
 #pragma unroll
           for (int sub = 0; sub < 2; ++sub, ++gc) {
-            const int sidx = gc & 1;
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(&ctl->stg_free[sidx], (uint32_t)(((gc >> 1) & 1) ^ 1), wc, kDevTimeoutEpi));
+            const int sidx = gc % kStgBufs;
+            ok = __all_sync(0xffffffffu, mbar_wait(&ctl->stg_free[sidx], (uint32_t)(((gc / kStgBufs) & 1) ^ 1), wc,
+                                                   kDevTimeoutEpi));
             if (!ok) break;
-            uint8_t* S = mbuf + sidx * kSliceBytes;
+            uint8_t* S = stg_buf(sidx);
             const float* vv = v + 32 * sub;
             if (O.tma) {
               // -lr*O (or O), 128-byte swizzled; the DMA warp adds it to W in L2
