@@ -262,11 +262,13 @@ def run_ours(args):
 
     from muon_newton_schulz_02_b200 import distributed as mdist
 
+    stepper = muon.PreparedStep(W, bufs, lr=w.lr, mu=w.mu)    # the training-loop call: same W and buf
+
     def one_step(s):
         if args.sharded and world > 1:
             mdist.sharded_step(W, gsets[s % args.grad_sets], bufs, lr=w.lr, mu=w.mu, nbuckets=args.buckets)
         else:
-            muon.step(W, gsets[s % args.grad_sets], bufs, lr=w.lr, mu=w.mu, stream=stream)
+            stepper(gsets[s % args.grad_sets], stream=stream)
 
     for s in range(args.warmup):
         one_step(s)

@@ -16,9 +16,10 @@ from __future__ import annotations
 import ctypes
 import os
 import re
+from array import array
 
 __all__ = [
-    "step", "orthogonalize", "step_host", "step_noalloc", "workspace_size", "sync_status", "last_error", "release",
+    "step", "PreparedStep", "orthogonalize", "step_host", "step_noalloc", "workspace_size", "sync_status", "last_error", "release",
     "profile_enable", "profile_read", "launch_count", "debug_set", "lib", "MuonError", "KINDS",
     "NS_A", "NS_B", "NS_C", "NS_STEPS", "NS_EPS", "LIB_PATH", "header_functions",
 ]
@@ -102,10 +103,6 @@ def _check(rc: int):
         raise MuonError(rc, last_error())
 
 
-def _ptrs(xs):
-    return (ctypes.c_void_p * len(xs))(*[ctypes.c_void_p(p) for p in xs])
-
-
 def _shapes(shapes):
     flat = [int(v) for s in shapes for v in s]
     return (ctypes.c_int64 * len(flat))(*flat)
@@ -120,56 +117,113 @@ def _stream(stream):
     return ctypes.c_void_p(int(stream))
 
 
-def _check_tensors(name, ts, device_kind="cuda"):
+def _bad(name, i, t, device_kind):
+    """The error for a tensor that failed the quick check (slow path, only on failure)."""
     import torch
+    if t.dim() != 2:
+        return ValueError(f"{name}[{i}] must be 2-D (the method is defined for matrices)")
+    if t.dtype != torch.float32 or not t.is_contiguous():
+        return ValueError(f"{name}[{i}] must be contiguous float32")
+    return ValueError(f"{name}[{i}] must live on {device_kind}")
+
+
+def _marshal(name, ts, device_kind="cuda", shapes=None):
+    """One pass over a tensor list: checks (2-D, contiguous fp32, device kind,
+    and equal shapes to `shapes` when given) and returns (pointer array,
+    list of shapes).  The arrays are ctypes views of array('q') buffers."""
+    import torch
+    f32, on_cuda = torch.float32, device_kind == "cuda"
+    ptrs, shp = array("q"), []
     for i, t in enumerate(ts):
-        if t.dim() != 2:
-            raise ValueError(f"{name}[{i}] must be 2-D (the method is defined for matrices)")
-        if t.dtype != torch.float32 or not t.is_contiguous():
-            raise ValueError(f"{name}[{i}] must be contiguous float32")
-        if t.device.type != device_kind:
-            raise ValueError(f"{name}[{i}] must live on {device_kind}")
+        if t.dtype is not f32 or t.is_cuda is not on_cuda or not t.is_contiguous() or t.dim() != 2:
+            raise _bad(name, i, t, device_kind)
+        sz = t.shape
+        if shapes is not None and sz != shapes[i]:
+            raise ValueError(f"matrix {i}: params, grads and bufs shapes differ")
+        shp.append(sz)
+        ptrs.append(t.data_ptr())
+    return (ctypes.c_void_p * len(ptrs)).from_buffer(ptrs), shp
+
+
+def _shape_array(shp):
+    flat = array("q")
+    for r, c in shp:
+        flat.append(r)
+        flat.append(c)
+    return (ctypes.c_int64 * len(flat)).from_buffer(flat)
+
+
+def _check_tensors(name, ts, device_kind="cuda"):
+    _marshal(name, ts, device_kind)
+
+
+def _marshal_step(params, grads, bufs, device_kind="cuda"):
+    n = len(params)
+    if not (len(grads) == n == len(bufs)) or n == 0:
+        raise ValueError("params, grads and bufs must be equally long, non-empty lists")
+    pp, shp = _marshal("params", params, device_kind)
+    gp, _ = _marshal("grads", grads, device_kind, shp)
+    bp, _ = _marshal("bufs", bufs, device_kind, shp)
+    return pp, gp, bp, _shape_array(shp), n
 
 
 def step(params, grads, bufs, lr: float, mu: float, ns_steps: int = NS_STEPS, *, a: float = NS_A,
          b: float = NS_B, c: float = NS_C, eps: float = NS_EPS, nesterov: bool = True, stream=None):
     """One Muon step, in place on ``params`` and ``bufs`` (lists of CUDA fp32 matrices)."""
-    n = len(params)
-    if not (len(grads) == n == len(bufs)) or n == 0:
-        raise ValueError("params, grads and bufs must be equally long, non-empty lists")
-    for name, ts in (("params", params), ("grads", grads), ("bufs", bufs)):
-        _check_tensors(name, ts)
-    for i in range(n):
-        if not (params[i].shape == grads[i].shape == bufs[i].shape):
-            raise ValueError(f"matrix {i}: params, grads and bufs shapes differ")
-    L = lib()
-    rc = L.muon_step_ex(_ptrs([t.data_ptr() for t in params]), _ptrs([t.data_ptr() for t in grads]),
-                        _ptrs([t.data_ptr() for t in bufs]), _shapes([t.shape for t in params]), n,
-                        float(lr), float(mu), int(ns_steps), float(a), float(b), float(c), float(eps),
-                        1 if nesterov else 0, _stream(stream))
+    pp, gp, bp, sh, n = _marshal_step(params, grads, bufs)
+    rc = lib().muon_step_ex(pp, gp, bp, sh, n, float(lr), float(mu), int(ns_steps), float(a), float(b), float(c),
+                            float(eps), 1 if nesterov else 0, _stream(stream))
     _check(rc)
+
+
+class PreparedStep:
+    """A Muon step bound to fixed ``params`` and ``bufs`` (the usual training
+    loop: the same weight and momentum tensors every step).  Their checks and
+    pointer arrays are built once; each call checks and marshals only the
+    gradients, then makes the same ``muon_step_ex`` call as :func:`step`.
+    The bound tensors must keep their storage (no re-allocation) while the
+    object is in use."""
+
+    def __init__(self, params, bufs, lr: float, mu: float, ns_steps: int = NS_STEPS, *, a: float = NS_A,
+                 b: float = NS_B, c: float = NS_C, eps: float = NS_EPS, nesterov: bool = True):
+        n = len(params)
+        if len(bufs) != n or n == 0:
+            raise ValueError("params and bufs must be equally long, non-empty lists")
+        self._pp, self._shp = _marshal("params", params)
+        self._bp, _ = _marshal("bufs", bufs, shapes=self._shp)
+        self._sh = _shape_array(self._shp)
+        self._keep = (list(params), list(bufs))
+        self.n = n
+        self.lr, self.mu, self.ns_steps = float(lr), float(mu), int(ns_steps)
+        self._abc = (float(a), float(b), float(c), float(eps), 1 if nesterov else 0)
+
+    def __call__(self, grads, lr: float = None, stream=None):
+        if len(grads) != self.n:
+            raise ValueError("params, grads and bufs must be equally long, non-empty lists")
+        gp, _ = _marshal("grads", grads, shapes=self._shp)
+        rc = lib().muon_step_ex(self._pp, gp, self._bp, self._sh, self.n, self.lr if lr is None else float(lr),
+                                self.mu, self.ns_steps, *self._abc, _stream(stream))
+        _check(rc)
 
 
 def orthogonalize(G, O=None, ns_steps: int = NS_STEPS, stream=None):
     """O_i = NS5(G_i) for a list of CUDA fp32 matrices; returns the list O."""
     import torch
-    _check_tensors("G", G)
+    gp, shp = _marshal("G", G)
     if O is None:
         O = [torch.empty_like(g) for g in G]
-    _check_tensors("O", O)
-    rc = lib().muon_orthogonalize(_ptrs([t.data_ptr() for t in G]), _ptrs([t.data_ptr() for t in O]),
-                                  _shapes([t.shape for t in G]), len(G), int(ns_steps), _stream(stream))
+    if len(O) != len(G):
+        raise ValueError("G and O must be equally long lists")
+    op, _ = _marshal("O", O, shapes=shp)
+    rc = lib().muon_orthogonalize(gp, op, _shape_array(shp), len(G), int(ns_steps), _stream(stream))
     _check(rc)
     return O
 
 
 def step_host(params, grads, bufs, lr: float, mu: float, ns_steps: int = NS_STEPS, stream=None):
     """Muon step on host (CPU, ideally pinned) fp32 matrices; blocks until done."""
-    for name, ts in (("params", params), ("grads", grads), ("bufs", bufs)):
-        _check_tensors(name, ts, device_kind="cpu")
-    rc = lib().muon_step_host(_ptrs([t.data_ptr() for t in params]), _ptrs([t.data_ptr() for t in grads]),
-                              _ptrs([t.data_ptr() for t in bufs]), _shapes([t.shape for t in params]),
-                              len(params), float(lr), float(mu), int(ns_steps), _stream(stream))
+    pp, gp, bp, sh, n = _marshal_step(params, grads, bufs, device_kind="cpu")
+    rc = lib().muon_step_host(pp, gp, bp, sh, n, float(lr), float(mu), int(ns_steps), _stream(stream))
     _check(rc)
 
 
@@ -177,11 +231,8 @@ def step_noalloc(params, grads, bufs, lr: float, mu: float, ns_steps: int = NS_S
     """muon_step for callers that cannot allocate device memory: the library's
     scratch is a fixed 64 MiB static device array instead of cudaMalloc'd
     workspace (see include/muon.h for the limits)."""
-    for name, ts in (("params", params), ("grads", grads), ("bufs", bufs)):
-        _check_tensors(name, ts)
-    rc = lib().muon_step_noalloc(_ptrs([t.data_ptr() for t in params]), _ptrs([t.data_ptr() for t in grads]),
-                                 _ptrs([t.data_ptr() for t in bufs]), _shapes([t.shape for t in params]),
-                                 len(params), float(lr), float(mu), int(ns_steps), _stream(stream))
+    pp, gp, bp, sh, n = _marshal_step(params, grads, bufs)
+    rc = lib().muon_step_noalloc(pp, gp, bp, sh, n, float(lr), float(mu), int(ns_steps), _stream(stream))
     _check(rc)
 
 

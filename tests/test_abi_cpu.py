@@ -114,3 +114,35 @@ def test_many_matrices_split_into_groups(L):
 def test_launch_count_and_debug_hooks_run_without_gpu(L):
     assert muon.launch_count() == 0
     muon.debug_set(0, 0)
+
+
+def test_binding_marshals_pointers_and_shapes_in_one_pass():
+    import torch
+    P = [torch.zeros(3, 5), torch.zeros(7, 2)]
+    G = [torch.ones(3, 5), torch.ones(7, 2)]
+    B = [torch.full((3, 5), 2.0), torch.full((7, 2), 2.0)]
+    pp, gp, bp, sh, n = muon._marshal_step(P, G, B, device_kind="cpu")
+    assert n == 2 and list(sh) == [3, 5, 7, 2]
+    assert [pp[i] for i in range(2)] == [t.data_ptr() for t in P]
+    assert [gp[i] for i in range(2)] == [t.data_ptr() for t in G]
+    assert [bp[i] for i in range(2)] == [t.data_ptr() for t in B]
+
+
+@pytest.mark.parametrize("bad,msg", [
+    (lambda torch: torch.zeros(3), "2-D"),
+    (lambda torch: torch.zeros(3, 4, dtype=torch.float64), "contiguous float32"),
+    (lambda torch: torch.zeros(4, 3).t(), "contiguous float32"),
+])
+def test_binding_rejects_bad_tensors_before_any_call(bad, msg):
+    import torch
+    t = bad(torch)
+    with pytest.raises(ValueError, match=msg):
+        muon._marshal_step([t], [t], [t], device_kind="cpu")
+    with pytest.raises(ValueError, match="live on cuda"):
+        muon._marshal_step([torch.zeros(3, 4)], [torch.zeros(3, 4)], [torch.zeros(3, 4)])
+    with pytest.raises(ValueError, match="shapes differ"):
+        muon._marshal_step([torch.zeros(3, 4)], [torch.zeros(4, 3)], [torch.zeros(3, 4)], device_kind="cpu")
+    with pytest.raises(ValueError, match="equally long"):
+        muon._marshal_step([torch.zeros(3, 4)], [], [torch.zeros(3, 4)], device_kind="cpu")
+    with pytest.raises(ValueError, match="live on cuda"):
+        muon.PreparedStep([torch.zeros(3, 4)], [torch.zeros(3, 4)], lr=0.02, mu=0.95)

@@ -126,6 +126,30 @@ def test_checkpoint_resume_bitwise():
         assert torch.equal(x, y)
 
 
+def test_prepared_step_matches_step_bitwise():
+    shapes = [(256, 768), (768, 256), (130, 250), (64, 2000)]
+    W, g, b = _inputs(shapes, seed=31)
+    dev = torch.device("cuda:0")
+    runs = []
+    for prepared in (False, True):
+        Wd = [torch.from_numpy(x).to(dev) for x in W]
+        bd = [torch.from_numpy(x).to(dev) for x in b]
+        gsets = [[torch.from_numpy(x).to(dev) * (1 + k) for x in g] for k in range(3)]
+        stepper = muon.PreparedStep(Wd, bd, lr=0.02, mu=0.95) if prepared else None
+        for k in range(3):
+            if prepared:
+                stepper(gsets[k])
+            else:
+                muon.step(Wd, gsets[k], bd, lr=0.02, mu=0.95)
+        torch.cuda.synchronize()
+        assert muon.sync_status() == 0, muon.last_error()
+        runs.append(([x.cpu() for x in Wd], [x.cpu() for x in bd]))
+    for a, c in zip(runs[0][0] + runs[0][1], runs[1][0] + runs[1][1]):
+        assert torch.equal(a, c)
+    with pytest.raises(ValueError, match="shapes differ"):
+        stepper([torch.zeros(3, 3, device=dev)] * len(shapes))
+
+
 def test_host_buffer_entry_point_matches_device_path():
     shapes = [(256, 512), (512, 256)]
     W, g, b = _inputs(shapes, 6)
