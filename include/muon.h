@@ -122,7 +122,9 @@ int muon_step_host(float* const* params, const float* const* grads, float* const
  *     shapes, and their scratch (the muon_workspace_size layout) must fit in
  *     64 MiB minus a 64 KiB table, e.g. one GPT-2-124M layer (4 x 768x768,
  *     768x3072, 3072x768).  Larger requests return MUON_ERR_UNSUPPORTED with
- *     the required size in muon_last_error(); nothing is launched.
+ *     the required size in muon_last_error(); nothing is launched.  Matrices
+ *     the fused kernels run whole (short side <= 128 and long side <= 512,
+ *     or both sides <= 256) use no scratch and do not count.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
@@ -161,7 +163,8 @@ void muon_release(void);
 #define MUON_KIND_UPDATE_APPLY 4
 #define MUON_KIND_APPLY_X0 5
 #define MUON_KIND_SMALL 6        /* fused single-CTA step of small matrices */
-#define MUON_NUM_KINDS 7
+#define MUON_KIND_PAIR 7         /* fused CTA-pair step, 128 < short side <= 256, long side <= 256 */
+#define MUON_NUM_KINDS 8
 
 /* 1: bracket every kernel launch with CUDA events on its stream; 0: stop. */
 int muon_profile_enable(int enable);
@@ -177,7 +180,9 @@ int64_t muon_launch_count(void);
 /* wait_limit_ns: bound of every device-side wait (0 keeps the default, 2 s).
  * flags bit 0: the next GEMM launch skips filling its first pipeline stage,
  * so its MMA warp's wait runs out and the call reports MUON_ERR_TIMEOUT
- * (fault injection that neither faults nor hangs the GPU). */
+ * (fault injection that neither faults nor hangs the GPU).
+ * flags bit 1: the same for the next CTA-pair launch, whose first product is
+ * not issued, so both CTAs' waits for it run out. */
 int muon_debug_set(int flags, int64_t wait_limit_ns);
 
 #ifdef __cplusplus

@@ -17,6 +17,8 @@
 //                     tcgen05.mma.cta_group::2; a template per phase.)
 //   ns_small_kernel   the whole step of a small matrix (short side <= 128,
 //                     long side <= 512) in one CTA, everything on chip.
+//   ns_pair_kernel    the same for 128 < short side <= 256, long side <= 256,
+//                     on a cluster of two CTAs (cta_group::2 products).
 //   apply_x0_kernel   ns_steps == 0: W -= lr * s * X0.
 #pragma once
 
@@ -808,6 +810,7 @@ struct SmallMat {
 
 struct SmallArgs {
   int nmats, ns_steps, nesterov, has_buf, assign;
+  int debug_flags;      // bit 0 (CTA-pair kernel): the first product is not issued
   float mu, eps, a, b, c, lr;
   int* status;
   unsigned long long wait_limit_ns;
@@ -1159,6 +1162,384 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_small_kernel(const __grid
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ======================================== CTA-pair fused step, k <= 256 ===
+// The whole step of a matrix with short side 128 < k <= 256 and long side
+// l <= 256 on one cluster of two CTAs.  CTA r holds rows [128r, 128r + 128) of
+// X (XO, all 256 columns), of A and then B' (AB), and all 256 rows of its own
+// column half of X (XC: the update's N operand).  Every product is one
+// tcgen05.mma.cta_group::2 with M = N = 256 issued by CTA 0:
+//   Gram     A = s^2 X X^T         both operands XO (K-major, K = 256)
+//   poly     B' = aI + bA + cAA     both operands AB (A symmetric)
+//   update   X' = s B' X            AB (K-major) x XC (MN-major, K = X rows)
+// and each CTA's TMEM holds its 128 rows x 256 fp32 columns.  The update's
+// epilogue writes the peer's column half of its rows into the peer's XC
+// through distributed shared memory.  Phases are separated by cluster
+// barriers; both CTAs take every barrier on every path (a CTA whose bounded
+// wait gave up only stops issuing and waiting), so neither can be left behind.
+constexpr int kPairMaxK = 256;
+constexpr int kPairMaxL = 256;
+constexpr uint32_t kPairXC = 256 * 64 * 2;                                   // 32 KB: 64 columns of 256 rows
+constexpr uint32_t kPairSmem = 4 * kSmallChunk + 2 * kPairXC + 4 * kSmallChunk + 256 + 1024;
+
+// Byte offset of element (row, c) in XC: 64-column chunks of 256 rows, 128-byte swizzle.
+__device__ __forceinline__ uint32_t xc_off(uint32_t row, uint32_t c) {
+  return (c >> 6) * kPairXC + row * 128u + ((((c & 63u) >> 3) ^ (row & 7u)) << 4) + (c & 7u) * 2u;
+}
+
+__global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_constant__ SmallArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* XO = smem;                                        // 4 chunks [128][64]
+  uint8_t* XC = XO + 4 * kSmallChunk;                        // 2 chunks [256][64]
+  uint8_t* AB = XC + 2 * kPairXC;                            // 4 chunks [128][64]
+  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(AB + 4 * kSmallChunk);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(abort_flag + 1);     // [0..3] warp partials, [4..5] CTA partials
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
+  const SmallMat& M = p.mats[cluster_id_x()];
+  const int row_base = (int)rank * 128;                      // X rows of this CTA
+  const uint32_t xc_peer = mapa_shared(XC, peer);            // the peer's XC (same layout)
+
+  if (tid == 0) {
+    mbar_init(mma_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(tmem_slot, 256);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  griddep_launch_dependents();
+  griddep_wait();
+
+  // Stores one bf16 quad / element of X row `xr` (global), column j into XO
+  // (local row) and into the XC of the CTA that owns column j's half.
+  auto put_quad = [&](int xr, int j, uint32_t lo, uint32_t hi) {
+    *reinterpret_cast<uint2*>(XO + chunk_off((uint32_t)(xr - row_base), (uint32_t)j)) = make_uint2(lo, hi);
+    const uint32_t off = xc_off((uint32_t)xr, (uint32_t)(j & 127));
+    if ((j >> 7) == (int)rank) *reinterpret_cast<uint2*>(XC + off) = make_uint2(lo, hi);
+    else st_cluster_v2(xc_peer + off, lo, hi);
+  };
+  auto put_one = [&](int xr, int j, __nv_bfloat16 v) {
+    *reinterpret_cast<__nv_bfloat16*>(XO + chunk_off((uint32_t)(xr - row_base), (uint32_t)j)) = v;
+    const uint32_t off = xc_off((uint32_t)xr, (uint32_t)(j & 127));
+    if ((j >> 7) == (int)rank) *reinterpret_cast<__nv_bfloat16*>(XC + off) = v;
+    else st_cluster_u16(xc_peer + off, __bfloat16_as_ushort(v));
+  };
+
+  // ---- momentum, norm partial, X0 (bf16; zero padding included)
+  const float* __restrict__ gp = M.g;
+  float* __restrict__ bp = M.buf;
+  float ss = 0.f;
+  auto load4 = [&](size_t off, int col, int ncols, float (&gv)[4], float (&bv)[4]) {
+    if (M.vec && col + 3 < ncols) {
+      const float4 g4 = __ldg(reinterpret_cast<const float4*>(gp + off));
+      gv[0] = g4.x; gv[1] = g4.y; gv[2] = g4.z; gv[3] = g4.w;
+      if (p.has_buf) {
+        const float4 b4 = *reinterpret_cast<const float4*>(bp + off);
+        bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (col + q < ncols) {
+          gv[q] = gp[off + q];
+          if (p.has_buf) bv[q] = bp[off + q];
+        }
+      }
+    }
+  };
+  auto store4 = [&](size_t off, int col, int ncols, const float (&bv)[4]) {
+    if (!p.has_buf) return;
+    if (M.vec && col + 3 < ncols) {
+      *reinterpret_cast<float4*>(bp + off) = make_float4(bv[0], bv[1], bv[2], bv[3]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (col + q < ncols) bp[off + q] = bv[q];
+    }
+  };
+  if (!M.trans) {
+    // X row i = G row i: a batch is 2 rows x 2 steps of 128 columns
+    for (int i0 = warp; i0 < 128; i0 += 8) {
+      float gv[2][2][4], bv[2][2][4];
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+        for (int cs = 0; cs < 2; ++cs) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) { gv[rr][cs][q] = 0.f; bv[rr][cs][q] = 0.f; }
+          const int i = row_base + i0 + 4 * rr, j = cs * 128 + 4 * lane;
+          if (i < M.m && j < M.n) load4((size_t)i * M.n + j, j, M.n, gv[rr][cs], bv[rr][cs]);
+        }
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+        for (int cs = 0; cs < 2; ++cs) {
+          const int i = row_base + i0 + 4 * rr, j = cs * 128 + 4 * lane;
+          float G[4] = {0.f, 0.f, 0.f, 0.f};
+          if (i < M.m && j < M.n) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (j + q < M.n) G[q] = nesterov_g(gv[rr][cs][q], bv[rr][cs][q], p.mu, p.nesterov, p.has_buf);
+            store4((size_t)i * M.n + j, j, M.n, bv[rr][cs]);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) ss = fmaf(G[q], G[q], ss);
+          put_quad(i, j, pack_bf16x2(G[0], G[1]), pack_bf16x2(G[2], G[3]));
+        }
+    }
+  } else {
+    // X row j = G column j (this CTA's 128 columns of G), X column i = G row i
+    for (int i0 = warp; i0 < kPairMaxL; i0 += 32) {
+      float gv[8][4], bv[8][4];
+      const int j = row_base + 4 * lane;                      // X rows j..j+3
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) { gv[t][q] = 0.f; bv[t][q] = 0.f; }
+        const int i = i0 + 4 * t;
+        if (i < M.m && j < M.n) load4((size_t)i * M.n + j, j, M.n, gv[t], bv[t]);
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int i = i0 + 4 * t;
+        float G[4] = {0.f, 0.f, 0.f, 0.f};
+        if (i < M.m && j < M.n) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (j + q < M.n) G[q] = nesterov_g(gv[t][q], bv[t][q], p.mu, p.nesterov, p.has_buf);
+          store4((size_t)i * M.n + j, j, M.n, bv[t]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          ss = fmaf(G[q], G[q], ss);
+          put_one(j + q, i, __float2bfloat16_rn(G[q]));
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  if (tid == 0) {
+    const float part = red[0] + red[1] + red[2] + red[3];
+    red[4 + rank] = part;
+    st_cluster_u32(mapa_shared(&red[4 + rank], peer), __float_as_uint(part));
+  }
+  fence_async_all();                                         // X0 (local and peer writes) -> tensor core
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const float scale = 1.0f / ((float)sqrt((double)red[4] + (double)red[5]) + p.eps);
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's 32 lanes
+  const int r = warp * 32 + lane;                            // local row owned by this thread
+  const bool leader = rank == 0 && tid == 0;
+  WaitCtx wc{abort_flag, p.status, p.wait_limit_ns, mapa_shared(abort_flag, peer)};
+  bool ok = true;
+  uint32_t phase = 0;
+
+  auto commit_both = [&]() {
+    tc_commit_pair(mapa_shared(mma_bar, 0));
+    tc_commit_pair(mapa_shared(mma_bar, 1));
+  };
+  auto wait_mma = [&]() {
+    bool got = ok && mbar_wait(mma_bar, phase, wc, kDevTimeoutAccum);
+    phase ^= 1u;
+    ok = __syncthreads_and(got) != 0;
+    tc_fence_after();
+  };
+  auto publish = [&]() {                                     // this phase's writes -> the next MMAs
+    fence_async_all();
+    tc_fence_before();
+    cluster_sync_all();
+    tc_fence_after();
+  };
+  // W -= lr * O (or O = result) for X columns cc*32 .. +31 of this thread's
+  // row: staged in AB (free once the update's MMAs are done), then written
+  // in whole 128-byte rows.
+  auto apply_chunk = [&](int cc, const float* v) {
+    float* S = reinterpret_cast<float*>(AB);
+    if (!M.trans) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float4*>(S + r * 32 + ((j ^ (r & 7)) << 2)) =
+            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 32; ++q) S[q * 128 + r] = v[q];
+    }
+    __syncthreads();
+    float4 o[8], w4[8];
+    float* wp[8];
+    bool okw[8], full[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int idx = tid + kSmallThreads * t;
+      int wi, wj;
+      if (!M.trans) {
+        const int row = idx >> 3, qd = idx & 7;
+        wi = row_base + row; wj = cc * 32 + 4 * qd;
+        o[t] = *reinterpret_cast<const float4*>(S + row * 32 + ((qd ^ (row & 7)) << 2));
+      } else {
+        const int c = idx >> 5, qd = idx & 31;
+        wi = cc * 32 + c; wj = row_base + 4 * qd;
+        o[t] = *reinterpret_cast<const float4*>(S + c * 128 + 4 * qd);
+      }
+      okw[t] = wi < M.m && wj < M.n;
+      full[t] = M.vec && wj + 3 < M.n;
+      wp[t] = M.w + (size_t)wi * M.n + wj;
+      w4[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (okw[t] && full[t] && !p.assign) w4[t] = *reinterpret_cast<const float4*>(wp[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (!okw[t]) continue;
+      if (full[t]) {
+        float4 r4 = w4[t];
+        if (p.assign) r4 = o[t];
+        else { r4.x -= p.lr * o[t].x; r4.y -= p.lr * o[t].y; r4.z -= p.lr * o[t].z; r4.w -= p.lr * o[t].w; }
+        *reinterpret_cast<float4*>(wp[t]) = r4;
+      } else {
+        const float ov[4] = {o[t].x, o[t].y, o[t].z, o[t].w};
+        const int wj = (int)((wp[t] - M.w) % M.n);
+        for (int e = 0; e < 4 && wj + e < M.n; ++e) wp[t][e] = p.assign ? ov[e] : wp[t][e] - p.lr * ov[e];
+      }
+    }
+    __syncthreads();
+  };
+
+  const uint32_t idesc_kk = idesc_bf16_f32(256, 256, 0, 0);
+  for (int it = 0; it < p.ns_steps; ++it) {
+    const float s = it == 0 ? scale : 1.0f;
+    const bool last = it == p.ns_steps - 1;
+    // ---- Gram: A = s^2 X X^T
+    const bool inject_skip = (p.debug_flags & 1) && it == 0;
+    if (leader && ok && !inject_skip) {
+      for (int kk = 0; kk < 16; ++kk) {
+        const uint64_t d = smem_desc_sw128(smem_u32(XO) + (kk >> 2) * kSmallChunk + (kk & 3) * 32, 16, 1024);
+        tc_mma_bf16_pair(tmem, d, d, idesc_kk, kk > 0 ? 1u : 0u);
+      }
+      commit_both();
+    }
+    wait_mma();
+#pragma unroll 1
+    for (int c64 = 0; c64 < 4 && ok; ++c64) {
+      float v[64];
+      tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v);
+#pragma unroll
+      for (int q = 0; q < 64; q += 8) {
+        uint4 o;
+        o.x = pack_bf16x2(s * s * v[q], s * s * v[q + 1]);
+        o.y = pack_bf16x2(s * s * v[q + 2], s * s * v[q + 3]);
+        o.z = pack_bf16x2(s * s * v[q + 4], s * s * v[q + 5]);
+        o.w = pack_bf16x2(s * s * v[q + 6], s * s * v[q + 7]);
+        *reinterpret_cast<uint4*>(AB + chunk_off((uint32_t)r, (uint32_t)(c64 * 64 + q))) = o;
+      }
+    }
+    publish();
+    // ---- polynomial: B' = aI + bA + cAA, in place over A
+    if (leader && ok) {
+      for (int kk = 0; kk < 16; ++kk) {
+        const uint64_t d = smem_desc_sw128(smem_u32(AB) + (kk >> 2) * kSmallChunk + (kk & 3) * 32, 16, 1024);
+        tc_mma_bf16_pair(tmem, d, d, idesc_kk, kk > 0 ? 1u : 0u);
+      }
+      commit_both();
+    }
+    wait_mma();
+    const int dcol = row_base + r;                           // this row's diagonal column
+#pragma unroll 1
+    for (int c64 = 0; c64 < 4 && ok; ++c64) {
+      float v[64];
+      tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v);
+#pragma unroll
+      for (int q = 0; q < 64; q += 8) {
+        uint8_t* ap = AB + chunk_off((uint32_t)r, (uint32_t)(c64 * 64 + q));
+        const uint4 araw = *reinterpret_cast<const uint4*>(ap);
+        const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&araw);
+        float o8[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(ah[e]);
+          const int c0 = c64 * 64 + q + 2 * e;
+          o8[2 * e] = fmaf(p.c, v[q + 2 * e], p.b * f.x) + (c0 == dcol ? p.a : 0.f);
+          o8[2 * e + 1] = fmaf(p.c, v[q + 2 * e + 1], p.b * f.y) + (c0 + 1 == dcol ? p.a : 0.f);
+        }
+        *reinterpret_cast<uint4*>(ap) = make_uint4(pack_bf16x2(o8[0], o8[1]), pack_bf16x2(o8[2], o8[3]),
+                                                   pack_bf16x2(o8[4], o8[5]), pack_bf16x2(o8[6], o8[7]));
+      }
+    }
+    publish();
+    // ---- update: X' = s B' X (X read MN-major from XC: K = the 256 rows of X)
+    if (leader && ok) {
+      const uint32_t idesc = idesc_bf16_f32(256, 256, 0, 1);
+      for (int kk = 0; kk < 16; ++kk) {
+        const uint64_t a = smem_desc_sw128(smem_u32(AB) + (kk >> 2) * kSmallChunk + (kk & 3) * 32, 16, 1024);
+        const uint64_t b = smem_desc_sw128(smem_u32(XC) + kk * (16 * 128), kPairXC, 1024);
+        tc_mma_bf16_pair(tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+      }
+      commit_both();
+    }
+    wait_mma();
+#pragma unroll 1
+    for (int c64 = 0; c64 < 4 && ok; ++c64) {
+      float v[64];
+      tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v);
+#pragma unroll
+      for (int i = 0; i < 64; ++i) v[i] *= s;
+      if (last) {
+        apply_chunk(2 * c64, v);
+        apply_chunk(2 * c64 + 1, v + 32);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 64; q += 8) {
+          const int j = c64 * 64 + q;
+          const uint4 o = make_uint4(pack_bf16x2(v[q], v[q + 1]), pack_bf16x2(v[q + 2], v[q + 3]),
+                                     pack_bf16x2(v[q + 4], v[q + 5]), pack_bf16x2(v[q + 6], v[q + 7]));
+          *reinterpret_cast<uint4*>(XO + chunk_off((uint32_t)r, (uint32_t)j)) = o;
+          const uint32_t off = xc_off((uint32_t)(row_base + r), (uint32_t)(j & 127));
+          if ((j >> 7) == (int)rank) *reinterpret_cast<uint4*>(XC + off) = o;
+          else st_cluster_v4(xc_peer + off, o);
+        }
+      }
+    }
+    if (!last) publish();
+  }
+  if (p.ns_steps == 0 && ok) {
+    // O = s * X0 (the listing with an empty loop)
+#pragma unroll 1
+    for (int cc = 0; cc < kPairMaxL / 32; ++cc) {
+      float v[32];
+#pragma unroll
+      for (int q = 0; q < 32; q += 8) {
+        const uint4 xraw = *reinterpret_cast<const uint4*>(XO + chunk_off((uint32_t)r, (uint32_t)(cc * 32 + q)));
+        const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xraw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(xh[e]);
+          v[q + 2 * e] = scale * f.x;
+          v[q + 2 * e + 1] = scale * f.y;
+        }
+      }
+      apply_chunk(cc, v);
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 256);
   }
 }
 

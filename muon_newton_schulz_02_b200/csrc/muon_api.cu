@@ -7,7 +7,8 @@
 // box shape.  A step is then 1 + 3*ns_steps kernel launches on the caller's
 // stream: the fused momentum/norm/cast prologue, then per NS iteration one
 // persistent tcgen05 GEMM launch per phase over all matrices of the group.
-// Small matrices (short side <= 128, long side <= 512) need no workspace:
+// Small matrices (short side <= 128, long side <= 512; or short side <= 256
+// and long side <= 256, run by CTA pairs) need no workspace:
 // one launch of the fused single-CTA kernel runs their whole step.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -98,6 +99,7 @@ struct Plan {
   std::vector<int64_t> shapes;
   std::vector<Group> groups;
   std::vector<MatDesc> small;               // matrices of the fused single-CTA kernel (no workspace)
+  std::vector<MatDesc> pair;                // matrices of the fused CTA-pair kernel (no workspace)
   size_t ws_bytes = 0;
   size_t tmap_bytes = 0;
   void* ws = nullptr;                       // workspace the tensor maps point into
@@ -140,6 +142,7 @@ int build_layout(const int64_t* shapes, int n, Plan& plan) {
     std::vector<MatDesc> big;
     for (const auto& d : all) {
       if (d.k <= kSmallMaxK && round_up(d.l, 64) <= kSmallMaxL) plan.small.push_back(d);
+      else if (d.k <= kPairMaxK && d.l <= kPairMaxL) plan.pair.push_back(d);
       else big.push_back(d);
     }
     all.swap(big);
@@ -346,6 +349,7 @@ int device_setup(int dev) {
     return fail(MUON_ERR_DEVICE, "this library is built for sm_100a (B200); device is sm_" +
                                      std::to_string(prop.major) + std::to_string(prop.minor));
   CUDA_TRY(cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallSmem));
+  CUDA_TRY(cudaFuncSetAttribute(ns_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem));
   CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kGemmSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModePoly, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -667,6 +671,60 @@ int run_small(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& small, co
   return MUON_OK;
 }
 
+// One launch of the fused CTA-pair kernel per kMaxMats matrices (one cluster of two CTAs each).
+int run_pair(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& mats, const StepIO& io, int* status) {
+  for (size_t base = 0; base < mats.size(); base += kMaxMats) {
+    const int nm = (int)std::min<size_t>(kMaxMats, mats.size() - base);
+    auto sa = std::make_unique<SmallArgs>();
+    std::memset(sa.get(), 0, sizeof(SmallArgs));
+    sa->nmats = nm;
+    sa->ns_steps = io.ns_steps;
+    sa->nesterov = io.nesterov;
+    sa->has_buf = io.buf != nullptr;
+    sa->assign = io.assign;
+    sa->mu = io.mu; sa->eps = io.eps; sa->a = io.a; sa->b = io.b; sa->c = io.c; sa->lr = io.lr;
+    sa->status = status;
+    sa->wait_limit_ns = g_wait_limit_ns;
+    for (int i = 0; i < nm; ++i) {
+      const MatDesc& d = mats[base + i];
+      SmallMat& m = sa->mats[i];
+      m.g = io.g[d.user];
+      m.buf = io.buf ? io.buf[d.user] : nullptr;
+      m.w = io.W[d.user];
+      m.m = d.m; m.n = d.n; m.trans = d.trans;
+      m.vec = (d.n % 4 == 0) && aligned16(m.g) && aligned16(m.w) && (!m.buf || aligned16(m.buf));
+      m.lp = kPairMaxL;
+    }
+    if (g_debug_flags & 2) { sa->debug_flags = 1; g_debug_flags &= ~2; }
+    auto go = [&] {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * nm, 1, 1);
+      cfg.blockDim = dim3(kSmallThreads, 1, 1);
+      cfg.dynamicSmemBytes = kPairSmem;
+      cfg.stream = stream;
+      cudaLaunchAttribute attr[2];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[1].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 2;
+      cudaLaunchKernelEx(&cfg, ns_pair_kernel, *sa);
+    };
+    if (c) {
+      int rc = launch(*c, MUON_KIND_PAIR, go);
+      if (rc) return rc;
+    } else {
+      go();
+      CUDA_TRY(cudaGetLastError());
+      g_launches.fetch_add(1);
+    }
+  }
+  return MUON_OK;
+}
+
 int validate_common(const int64_t* shapes, int n, int ns_steps) {
   if (!shapes) return fail(MUON_ERR_INVALID_ARG, "shapes is null");
   if (n <= 0) return fail(MUON_ERR_INVALID_ARG, "n must be > 0");
@@ -691,6 +749,7 @@ int step_impl(const StepIO& io, const int64_t* shapes, int n, void* stream) {
   Plan* plan = nullptr;
   if ((rc = get_plan(*c, shapes, n, &plan))) return rc;
   if (!plan->small.empty() && (rc = run_small(c, c->stream, plan->small, io, c->status_d))) return rc;
+  if (!plan->pair.empty() && (rc = run_pair(c, c->stream, plan->pair, io, c->status_d))) return rc;
   for (size_t gi = 0; gi < plan->groups.size(); ++gi)
     if ((rc = run_group(*c, *plan, gi, io))) return rc;
   return MUON_OK;
@@ -809,6 +868,7 @@ int muon_step_host(float* const* params, const float* const* grads, float* const
     StepIO io{dW.data() + i0, (const float* const*)dg.data() + i0, db.data() + i0, lr, mu, MUON_NS_A, MUON_NS_B,
               MUON_NS_C, MUON_NS_EPS, ns_steps, 1, 0};
     if (!plan->small.empty() && (rc = run_small(c, c->stream, plan->small, io, c->status_d))) return rc;
+    if (!plan->pair.empty() && (rc = run_pair(c, c->stream, plan->pair, io, c->status_d))) return rc;
     for (size_t gi = 0; gi < plan->groups.size(); ++gi)
       if ((rc = run_group(*c, *plan, gi, io))) return rc;
     CUDA_TRY(cudaEventRecord(ev[2 * ci + 1], c->stream));
@@ -1076,10 +1136,9 @@ extern "C" int muon_step_noalloc(float* const* params, const float* const* grads
   CUDA_TRY(cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev));
   StepIO io{params, grads, momentum_bufs, lr, mu, MUON_NS_A, MUON_NS_B, MUON_NS_C, MUON_NS_EPS, ns_steps, 1, 0};
   int* status = (int*)((char*)base + kNoAllocBytes - 256);
-  if (!plan.small.empty()) {
-    CUDA_TRY(cudaMemsetAsync(status, 0, 256, (cudaStream_t)stream));
-    if ((rc = run_small(nullptr, (cudaStream_t)stream, plan.small, io, status))) return rc;
-  }
+  if (!plan.small.empty() || !plan.pair.empty()) CUDA_TRY(cudaMemsetAsync(status, 0, 256, (cudaStream_t)stream));
+  if (!plan.small.empty() && (rc = run_small(nullptr, (cudaStream_t)stream, plan.small, io, status))) return rc;
+  if (!plan.pair.empty() && (rc = run_pair(nullptr, (cudaStream_t)stream, plan.pair, io, status))) return rc;
   if (plan.groups.empty()) return MUON_OK;
   return noalloc_launch((cudaStream_t)stream, (char*)base, plan, io, sm_count);
 }

@@ -63,13 +63,15 @@ def _expect_ws(shapes):
     arrival counters, then per shape class (padded short side kp, long side
     lp, both multiples of 128) two bf16 iterates [B][kp][lp] and two bf16
     [B][kp][kp] matrices, then per-tile norm partials (64x128 tiles) and
-    per-matrix scales, each region rounded to 1 KiB."""
+    per-matrix scales, each region rounded to 1 KiB.  Matrices that a fused
+    kernel runs whole (short side <= 128 and long side <= 512 on one CTA, or
+    short side <= 256 and long side <= 256 on a CTA pair) take none."""
     up = lambda v, a: (v + a - 1) // a * a
     classes = {}
     for r, c in shapes:
         k, l = min(r, c), max(r, c)
-        if k <= 128 and up(l, 64) <= 512:
-            continue                      # fused single-CTA kernel: no workspace
+        if (k <= 128 and up(l, 64) <= 512) or (k <= 256 and l <= 256):
+            continue                      # fused single-CTA or CTA-pair kernel: no workspace
         classes.setdefault((up(k, 128), up(l, 128)), []).append((r, c))
     if not classes:
         return 4096
@@ -93,6 +95,7 @@ def _expect_ws(shapes):
     [(768, 768)] * 4 + [(768, 3072), (3072, 768)],
     [(1, 1), (127, 129), (129, 127), (1000, 300)],
     [(128, 640), (129, 512), (256, 256), (64, 64)],
+    [(256, 256), (200, 256), (257, 256), (256, 257)],
 ])
 def test_workspace_size_matches_layout(L, shapes):
     assert _ws(shapes) == _expect_ws(shapes)

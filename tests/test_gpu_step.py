@@ -162,14 +162,15 @@ def test_host_buffer_entry_point_matches_device_path():
         assert np.array_equal(x.numpy(), y)
 
 
-def test_bounded_wait_timeout_is_reported_and_context_survives():
-    shapes = [(256, 256)]
+@pytest.mark.parametrize("shape,flag", [((384, 384), 1), ((256, 256), 2)], ids=["gemm", "pair"])
+def test_bounded_wait_timeout_is_reported_and_context_survives(shape, flag):
+    shapes = [shape]
     W, g, b = _inputs(shapes, 7)
     dev = torch.device("cuda:0")
     Wd = [torch.as_tensor(x).to(dev) for x in W]
     gd = [torch.as_tensor(x).to(dev) for x in g]
     bd = [torch.as_tensor(x).to(dev) for x in b]
-    muon.debug_set(1, 20_000_000)                     # next GEMM skips its first stage; 20 ms bound
+    muon.debug_set(flag, 20_000_000)                  # next GEMM / pair launch skips a stage; 20 ms bound
     try:
         muon.step(Wd, gd, bd, lr=0.02, mu=0.95)
         assert muon.sync_status() == -5               # MUON_ERR_TIMEOUT

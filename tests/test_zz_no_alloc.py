@@ -72,4 +72,5 @@ def _refused(shapes):
 def test_noalloc_rejects_requests_beyond_its_scratch():
     assert _refused([(4096, 4096)]) == -7             # needs 4 x 32 MiB of iterates and matrices
     assert "static scratch" in muon.last_error()
-    assert _refused([(192, 192)] * 400) == -7         # more matrices than one call takes
+    assert _refused([(320, 320)] * 400) == -7         # more matrices than one call takes
+    assert _refused([(192, 192)] * 400) == 0          # the CTA-pair kernel needs no scratch
