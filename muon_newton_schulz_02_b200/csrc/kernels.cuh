@@ -1181,6 +1181,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_small_kernel(const __grid
 // wait gave up only stops issuing and waiting), so neither can be left behind.
 constexpr int kPairMaxK = 256;
 constexpr int kPairMaxL = 256;
+constexpr int kPairWarps = 8;        // two warpgroups: one per column half of the accumulator
+constexpr int kPairThreads = 32 * kPairWarps;
 constexpr uint32_t kPairXC = 256 * 64 * 2;                                   // 32 KB: 64 columns of 256 rows
 constexpr uint32_t kPairSmem = 4 * kSmallChunk + 2 * kPairXC + 4 * kSmallChunk + 256 + 1024;
 
@@ -1189,7 +1191,7 @@ __device__ __forceinline__ uint32_t xc_off(uint32_t row, uint32_t c) {
   return (c >> 6) * kPairXC + row * 128u + ((((c & 63u) >> 3) ^ (row & 7u)) << 4) + (c & 7u) * 2u;
 }
 
-__global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_constant__ SmallArgs p) {
+__global__ void __launch_bounds__(kPairThreads, 1) ns_pair_kernel(const __grid_constant__ SmallArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* XO = smem;                                        // 4 chunks [128][64]
@@ -1198,7 +1200,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(AB + 4 * kSmallChunk);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  float* red = reinterpret_cast<float*>(abort_flag + 1);     // [0..3] warp partials, [4..5] CTA partials
+  float* red = reinterpret_cast<float*>(abort_flag + 1);     // [0..7] warp partials, [8..9] CTA partials
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
@@ -1269,8 +1271,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_
     }
   };
   if (!M.trans) {
-    // X row i = G row i: a batch is 2 rows x 2 steps of 128 columns
-    for (int i0 = warp; i0 < 128; i0 += 8) {
+    // X row i = G row i: a batch is rows i0 and i0 + 8, 2 steps of 128 columns each
+    for (int i0 = warp; i0 < 128; i0 += 2 * kPairWarps) {
       float gv[2][2][4], bv[2][2][4];
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr)
@@ -1278,14 +1280,14 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_
         for (int cs = 0; cs < 2; ++cs) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) { gv[rr][cs][q] = 0.f; bv[rr][cs][q] = 0.f; }
-          const int i = row_base + i0 + 4 * rr, j = cs * 128 + 4 * lane;
+          const int i = row_base + i0 + kPairWarps * rr, j = cs * 128 + 4 * lane;
           if (i < M.m && j < M.n) load4((size_t)i * M.n + j, j, M.n, gv[rr][cs], bv[rr][cs]);
         }
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
         for (int cs = 0; cs < 2; ++cs) {
-          const int i = row_base + i0 + 4 * rr, j = cs * 128 + 4 * lane;
+          const int i = row_base + i0 + kPairWarps * rr, j = cs * 128 + 4 * lane;
           float G[4] = {0.f, 0.f, 0.f, 0.f};
           if (i < M.m && j < M.n) {
 #pragma unroll
@@ -1299,20 +1301,21 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_
         }
     }
   } else {
-    // X row j = G column j (this CTA's 128 columns of G), X column i = G row i
-    for (int i0 = warp; i0 < kPairMaxL; i0 += 32) {
+    // X row j = G column j (this CTA's 128 columns of G), X column i = G row i;
+    // a batch is 8 rows of G, kPairWarps apart
+    for (int i0 = warp; i0 < kPairMaxL; i0 += 8 * kPairWarps) {
       float gv[8][4], bv[8][4];
       const int j = row_base + 4 * lane;                      // X rows j..j+3
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) { gv[t][q] = 0.f; bv[t][q] = 0.f; }
-        const int i = i0 + 4 * t;
+        const int i = i0 + kPairWarps * t;
         if (i < M.m && j < M.n) load4((size_t)i * M.n + j, j, M.n, gv[t], bv[t]);
       }
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        const int i = i0 + 4 * t;
+        const int i = i0 + kPairWarps * t;
         float G[4] = {0.f, 0.f, 0.f, 0.f};
         if (i < M.m && j < M.n) {
 #pragma unroll
@@ -1333,18 +1336,22 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_
   if (lane == 0) red[warp] = ss;
   __syncthreads();
   if (tid == 0) {
-    const float part = red[0] + red[1] + red[2] + red[3];
-    red[4 + rank] = part;
-    st_cluster_u32(mapa_shared(&red[4 + rank], peer), __float_as_uint(part));
+    float part = 0.f;
+    for (int w = 0; w < kPairWarps; ++w) part += red[w];
+    red[kPairWarps + rank] = part;
+    st_cluster_u32(mapa_shared(&red[kPairWarps + rank], peer), __float_as_uint(part));
   }
   fence_async_all();                                         // X0 (local and peer writes) -> tensor core
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
-  const float scale = 1.0f / ((float)sqrt((double)red[4] + (double)red[5]) + p.eps);
+  const float scale =
+      1.0f / ((float)sqrt((double)red[kPairWarps] + (double)red[kPairWarps + 1]) + p.eps);
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's 32 lanes
-  const int r = warp * 32 + lane;                            // local row owned by this thread
+  const int q4 = warp & 3;                                   // TMEM lane quarter of this warp
+  const int hw = warp >> 2;                                  // column half of the accumulator it reads
+  const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);    // this warp's 32 lanes
+  const int r = q4 * 32 + lane;                              // local row owned by this thread
   const bool leader = rank == 0 && tid == 0;
   WaitCtx wc{abort_flag, p.status, p.wait_limit_ns, mapa_shared(abort_flag, peer)};
   bool ok = true;
@@ -1366,19 +1373,20 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_
     cluster_sync_all();
     tc_fence_after();
   };
-  // W -= lr * O (or O = result) for X columns cc*32 .. +31 of this thread's
-  // row: staged in AB (free once the update's MMAs are done), then written
+  // One apply round: every thread holds 32 values of its row, X columns
+  // 128 hw + 32 j .. +31; the two halves stage theirs in AB (free once the
+  // update's MMAs are done) and all threads write both chunks to W (or O)
   // in whole 128-byte rows.
-  auto apply_chunk = [&](int cc, const float* v) {
-    float* S = reinterpret_cast<float*>(AB);
+  auto apply_round = [&](int j, const float* v) {
+    float* Sh = reinterpret_cast<float*>(AB + hw * 16384);
     if (!M.trans) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<float4*>(S + r * 32 + ((j ^ (r & 7)) << 2)) =
-            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<float4*>(Sh + r * 32 + ((u ^ (r & 7)) << 2)) =
+            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
     } else {
 #pragma unroll
-      for (int q = 0; q < 32; ++q) S[q * 128 + r] = v[q];
+      for (int c = 0; c < 32; ++c) Sh[c * 128 + r] = v[c];
     }
     __syncthreads();
     float4 o[8], w4[8];
@@ -1386,14 +1394,17 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_
     bool okw[8], full[8];
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
-      const int idx = tid + kSmallThreads * t;
+      const int idx = tid + kPairThreads * t;               // 2 staged chunks x 1024 float4
+      const int sel = idx >> 10, loc = idx & 1023;
+      const int cc = 4 * sel + j;                            // 32-column chunk of X
+      const float* S = reinterpret_cast<const float*>(AB + sel * 16384);
       int wi, wj;
       if (!M.trans) {
-        const int row = idx >> 3, qd = idx & 7;
+        const int row = loc >> 3, qd = loc & 7;
         wi = row_base + row; wj = cc * 32 + 4 * qd;
         o[t] = *reinterpret_cast<const float4*>(S + row * 32 + ((qd ^ (row & 7)) << 2));
       } else {
-        const int c = idx >> 5, qd = idx & 31;
+        const int c = loc >> 5, qd = loc & 31;
         wi = cc * 32 + c; wj = row_base + 4 * qd;
         o[t] = *reinterpret_cast<const float4*>(S + c * 128 + 4 * qd);
       }
@@ -1435,7 +1446,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_
     }
     wait_mma();
 #pragma unroll 1
-    for (int c64 = 0; c64 < 4 && ok; ++c64) {
+    for (int jj = 0; jj < 2 && ok; ++jj) {
+      const int c64 = 2 * hw + jj;
       float v[64];
       tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v);
 #pragma unroll
@@ -1460,7 +1472,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_
     wait_mma();
     const int dcol = row_base + r;                           // this row's diagonal column
 #pragma unroll 1
-    for (int c64 = 0; c64 < 4 && ok; ++c64) {
+    for (int jj = 0; jj < 2 && ok; ++jj) {
+      const int c64 = 2 * hw + jj;
       float v[64];
       tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v);
 #pragma unroll
@@ -1493,14 +1506,15 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_
     }
     wait_mma();
 #pragma unroll 1
-    for (int c64 = 0; c64 < 4 && ok; ++c64) {
+    for (int jj = 0; jj < 2 && ok; ++jj) {
+      const int c64 = 2 * hw + jj;
       float v[64];
       tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v);
 #pragma unroll
       for (int i = 0; i < 64; ++i) v[i] *= s;
       if (last) {
-        apply_chunk(2 * c64, v);
-        apply_chunk(2 * c64 + 1, v + 32);
+        apply_round(2 * jj, v);
+        apply_round(2 * jj + 1, v + 32);
       } else {
 #pragma unroll
         for (int q = 0; q < 64; q += 8) {
@@ -1519,7 +1533,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_
   if (p.ns_steps == 0 && ok) {
     // O = s * X0 (the listing with an empty loop)
 #pragma unroll 1
-    for (int cc = 0; cc < kPairMaxL / 32; ++cc) {
+    for (int j = 0; j < 4; ++j) {
+      const int cc = 4 * hw + j;
       float v[32];
 #pragma unroll
       for (int q = 0; q < 32; q += 8) {
@@ -1532,7 +1547,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_pair_kernel(const __grid_
           v[q + 2 * e + 1] = scale * f.y;
         }
       }
-      apply_chunk(cc, v);
+      apply_round(j, v);
     }
   }
   tc_fence_before();

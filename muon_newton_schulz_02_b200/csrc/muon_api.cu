@@ -699,7 +699,7 @@ int run_pair(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& mats, cons
     auto go = [&] {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2 * nm, 1, 1);
-      cfg.blockDim = dim3(kSmallThreads, 1, 1);
+      cfg.blockDim = dim3(kPairThreads, 1, 1);
       cfg.dynamicSmemBytes = kPairSmem;
       cfg.stream = stream;
       cudaLaunchAttribute attr[2];
