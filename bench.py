@@ -21,6 +21,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -63,10 +64,15 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the device code the ncu figures were taken on: the kernel
+    sources with comments and whitespace removed (a comment edit keeps it)."""
     h = hashlib.sha256()
     for f in ("kernels.cuh", "ptx.cuh"):
-        with open(os.path.join(ROOT, "muon_newton_schulz_02_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "muon_newton_schulz_02_b200", "csrc", f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -369,18 +369,18 @@ static_assert(kStgLag >= 1 && kStgLag < kStgBufs, "staging ring");
 // even CTA issues the MMAs over both CTAs' shared memory, and each CTA's TMEM
 // holds its 128 rows x 256 fp32 columns (two accumulators, double-buffered).
 // Roles per CTA: warp 0 TMA producer; warp 1 MMA issuer (even CTA) and TMEM
-// allocator; warp 2 epilogue DMA (loads the epilogue's input slices, issues the
-// TMA stores / add-reductions of its output slices and recycles their
-// buffers); warps 3..6 epilogue math (per 64-column slice: tcgen05.ld -> fp32
-// math -> bf16 -> 128B-swizzled smem).  The math warps hand slices to the DMA
+// allocator; warp 2 epilogue DMA (loads the polynomial epilogue's A slices,
+// issues the TMA stores / add-reductions of the output slices and recycles
+// their buffers); warps 3..6 epilogue math (per 64-column slice: tcgen05.ld ->
+// fp32 math -> bf16 -> 128B-swizzled smem).  The math warps hand slices to the DMA
 // warp through mbarriers and never wait on TMA latency themselves.
 template <int kMode, bool kFinal>
 __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ GemmArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  uint8_t* dbuf = smem + kStages * kStageBytes;        // 2 x 16 KB: epilogue input / output slices
-  uint8_t* mbuf = dbuf + 2 * kSliceBytes;              // 2 x 16 KB: slice buffers 2, 3 / fp32 staging
+  uint8_t* dbuf = smem + kStages * kStageBytes;        // 2 x 16 KB: slice buffers 0, 1 / fp32 staging 2, 3
+  uint8_t* mbuf = dbuf + 2 * kSliceBytes;              // 2 x 16 KB: slice buffers 2, 3 / fp32 staging 0, 1
   GemmCtrl* ctl = reinterpret_cast<GemmCtrl*>(mbuf + 2 * kSliceBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -390,11 +390,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   constexpr bool has_d = kMode == kModePoly;           // the epilogue reads an input tile (A)
   constexpr bool final_w = kMode == kModeUpdate && kFinal;
   // Slice buffers: every phase but the final update uses all four 16 KB buffers
-  // for input/output slices, with two output stores in flight; the final update
-  // uses two, plus two for fp32 staging of the weight update.
+  // for its output slices (the polynomial phase loads its A input into them
+  // first), with two output stores in flight.  The final update stores no bf16
+  // output and reads no input: its two slice buffers carry no data, and all
+  // four buffers serve as its fp32 staging ring for the weight update.
   constexpr int nbuf = kFinal ? 2 : 4;
   auto slice_buf = [&](int b) { return b < 2 ? dbuf + b * kSliceBytes : mbuf + (b - 2) * kSliceBytes; };
-  // fp32 staging buffers of the final update (its epilogue reads no input slices)
+  // fp32 staging buffers of the final update
   auto stg_buf = [&](int i) { return i < 2 ? mbuf + i * kSliceBytes : dbuf + (i - 2) * kSliceBytes; };
 
   if (threadIdx.x == 0) {
