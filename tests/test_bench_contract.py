@@ -43,3 +43,20 @@ def test_gpu_arm_line():
     assert d["e2e"]["h2d_bytes_per_step"] > 0 and d["e2e"]["d2h_bytes_per_step"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle"
     assert set(d["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
+
+
+def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    import shutil
+    sys.path.insert(0, ROOT)
+    import bench
+    csrc = tmp_path / "muon_newton_schulz_02_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in ("kernels.cuh", "ptx.cuh"):
+        shutil.copy(os.path.join(ROOT, "muon_newton_schulz_02_b200", "csrc", f), csrc / f)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash()
+    k = csrc / "kernels.cuh"
+    k.write_text(k.read_text() + "\n// a new comment\n/* and a block\n comment */\n")
+    assert bench.kernel_source_hash() == h0
+    k.write_text(k.read_text() + "\nconstexpr int kUnused = 1;\n")
+    assert bench.kernel_source_hash() != h0
