@@ -634,39 +634,53 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
   return MUON_OK;
 }
 
-// One launch of the fused kernel per kMaxMats small matrices (one CTA each).
+// Arguments of one fused launch (single-CTA or CTA-pair kernel) over
+// mats[base, base + nm); lp is the padded long side each kernel works with.
+std::unique_ptr<SmallArgs> fused_args(const std::vector<MatDesc>& mats, size_t base, int nm, const StepIO& io,
+                                      int* status, bool pair) {
+  auto sa = std::make_unique<SmallArgs>();
+  std::memset(sa.get(), 0, sizeof(SmallArgs));
+  sa->nmats = nm;
+  sa->ns_steps = io.ns_steps;
+  sa->nesterov = io.nesterov;
+  sa->has_buf = io.buf != nullptr;
+  sa->assign = io.assign;
+  sa->mu = io.mu; sa->eps = io.eps; sa->a = io.a; sa->b = io.b; sa->c = io.c; sa->lr = io.lr;
+  sa->status = status;
+  sa->wait_limit_ns = g_wait_limit_ns;
+  for (int i = 0; i < nm; ++i) {
+    const MatDesc& d = mats[base + i];
+    SmallMat& m = sa->mats[i];
+    m.g = io.g[d.user];
+    m.buf = io.buf ? io.buf[d.user] : nullptr;
+    m.w = io.W[d.user];
+    m.m = d.m; m.n = d.n; m.trans = d.trans;
+    m.vec = (d.n % 4 == 0) && aligned16(m.g) && aligned16(m.w) && (!m.buf || aligned16(m.buf));
+    m.lp = pair ? kPairMaxL : round_up(d.l, 64);
+  }
+  return sa;
+}
+
+// Runs `go` as launch kind `kind`: through the context's bookkeeping when
+// there is one, else directly (the no-allocation entry point).
+template <class F>
+int launch_fused(Ctx* c, int kind, F&& go) {
+  if (c) return launch(*c, kind, go);
+  go();
+  CUDA_TRY(cudaGetLastError());
+  g_launches.fetch_add(1);
+  return MUON_OK;
+}
+
+// One launch of the fused single-CTA kernel per kMaxMats small matrices (one CTA each).
 int run_small(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& small, const StepIO& io, int* status) {
   for (size_t base = 0; base < small.size(); base += kMaxMats) {
     const int nm = (int)std::min<size_t>(kMaxMats, small.size() - base);
-    auto sa = std::make_unique<SmallArgs>();
-    std::memset(sa.get(), 0, sizeof(SmallArgs));
-    sa->nmats = nm;
-    sa->ns_steps = io.ns_steps;
-    sa->nesterov = io.nesterov;
-    sa->has_buf = io.buf != nullptr;
-    sa->assign = io.assign;
-    sa->mu = io.mu; sa->eps = io.eps; sa->a = io.a; sa->b = io.b; sa->c = io.c; sa->lr = io.lr;
-    sa->status = status;
-    sa->wait_limit_ns = g_wait_limit_ns;
-    for (int i = 0; i < nm; ++i) {
-      const MatDesc& d = small[base + i];
-      SmallMat& m = sa->mats[i];
-      m.g = io.g[d.user];
-      m.buf = io.buf ? io.buf[d.user] : nullptr;
-      m.w = io.W[d.user];
-      m.m = d.m; m.n = d.n; m.trans = d.trans;
-      m.vec = (d.n % 4 == 0) && aligned16(m.g) && aligned16(m.w) && (!m.buf || aligned16(m.buf));
-      m.lp = round_up(d.l, 64);
-    }
-    auto go = [&] { launch_pdl(ns_small_kernel, dim3(nm), dim3(kSmallThreads), kSmallSmem, stream, *sa); };
-    if (c) {
-      int rc = launch(*c, MUON_KIND_SMALL, go);
-      if (rc) return rc;
-    } else {
-      go();
-      CUDA_TRY(cudaGetLastError());
-      g_launches.fetch_add(1);
-    }
+    auto sa = fused_args(small, base, nm, io, status, false);
+    int rc = launch_fused(c, MUON_KIND_SMALL, [&] {
+      launch_pdl(ns_small_kernel, dim3(nm), dim3(kSmallThreads), kSmallSmem, stream, *sa);
+    });
+    if (rc) return rc;
   }
   return MUON_OK;
 }
@@ -675,28 +689,9 @@ int run_small(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& small, co
 int run_pair(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& mats, const StepIO& io, int* status) {
   for (size_t base = 0; base < mats.size(); base += kMaxMats) {
     const int nm = (int)std::min<size_t>(kMaxMats, mats.size() - base);
-    auto sa = std::make_unique<SmallArgs>();
-    std::memset(sa.get(), 0, sizeof(SmallArgs));
-    sa->nmats = nm;
-    sa->ns_steps = io.ns_steps;
-    sa->nesterov = io.nesterov;
-    sa->has_buf = io.buf != nullptr;
-    sa->assign = io.assign;
-    sa->mu = io.mu; sa->eps = io.eps; sa->a = io.a; sa->b = io.b; sa->c = io.c; sa->lr = io.lr;
-    sa->status = status;
-    sa->wait_limit_ns = g_wait_limit_ns;
-    for (int i = 0; i < nm; ++i) {
-      const MatDesc& d = mats[base + i];
-      SmallMat& m = sa->mats[i];
-      m.g = io.g[d.user];
-      m.buf = io.buf ? io.buf[d.user] : nullptr;
-      m.w = io.W[d.user];
-      m.m = d.m; m.n = d.n; m.trans = d.trans;
-      m.vec = (d.n % 4 == 0) && aligned16(m.g) && aligned16(m.w) && (!m.buf || aligned16(m.buf));
-      m.lp = kPairMaxL;
-    }
+    auto sa = fused_args(mats, base, nm, io, status, true);
     if (g_debug_flags & 2) { sa->debug_flags = 1; g_debug_flags &= ~2; }
-    auto go = [&] {
+    int rc = launch_fused(c, MUON_KIND_PAIR, [&] {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2 * nm, 1, 1);
       cfg.blockDim = dim3(kPairThreads, 1, 1);
@@ -712,15 +707,8 @@ int run_pair(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& mats, cons
       cfg.attrs = attr;
       cfg.numAttrs = 2;
       cudaLaunchKernelEx(&cfg, ns_pair_kernel, *sa);
-    };
-    if (c) {
-      int rc = launch(*c, MUON_KIND_PAIR, go);
-      if (rc) return rc;
-    } else {
-      go();
-      CUDA_TRY(cudaGetLastError());
-      g_launches.fetch_add(1);
-    }
+    });
+    if (rc) return rc;
   }
   return MUON_OK;
 }
