@@ -32,6 +32,10 @@
  *     It is allocated by the first call that needs it (cudaMalloc, which is
  *     not allowed during stream capture: make the first call for a given set
  *     of shapes outside capture) and freed by muon_release().
+ *   - Matrices with short side <= 128 and long side <= 512, or with both
+ *     sides <= 256, run their whole step in one fused launch (one CTA, or
+ *     a cluster of two CTAs, per matrix) and use no workspace; the others
+ *     run as one launch per Newton-Schulz phase over all of them.
  *   - Concurrent calls on different streams use different workspaces; calls
  *     on one stream are serialised by the stream.
  *   - NaN / Inf in the inputs propagate to the outputs; nothing checks them.
