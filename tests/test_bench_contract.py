@@ -60,3 +60,36 @@ def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     assert bench.kernel_source_hash() == h0
     k.write_text(k.read_text() + "\nconstexpr int kUnused = 1;\n")
     assert bench.kernel_source_hash() != h0
+
+
+def test_flop_counts_use_the_symmetric_products_once():
+    sys.path.insert(0, ROOT)
+    import bench
+    from muon_newton_schulz_02_b200 import workloads
+    k, l = 768, 3072
+    per_iter = k * (k + 1) * l + k * k * (k + 1) + 2 * k * k * l      # Gram, polynomial, update
+    assert bench.ns_flops([(k, l)]) == 5 * per_iter == bench.ns_flops([(l, k)])
+    assert bench.ns_flops([(k, l)], ns_steps=2) == 2 * per_iter
+    shapes = workloads.get("gpt2_124m").shapes
+    assert sum(bench.flops_by_kind(shapes).values()) == bench.ns_flops(shapes)
+    assert abs(bench.ns_flops(shapes) / 1.142e12 - 1) < 5e-3              # the step total the docs quote
+
+
+def test_traffic_is_reported_only_for_the_profiled_kernel_source(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    stored = json.load(open(os.path.join(ROOT, "profiles", "ns_gemm_traffic.json")))
+    assert bench.ncu_traffic() == stored["dram_bytes_per_launch_full_workload"]
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
+    assert bench.ncu_traffic() is None
+
+
+def test_peaks_fall_back_when_no_measurement_exists(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, src = bench.load_peaks()
+    assert src == "fallback" and peaks == bench.FALLBACK_PEAKS
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 1.0, "bf16_tflops": 2.0}))
+    peaks, src = bench.load_peaks()
+    assert src == "measured" and peaks["bf16_tflops"] == 2.0
