@@ -153,10 +153,6 @@ def _shape_array(shp):
     return (ctypes.c_int64 * len(flat)).from_buffer(flat)
 
 
-def _check_tensors(name, ts, device_kind="cuda"):
-    _marshal(name, ts, device_kind)
-
-
 def _marshal_step(params, grads, bufs, device_kind="cuda"):
     n = len(params)
     if not (len(grads) == n == len(bufs)) or n == 0:
