@@ -13,6 +13,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -460,6 +461,11 @@ cudaEvent_t pool_event(Ctx& c) {
   return e;
 }
 
+// NVTX range names of the launch kinds (MUON_KIND_*), for timeline tools; the
+// ranges cost nothing when no tool is attached.
+const char* const kKindNames[MUON_NUM_KINDS] = {"muon.prologue", "muon.gram", "muon.poly", "muon.update",
+                                                "muon.update_apply", "muon.apply_x0", "muon.small", "muon.pair"};
+
 template <class F>
 int launch(Ctx& c, int kind, F&& f) {
   cudaEvent_t e0 = nullptr, e1 = nullptr;
@@ -468,7 +474,9 @@ int launch(Ctx& c, int kind, F&& f) {
     e1 = pool_event(c);
     cudaEventRecord(e0, c.stream);
   }
+  nvtxRangePushA(kKindNames[kind]);
   f();
+  nvtxRangePop();
   cudaError_t err = cudaGetLastError();
   if (g_profile) {
     cudaEventRecord(e1, c.stream);
@@ -730,6 +738,10 @@ int validate_ptrs(const void* const* arr, int n, const char* what) {
 }
 
 int step_impl(const StepIO& io, const int64_t* shapes, int n, void* stream) {
+  struct Range {                                     // one NVTX range per library call
+    Range() { nvtxRangePushA("muon.step"); }
+    ~Range() { nvtxRangePop(); }
+  } range;
   Ctx* c = nullptr;
   int rc = get_ctx(stream, &c);
   if (rc) return rc;
