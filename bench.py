@@ -150,14 +150,26 @@ class ClockSampler:
 def cpu_oracle_rate(w, budget_s=12.0):
     """Times the oracle as it stands on a bounded sample of the workload's
     matrices (cycling through its distinct shapes) on the host cores."""
+    import contextlib
+    # all host cores for the BLAS pool, whatever OMP_NUM_THREADS a launcher set
+    # (torchrun sets 1; under it only rank 0 runs this)
+    try:
+        from threadpoolctl import threadpool_info, threadpool_limits
+        pool = threadpool_limits(limits=os.cpu_count() or 1, user_api="blas")
+    except Exception:
+        threadpool_info, pool = None, contextlib.nullcontext()
+    with pool:
+        if threadpool_info is not None:
+            cores = max([d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"] or [1])
+        else:
+            cores = os.cpu_count() or 1
+        return _time_oracle(w, budget_s, cores)
+
+
+def _time_oracle(w, budget_s, cores):
     import numpy as np
     from muon_newton_schulz_02_b200 import workloads
     from oracle import muon_oracle
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"] or [1])
-    except Exception:
-        cores = os.cpu_count() or 1
     idx = workloads.sample_indices(w, per_shape=64)
     order = []
     by_shape = {}
