@@ -109,4 +109,4 @@ def test_reference_arm_under_torchrun_prints_once_from_rank_0():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2
-    assert d["cpu_baseline"]["cores"] == (os.cpu_count() or 1)     # not the launcher's one thread
+    assert d["cpu_baseline"]["cores"] > 1 or (os.cpu_count() or 1) == 1   # not the launcher's one thread
