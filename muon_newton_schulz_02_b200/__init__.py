@@ -128,15 +128,22 @@ def _bad(name, i, t, device_kind):
 
 
 def _marshal(name, ts, device_kind="cuda", shapes=None):
-    """One pass over a tensor list: checks (2-D, contiguous fp32, device kind,
-    and equal shapes to `shapes` when given) and returns (pointer array,
-    list of shapes).  The arrays are ctypes views of array('q') buffers."""
+    """One pass over a tensor list: checks (2-D, contiguous fp32, device kind
+    -- for CUDA, the current device, where the library launches -- and equal
+    shapes to `shapes` when given) and returns (pointer array, list of
+    shapes).  The arrays are ctypes views of array('q') buffers."""
     import torch
     f32, on_cuda = torch.float32, device_kind == "cuda"
+    dev = None
     ptrs, shp = array("q"), []
     for i, t in enumerate(ts):
         if t.dtype is not f32 or t.is_cuda is not on_cuda or not t.is_contiguous() or t.dim() != 2:
             raise _bad(name, i, t, device_kind)
+        if on_cuda:
+            if dev is None:
+                dev = torch.cuda.current_device()
+            if t.get_device() != dev:
+                raise ValueError(f"{name}[{i}] is on cuda:{t.get_device()} but the current device is cuda:{dev}")
         sz = t.shape
         if shapes is not None and sz != shapes[i]:
             raise ValueError(f"matrix {i}: params, grads and bufs shapes differ")
