@@ -3,5 +3,5 @@ see ``oracle.muon_oracle``."""
 
 from .muon_oracle import (  # noqa: F401
     NS_A, NS_B, NS_C, NS_EPS, NS_STEPS,
-    quintic, zeroth_power_via_newtonschulz5, momentum_update, muon_update, muon_step,
+    quintic, newton_schulz5, momentum_update, muon_update,
 )

@@ -59,13 +59,16 @@ def quintic(x, a=NS_A, b=NS_B, c=NS_C):
     return a * x + b * x**3 + c * x**5
 
 
-def zeroth_power_via_newtonschulz5(G, steps=NS_STEPS, eps=NS_EPS,
-                                   a=NS_A, b=NS_B, c=NS_C):
-    """NS5 orthogonalisation of one 2-D matrix, in float64.
+def newton_schulz5(G, steps=NS_STEPS, eps=NS_EPS, a=NS_A, b=NS_B, c=NS_C):
+    """NewtonSchulz5(G): the quintic Newton-Schulz orthogonalisation of one
+    2-D matrix, in float64 (the article's definition sentence names it; its
+    code listing, zeroth_power_via_newtonschulz5, fixes the steps).
 
-    Steps in the order of the listing ("Muon optimizer" section):
-    X = G / (||G||_F + eps); transpose if rows > cols; ``steps`` times
-    {A = X X^T; B = b A + c A A; X = a X + B X}; transpose back.
+    The iteration works on the wide orientation (rows <= cols) of G scaled to
+    unit Frobenius norm (plus eps); each of the ``steps`` rounds forms the
+    Gram matrix A of the iterate, the polynomial B = b A + c A^2 in it, and
+    the next iterate a X + B X.  The result is brought back to G's
+    orientation.
     """
     G = np.asarray(G, dtype=np.float64)
     if G.ndim != 2:
@@ -111,21 +114,8 @@ def muon_update(W, g, buf, lr, mu, steps=NS_STEPS, nesterov=True,
     float32 W, then stored as float32).
     """
     new_buf, G = momentum_update(g, buf, mu, nesterov)
-    O = zeroth_power_via_newtonschulz5(G, steps=steps, eps=eps, a=a, b=b, c=c)
+    O = newton_schulz5(G, steps=steps, eps=eps, a=a, b=b, c=c)
     lr64 = float(np.float32(lr))
     W_new = (np.asarray(W, dtype=np.float32).astype(np.float64) - lr64 * O).astype(np.float32)
     return W_new, new_buf, O
 
-
-def muon_step(params, grads, bufs, lr, mu, steps=NS_STEPS, nesterov=True,
-              eps=NS_EPS, a=NS_A, b=NS_B, c=NS_C):
-    """One Muon step over a list of weight matrices (each one independent).
-
-    Returns (list of W_new, list of buf_new, list of O)."""
-    Ws, bs, Os = [], [], []
-    for W, g, buf in zip(params, grads, bufs):
-        W_new, b_new, O = muon_update(W, g, buf, lr, mu, steps, nesterov, eps, a, b, c)
-        Ws.append(W_new)
-        bs.append(b_new)
-        Os.append(O)
-    return Ws, bs, Os

@@ -106,7 +106,7 @@ def test_repeated_quintic_band_matches_lessons_paragraph():
 def test_repeated_ns_on_matrix_lands_in_band():
     rng = np.random.default_rng(7)
     G = rng.standard_normal((24, 40))
-    O = orc.zeroth_power_via_newtonschulz5(G, steps=60)
+    O = orc.newton_schulz5(G, steps=60)
     s = np.linalg.svd(O, compute_uv=False)
     assert s.min() > 0.675 and s.max() < 1.135
 
@@ -117,7 +117,7 @@ def test_repeated_ns_on_matrix_lands_in_band():
 def test_svd_closed_form_lapack(shape):
     rng = np.random.default_rng(hash(shape) % 2**32)
     G = rng.standard_normal(shape) * 0.3
-    O = orc.zeroth_power_via_newtonschulz5(G)
+    O = orc.newton_schulz5(G)
     assert O.shape == G.shape
     assert _rel(O, _closed_form_lapack(G)) < 1e-12
 
@@ -130,21 +130,21 @@ def test_svd_closed_form_jacobi(shape):
     assert _rel((U * s) @ V.T, G) < 1e-13                  # the Jacobi SVD itself
     x = s / (np.linalg.norm(s) + orc.NS_EPS)
     expect = (U * _p5_scalar(x)) @ V.T
-    assert _rel(orc.zeroth_power_via_newtonschulz5(G), expect) < 1e-12
+    assert _rel(orc.newton_schulz5(G), expect) < 1e-12
 
 
 @pytest.mark.parametrize("steps", [0, 1, 2, 7])
 def test_svd_closed_form_other_step_counts(steps):
     rng = np.random.default_rng(100 + steps)
     G = rng.standard_normal((20, 33))
-    assert _rel(orc.zeroth_power_via_newtonschulz5(G, steps=steps),
+    assert _rel(orc.newton_schulz5(G, steps=steps),
                 _closed_form_lapack(G, steps=steps)) < 1e-12
 
 
 def test_zero_steps_is_normalisation():
     rng = np.random.default_rng(3)
     G = rng.standard_normal((9, 4))
-    O = orc.zeroth_power_via_newtonschulz5(G, steps=0)
+    O = orc.newton_schulz5(G, steps=0)
     assert np.allclose(O, G / (np.linalg.norm(G) + 1e-7), rtol=0, atol=1e-15)
 
 
@@ -164,7 +164,7 @@ def test_diagonal_input_exact_rational(shape):
     G = np.zeros(shape)
     for i, v in enumerate(d):
         G[i, i] = v
-    O = orc.zeroth_power_via_newtonschulz5(G)
+    O = orc.newton_schulz5(G)
     mask = np.zeros(shape, dtype=bool)
     for i, v in enumerate(d):
         mask[i, i] = True
@@ -179,29 +179,29 @@ def test_diagonal_input_exact_rational(shape):
 def test_transpose_symmetry():
     rng = np.random.default_rng(5)
     G = rng.standard_normal((30, 70))
-    assert np.array_equal(orc.zeroth_power_via_newtonschulz5(G.T),
-                          orc.zeroth_power_via_newtonschulz5(G).T)
+    assert np.array_equal(orc.newton_schulz5(G.T),
+                          orc.newton_schulz5(G).T)
 
 
 def test_sign_and_orthogonal_invariance():
     rng = np.random.default_rng(6)
     G = rng.standard_normal((20, 35))
-    O = orc.zeroth_power_via_newtonschulz5(G)
-    assert np.array_equal(orc.zeroth_power_via_newtonschulz5(-G), -O)
+    O = orc.newton_schulz5(G)
+    assert np.array_equal(orc.newton_schulz5(-G), -O)
     Q, _ = np.linalg.qr(rng.standard_normal((20, 20)))
     R, _ = np.linalg.qr(rng.standard_normal((35, 35)))
-    assert _rel(orc.zeroth_power_via_newtonschulz5(Q @ G @ R), Q @ O @ R) < 1e-12
+    assert _rel(orc.newton_schulz5(Q @ G @ R), Q @ O @ R) < 1e-12
 
 
 @pytest.mark.parametrize("scale", [1e-3, 1e3])
 def test_scale_invariance(scale):
     rng = np.random.default_rng(8)
     G = rng.standard_normal((16, 48))
-    a = orc.zeroth_power_via_newtonschulz5(G * scale, eps=0.0)
-    b = orc.zeroth_power_via_newtonschulz5(G, eps=0.0)
+    a = orc.newton_schulz5(G * scale, eps=0.0)
+    b = orc.newton_schulz5(G, eps=0.0)
     assert _rel(a, b) < 1e-12
     # with the default eps the only difference is eps against the norm
-    c = orc.zeroth_power_via_newtonschulz5(G * scale)
+    c = orc.newton_schulz5(G * scale)
     assert _rel(c, b) < 1e-5
 
 
@@ -211,15 +211,15 @@ def test_zero_padding_leaves_block_unchanged(pad):
     G = rng.standard_normal((12, 20))
     P = np.zeros((12 + pad[0], 20 + pad[1]))
     P[:12, :20] = G
-    O = orc.zeroth_power_via_newtonschulz5(P)
-    assert _rel(O[:12, :20], orc.zeroth_power_via_newtonschulz5(G)) < 1e-12
+    O = orc.newton_schulz5(P)
+    assert _rel(O[:12, :20], orc.newton_schulz5(G)) < 1e-12
     assert np.all(O[12:, :] == 0.0) and np.all(O[:, 20:] == 0.0)
 
 
 def test_rank_preserved():
     rng = np.random.default_rng(10)
     G = rng.standard_normal((30, 3)) @ rng.standard_normal((3, 50))
-    s = np.linalg.svd(orc.zeroth_power_via_newtonschulz5(G), compute_uv=False)
+    s = np.linalg.svd(orc.newton_schulz5(G), compute_uv=False)
     assert np.all(s[:3] > 0.5) and np.all(s[3:] < 1e-10)
 
 
@@ -254,10 +254,45 @@ def test_muon_update_mu_zero_is_plain_ns5_and_applies_lr():
     W = (rng.standard_normal((10, 24)) * 0.02).astype(np.float32)
     g = rng.standard_normal((10, 24)).astype(np.float32)
     W_new, b_new, O = orc.muon_update(W, g, np.zeros_like(g), lr=0.02, mu=0.0)
-    assert _rel(O, orc.zeroth_power_via_newtonschulz5(g.astype(np.float64))) < 1e-15
+    assert _rel(O, orc.newton_schulz5(g.astype(np.float64))) < 1e-15
     lr = float(np.float32(0.02))
     assert np.array_equal(W_new, (W.astype(np.float64) - lr * O).astype(np.float32))
     assert np.array_equal(b_new, g)
+
+
+@pytest.mark.parametrize("shape", [(12, 30), (30, 12), (9, 9)])
+@pytest.mark.parametrize("lr", [1.0, 0.02])
+def test_muon_update_apply_matches_svd_closed_form(shape, lr):
+    # With mu = 0 the momentum step passes g through, and with W = 0 the new
+    # weights are -lr times the orthogonalised gradient: W_new must equal
+    # -lr * U p^5(S/(||g||+eps)) V^T, the replacement of G by (a smoothed)
+    # U V^T that the article's definition sentence states, from LAPACK and
+    # from the Jacobi SVD written here.
+    rng = np.random.default_rng(20 + shape[0] + 7 * shape[1])
+    g = rng.standard_normal(shape).astype(np.float32)
+    W0 = np.zeros(shape, dtype=np.float32)
+    W_new, b_new, O = orc.muon_update(W0, g, np.zeros_like(g), lr=lr, mu=0.0)
+    g64 = g.astype(np.float64)
+    lr64 = float(np.float32(lr))
+    U, s, V = _jacobi_svd(g64)
+    x = s / (np.linalg.norm(s) + orc.NS_EPS)
+    for ref in (-lr64 * _closed_form_lapack(g64), -lr64 * (U * _p5_scalar(x)) @ V.T):
+        # W_new is stored in float32: one rounding of each entry
+        assert np.max(np.abs(W_new - ref)) <= 2.0 ** -23 * np.max(np.abs(ref)) * 2
+        assert _rel(W_new, ref) < 1e-6
+    assert np.array_equal(b_new, g)
+
+
+def test_muon_update_apply_adds_to_existing_weights():
+    # W_new - W is the same -lr * O for any W (the update is additive): two
+    # starting points that differ by a constant matrix end up differing by it.
+    rng = np.random.default_rng(31)
+    g = rng.standard_normal((8, 20)).astype(np.float32)
+    W1 = np.zeros((8, 20), dtype=np.float32)
+    W2 = np.full((8, 20), 0.5, dtype=np.float32)       # 0.5 - lr*O stays exact enough in fp32
+    a1, _, _ = orc.muon_update(W1, g, np.zeros_like(g), lr=0.25, mu=0.0)
+    a2, _, _ = orc.muon_update(W2, g, np.zeros_like(g), lr=0.25, mu=0.0)
+    assert np.max(np.abs((a2.astype(np.float64) - 0.5) - a1)) < 1e-6
 
 
 def test_zero_gradient_leaves_weights():
@@ -304,3 +339,32 @@ def test_planted_mistakes_are_caught(mistake):
     except ValueError:
         err = np.inf
     assert err > 1e-3
+
+
+# Planted mistakes in the apply (copies of muon_update with one error each):
+# each must fail the SVD closed-form pin of the apply above.
+def _update_variant(W, g, lr, mistake):
+    O = orc.newton_schulz5(np.asarray(g, np.float64))
+    lr64 = float(np.float32(lr))
+    W64 = np.asarray(W, np.float64)
+    if mistake == "apply_sign":
+        return (W64 + lr64 * O).astype(np.float32)
+    if mistake == "lr_applied_twice":
+        return (W64 - lr64 * lr64 * O).astype(np.float32)
+    if mistake == "apply_transposed":
+        return (W64 - lr64 * O.T).astype(np.float32) if O.shape[0] == O.shape[1] else None
+    raise ValueError(mistake)
+
+
+@pytest.mark.parametrize("mistake", ["apply_sign", "lr_applied_twice", "apply_transposed"])
+def test_planted_apply_mistakes_are_caught(mistake):
+    rng = np.random.default_rng(16)
+    shape = (10, 10) if mistake == "apply_transposed" else (10, 26)
+    g = rng.standard_normal(shape).astype(np.float32)
+    lr = 0.02
+    W_bad = _update_variant(np.zeros(shape, np.float32), g, lr, mistake)
+    ref = -float(np.float32(lr)) * _closed_form_lapack(g.astype(np.float64))
+    assert _rel(W_bad, ref) > 1e-3
+    # and the oracle itself passes the same check
+    W_ok, _, _ = orc.muon_update(np.zeros(shape, np.float32), g, np.zeros_like(g), lr=lr, mu=0.0)
+    assert _rel(W_ok, ref) < 1e-6

@@ -62,7 +62,7 @@ def _rel(O, ref):
 @pytest.fixture(scope="module")
 def case():
     G = np.random.default_rng(0).standard_normal((384, 768)) * 0.02
-    return G, orc.zeroth_power_via_newtonschulz5(G)
+    return G, orc.newton_schulz5(G)
 
 
 def test_bf16_fused_epilogue_error_is_about_one_percent(case):
