@@ -22,6 +22,46 @@ def relF(a, b):
     return float(np.linalg.norm(a - b) / nb) if nb > 0 else float(np.linalg.norm(a - b))
 
 
+# Blockwise bar: every BLOCK x BLOCK block of O must match the oracle's block
+# to REL_BLOCK of that block's norm, plus a floor of FLOOR_BLOCK times the
+# matrix's root-mean-square block norm (so that blocks the oracle leaves near
+# zero, as in a low-rank input, are not judged on their own tiny norm).  A
+# wrong or stale tile is a large error in its own blocks even where it is a
+# small part of the whole matrix's Frobenius norm.
+BLOCK = 128
+REL_BLOCK = 6e-2
+FLOOR_BLOCK = 1e-3
+
+
+def block_errors(O, ref, bs=BLOCK):
+    """Worst ratio err_B / (REL_BLOCK*||ref_B|| + floor) over all blocks (<= 1
+    passes), and the worst block's (row, col) origin."""
+    O = np.asarray(O, np.float64)
+    ref = np.asarray(ref, np.float64)
+    m, n = ref.shape
+    nb = ((m + bs - 1) // bs) * ((n + bs - 1) // bs)
+    floor = FLOOR_BLOCK * np.linalg.norm(ref) / np.sqrt(nb)
+    worst, where = 0.0, (0, 0)
+    for i in range(0, m, bs):
+        for j in range(0, n, bs):
+            rb = ref[i:i + bs, j:j + bs]
+            eb = np.linalg.norm(O[i:i + bs, j:j + bs] - rb)
+            ratio = eb / (REL_BLOCK * np.linalg.norm(rb) + floor) if eb > 0 else 0.0
+            if ratio > worst:
+                worst, where = ratio, (i, j)
+    return worst, where
+
+
+def check_o(O, ref, what=""):
+    """The parity bar on one orthogonalised update: relF <= REL_O and every
+    block within the blockwise bar.  Returns (relF, worst block ratio)."""
+    err = relF(O, ref)
+    assert err <= REL_O, f"{what}: relF(O) = {err:.3e} > {REL_O}"
+    worst, where = block_errors(O, ref)
+    assert worst <= 1.0, f"{what}: block at {where} off by {worst:.2f} x the blockwise bar (relF {err:.3e})"
+    return err, worst
+
+
 def o_from_w(W_old, W_new, lr):
     return (np.asarray(W_old, np.float64) - np.asarray(W_new, np.float64)) / float(np.float32(lr))
 

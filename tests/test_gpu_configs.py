@@ -11,7 +11,7 @@ import muon_newton_schulz_02_b200 as muon
 from muon_newton_schulz_02_b200 import workloads
 from oracle import muon_oracle
 
-from gpu_helpers import REL_BUF, REL_O, check_band, o_from_w, relF
+from gpu_helpers import REL_BUF, check_band, check_o, o_from_w, relF
 
 pytestmark = pytest.mark.gpu
 
@@ -37,8 +37,7 @@ def _run_and_check(w, steps, subset, band_subset=None, svd_device="cpu"):
         for i in subset:
             W_ref, b_ref, O_ref = muon_oracle.muon_update(W_pre[i], g_h[i], b_pre[i], w.lr, w.mu)
             O = o_from_w(W_pre[i], W[i].cpu().numpy(), w.lr)
-            err = relF(O, O_ref)
-            assert err <= REL_O, (w.name, step, i, w.shapes[i], err)
+            check_o(O, O_ref, f"{w.name} step {step} matrix {i} {w.shapes[i]}")
             assert relF(bufs[i].cpu().numpy(), b_ref) <= REL_BUF, (w.name, step, i)
             if band_subset is not None and i in band_subset and step in (0, steps - 1):
                 _, G = muon_oracle.momentum_update(g_h[i], b_pre[i], w.mu)
@@ -51,7 +50,7 @@ def _run_and_check(w, steps, subset, band_subset=None, svd_device="cpu"):
 @pytest.mark.parametrize("n", [256, 512, 1024, 2048, 4096])
 def test_square_sweep_64_matrices(n):
     w = workloads.get(f"square_n{n}")
-    subset = [0, 63] if n <= 1024 else [37]
+    subset = [0, 63]                          # the first and the last matrix of the batch
     _run_and_check(w, 1, subset, band_subset=subset, svd_device="cpu" if n <= 2048 else "cuda:0")
 
 

@@ -11,7 +11,7 @@ import muon_newton_schulz_02_b200 as muon
 from muon_newton_schulz_02_b200 import workloads
 from oracle import muon_oracle
 
-from gpu_helpers import REL_BUF, REL_O, check_band, gpu_step, o_from_w, relF
+from gpu_helpers import REL_BUF, check_band, check_o, gpu_step, o_from_w, relF
 
 pytestmark = pytest.mark.gpu
 
@@ -33,7 +33,7 @@ def _inputs(shapes, seed, gscale=1.0, bscale=0.1):
 def _check_step(W, g, bufs, W_new, b_new, lr=0.02, mu=0.95, **kw):
     for i in range(len(W)):
         W_ref, b_ref, O_ref = muon_oracle.muon_update(W[i], g[i], bufs[i], lr, mu, **kw)
-        assert relF(o_from_w(W[i], W_new[i], lr), O_ref) <= REL_O, f"matrix {i} {W[i].shape}"
+        check_o(o_from_w(W[i], W_new[i], lr), O_ref, f"matrix {i} {W[i].shape}")
         assert relF(b_new[i], b_ref) <= REL_BUF, f"buf {i}"
 
 
@@ -199,8 +199,37 @@ def test_gpt2_124m_ten_steps_against_oracle_subset():
         for j, i in enumerate(sub):
             W_ref, b_ref, O_ref = muon_oracle.muon_update(W_pre[j], g_h[j], b_pre[j], w.lr, w.mu)
             O = o_from_w(W_pre[j], Wd[i].cpu().numpy(), w.lr)
-            assert relF(O, O_ref) <= REL_O, (step, i)
+            check_o(O, O_ref, f"step {step} matrix {i}")
             assert relF(bd[i].cpu().numpy(), b_ref) <= REL_BUF, (step, i)
             if step in (0, w.steps - 1):
                 _, G = muon_oracle.momentum_update(g_h[j], b_pre[j], w.mu)
                 check_band(O, G)
+
+
+def test_non_default_eps():
+    # eps comparable to ||G||_F changes the scale of X0 and so every
+    # singular value the quintic sees; the oracle takes the same eps
+    shapes = [(128, 512), (256, 256), (384, 768)]       # single-CTA, CTA-pair and GEMM paths
+    W, g, b = _inputs(shapes, 9, gscale=0.01, bscale=0.0)
+    for eps in (0.5, 2.0):
+        W_new, b_new = gpu_step(W, g, b, 0.02, 0.95, eps=eps)
+        _check_step(W, g, b, W_new, b_new, eps=eps)
+
+
+@pytest.mark.parametrize("poison", [float("nan"), float("inf")], ids=["nan", "inf"])
+def test_nan_and_inf_propagate(poison):
+    # A non-finite gradient entry makes that matrix's Frobenius norm non-finite,
+    # so its whole update is NaN (the arithmetic carries it; nothing checks);
+    # its momentum buffer is non-finite exactly where the gradient is, and the
+    # other matrices of the same call are unaffected.
+    shapes = [(128, 512), (256, 256), (384, 768), (300, 200)]
+    W, g, b = _inputs(shapes, 10)
+    for bad in range(3):
+        g_bad = [x.copy() for x in g]
+        g_bad[bad][5, 7] = poison
+        W_new, b_new = gpu_step(W, g_bad, b, 0.02, 0.95)
+        assert np.isnan(W_new[bad]).all(), f"matrix {bad}: the update is not NaN everywhere"
+        assert np.array_equal(~np.isfinite(b_new[bad]), ~np.isfinite(g_bad[bad])), f"buf {bad}"
+        ok = [i for i in range(len(shapes)) if i != bad]
+        _check_step([W[i] for i in ok], [g[i] for i in ok], [b[i] for i in ok],
+                    [W_new[i] for i in ok], [b_new[i] for i in ok])
