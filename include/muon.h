@@ -129,17 +129,26 @@ int muon_step_host(float* const* params, const float* const* grads, float* const
  *     the required size in muon_last_error(); nothing is launched.  Matrices
  *     the fused kernels run whole (short side <= 128 and long side <= 512,
  *     or both sides <= 256) use no scratch and do not count.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *   - The array is part of this library's device code: it comes into being
+ *     when that code is loaded on a device, which with CUDA's lazy module
+ *     loading (the default) is the first call of this library on that device
+ *     -- any entry point, this one included.  That first load allocates the
+ *     array and the code, so make one call on each device (this entry point
+ *     with real buffers, or any other) before entering a context that must not
+ *     allocate, and before any stream capture.  Each call then looks up the
+ *     array's device address with the device current, which allocates
+ *     nothing.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind; each call clears what must start at zero.  Calls that overlap
  *     on the GPU (e.g. on two streams) race on it: serialise them.
- *   - The tensor-map table is copied from pageable host memory, so the call
- *     may wait for earlier work on `stream` before returning.
- *   - A bounded wait that runs out inside its kernels stops them cleanly; it
- *     is recorded in the array's status word but not returned here (use
- *     muon_step where device-side error reporting is needed).
+ *   - The call waits for earlier work on `stream` before it launches: it
+ *     reads back the status word its kernels keep in the array.  A bounded
+ *     wait that ran out in the previous call's kernels is returned here as
+ *     MUON_ERR_TIMEOUT (nothing is launched; the word is cleared, so the next
+ *     call runs normally).  The tensor-map table is copied from pageable host
+ *     memory on `stream`.
+ *   - muon_debug_set applies as for muon_step (wait bound, fault injection).
+ *   - After cudaDeviceReset, call muon_release() before the next call.
  */
 int muon_step_noalloc(float* const* params, const float* const* grads, float* const* momentum_bufs,
                       const int64_t* shapes, int n, float lr, float mu, int ns_steps, void* stream);
@@ -154,7 +163,8 @@ int muon_sync_status(void* stream);
 /* Human-readable description of the last error seen by this thread. */
 const char* muon_last_error(void);
 
-/* Frees every cached workspace and staging buffer on every device. */
+/* Frees every cached workspace and staging buffer on every device and
+ * forgets the per-device set-up (call it before cudaDeviceReset). */
 void muon_release(void);
 
 /* ---- measurement hooks (used by the benchmark; off by default) ---------- */

@@ -922,6 +922,7 @@ void muon_release(void) {
     if (c.d2h) cudaStreamDestroy(c.d2h);
   }
   g_ctx.clear();
+  g_dev_ready.clear();                     // a context created after this is set up again
   cudaSetDevice(cur);
 }
 
@@ -972,24 +973,20 @@ namespace {
 
 constexpr size_t kNoAllocBytes = size_t(64) << 20;      // 64 MiB of static scratch per device
 constexpr size_t kNoAllocTableBytes = size_t(64) << 10; // tensor maps + status word at the end
-constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
-// Device address of g_noalloc_scratch, looked up once per device (with that
-// device current) by the first muon_step_noalloc call on it.
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
-
-int noalloc_setup(int dev, void** out) {
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(MUON_ERR_DEVICE, "device index out of range");
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(MUON_ERR_CUDA, std::string("cudaGetSymbolAddress(static scratch): ") + cudaGetErrorString(e));
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+// Device address of g_noalloc_scratch on the current device.  Host code only
+// holds a host-side stand-in under that name, so the address is looked up
+// with the device current -- on every call: once the module is loaded the
+// lookup allocates nothing, and a fresh lookup stays right if the context was
+// torn down and the module loaded again (the array's address can change).
+int noalloc_scratch_address(void** out) {
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p)
+    return fail(MUON_ERR_CUDA, std::string("cudaGetSymbolAddress(static scratch): ") + cudaGetErrorString(e));
+  *out = p;
   return MUON_OK;
 }
 
@@ -1002,9 +999,9 @@ int noalloc_launch(cudaStream_t stream, char* base, const Plan& plan, const Step
   float* scale = (float*)(base + g.off_scale);
   const int nm = (int)g.mats.size();
 
-  // Everything that must start at zero: the norm arrival counters and the status word.
+  // The norm arrival counters must start at zero (the status word was read
+  // and found clear at the start of the call).
   CUDA_TRY(cudaMemsetAsync(base, 0, kTicketBytes, stream));
-  CUDA_TRY(cudaMemsetAsync(status, 0, 256, stream));
 
   // Tensor maps of this call (scratch buffers and the caller's outputs), copied
   // from host memory into the table at the end of the scratch.
@@ -1078,7 +1075,7 @@ int noalloc_launch(cudaStream_t stream, char* base, const Plan& plan, const Step
   ga->wmaps = wmaps;
   ga->scale = scale;
   ga->status = status;
-  ga->wait_limit_ns = 2000000000ull;
+  ga->wait_limit_ns = g_wait_limit_ns;
   ga->nclasses = (int)g.classes.size();
   ga->a = io.a; ga->b = io.b; ga->c = io.c; ga->lr = io.lr;
   ga->assign = 0;
@@ -1096,6 +1093,7 @@ int noalloc_launch(cudaStream_t stream, char* base, const Plan& plan, const Step
       ga->first = it == 0;
       ga->final_apply = (mode == kModeUpdate) && (it == io.ns_steps - 1);
       ga->debug_flags = 0;
+      if (g_debug_flags & 1) { ga->debug_flags = 1; g_debug_flags &= ~1; }
       CUDA_TRY(launch_gemm(stream, *ga, sm_count));
       g_launches.fetch_add(1);
     }
@@ -1131,12 +1129,23 @@ extern "C" int muon_step_noalloc(float* const* params, const float* const* grads
   CUDA_TRY(cudaGetDevice(&dev));
   if ((rc = device_setup(dev))) return rc;
   void* base = nullptr;
-  if ((rc = noalloc_setup(dev, &base))) return rc;
+  if ((rc = noalloc_scratch_address(&base))) return rc;
   int sm_count = 148;
   CUDA_TRY(cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev));
   StepIO io{params, grads, momentum_bufs, lr, mu, MUON_NS_A, MUON_NS_B, MUON_NS_C, MUON_NS_EPS, ns_steps, 1, 0};
+  // The status word at the end of the scratch holds what the kernels of the
+  // previous call on this device recorded: wait for that call, report a
+  // bounded wait that ran out (and clear the word), else go on with it clear.
   int* status = (int*)((char*)base + kNoAllocBytes - 256);
-  if (!plan.small.empty() || !plan.pair.empty()) CUDA_TRY(cudaMemsetAsync(status, 0, 256, (cudaStream_t)stream));
+  int prev = 0;
+  CUDA_TRY(cudaMemcpyAsync(&prev, status, sizeof(int), cudaMemcpyDeviceToHost, (cudaStream_t)stream));
+  CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
+  if (prev != 0) {
+    CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), (cudaStream_t)stream));
+    CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
+    return fail(MUON_ERR_TIMEOUT, "an earlier muon_step_noalloc call gave up on a bounded wait (device code " +
+                                      std::to_string(prev) + "); nothing was launched by this call");
+  }
   if (!plan.small.empty() && (rc = run_small(nullptr, (cudaStream_t)stream, plan.small, io, status))) return rc;
   if (!plan.pair.empty() && (rc = run_pair(nullptr, (cudaStream_t)stream, plan.pair, io, status))) return rc;
   if (plan.groups.empty()) return MUON_OK;
