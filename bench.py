@@ -7,12 +7,21 @@ A step is one Muon update (Nesterov momentum, NS5, W -= lr*O) over every
 matrix of the workload, with inputs resident in HBM.  ``value`` is
 algorithmic NS5 TFLOP/s of the whole job (symmetry of X X^T and A A
 exploited, 5*(k(k+1)l + k^2(k+1) + 2k^2 l) per k x l matrix, k <= l);
-``ms_per_step`` the device time per step.  Under torchrun every rank runs its
-own copy of the workload (independent problems, no collective on the data
-path: weak scaling) and the time is the maximum over ranks.
+``ms_per_step`` the device time per step; under torchrun the time is the
+maximum over ranks.
 
 ``--impl reference`` times the CPU oracle (float64 numpy) on the host cores on
 a bounded sample of the same workload, per the same metric.
+
+Under torchrun (N > 1) the default is the data-parallel step: the ranks split
+one model's matrices (greedy by flops) and exchange the updated weights with
+an all_gather ("scaling": "strong"); ``--replicas`` runs an independent copy
+per rank instead ("scaling": "weak").
+
+The line also carries a ``sweep`` of the 64-matrix square batches
+(n = 1024, 2048, 4096) with the GEMM kernel's throughput per size, so that the
+fraction of the dense bf16 peak on those batches is measured in the same run
+(``--sweep ""`` leaves it out).
 """
 
 from __future__ import annotations
@@ -33,7 +42,10 @@ if ROOT not in sys.path:
 
 METRIC = "Muon NS5 bf16 TFLOP/s (% of B200 tensor peak); ms per GPT-2-124M Muon step"
 UNIT = "TFLOP/s"
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Used only when MEASURED_PEAKS.json is absent: an earlier measurement of a
+# plain copy and of a cuBLAS bf16 GEMM (burst) on this machine's B200s.  There is
+# no sustained GEMM figure without the measurement file.
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
 def ns_flops(shapes, ns_steps=5) -> float:
@@ -147,15 +159,16 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- CPU oracle ---
-def cpu_oracle_rate(w, budget_s=12.0):
+def cpu_oracle_rate(w, budget_s=12.0, threads=None):
     """Times the oracle as it stands on a bounded sample of the workload's
-    matrices (cycling through its distinct shapes) on the host cores."""
+    matrices (cycling through its distinct shapes) on the host cores (all of
+    them, or `threads`)."""
     import contextlib
     # all host cores for the BLAS pool, whatever OMP_NUM_THREADS a launcher set
     # (torchrun sets 1; under it only rank 0 runs this)
     try:
         from threadpoolctl import threadpool_info, threadpool_limits
-        pool = threadpool_limits(limits=os.cpu_count() or 1, user_api="blas")
+        pool = threadpool_limits(limits=threads or os.cpu_count() or 1, user_api="blas")
     except Exception:
         threadpool_info, pool = None, contextlib.nullcontext()
     with pool:
@@ -212,6 +225,7 @@ def run_reference(args):
         return 0
     from muon_newton_schulz_02_b200 import workloads
     w = workloads.get(args.workload)
+    sharded = world > 1 and not args.replicas           # the GPU arm's configuration at this N
     # each step: a bounded sample (at least one matrix), sized so the whole
     # run stays within --ref-total seconds of CPU work
     per_step = args.ref_total / max(1, args.steps + args.warmup)
@@ -228,9 +242,9 @@ def run_reference(args):
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": flops_step / (val * 1e12) * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,0.02) gradients of the GPT-2-124M hidden-matrix shapes)",
-        "config": workload_config(w, args),
+        "config": workload_config(w, args, sharded),
         "cpu_baseline": {k: base[k] for k in ("kind", "cores", "sample")} | {"value": val, "unit": UNIT},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -238,7 +252,7 @@ def run_reference(args):
     return 0
 
 
-def workload_config(w, args):
+def workload_config(w, args, sharded=False):
     shapes = {}
     for s in w.shapes:
         shapes[f"{s[0]}x{s[1]}"] = shapes.get(f"{s[0]}x{s[1]}", 0) + 1
@@ -246,8 +260,104 @@ def workload_config(w, args):
             "mu": w.mu, "lr": w.lr, "nesterov": True, "grad_sets": args.grad_sets,
             "l2": f"inputs larger than L2: W, g, buf are {w.n_elements * 12 / 1e9:.2f} GB per step",
             "parallelism": (f"matrices sharded over {args.gpus} ranks + all_gather in {args.buckets} run(s)"
-                            if args.sharded
-                            else f"independent replicas x{args.gpus}")}
+                            if sharded else f"independent replicas x{args.gpus}")}
+
+
+def pick_peak(peaks, clk, timed_s):
+    """The GEMM peak a kernel is judged against: the burst figure when the
+    timed region is short (under a second) or ran at (nearly) full clock, the
+    sustained figure when a long region settled under the power cap."""
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sust = peaks.get("bf16_tflops_sustained")
+    full_clock = bool(clk) and clk["sm_mhz"] >= 0.95 * clk["sm_max_mhz"]
+    if sust is None or timed_s < 1.0 or full_clock:
+        why = ("no sustained figure" if sust is None else
+               f"timed region {timed_s:.2f} s < 1 s" if timed_s < 1.0 else "median SM clock >= 0.95 of max")
+        return burst, "bf16_tflops (burst: " + why + ")"
+    return float(sust), "bf16_tflops_sustained (timed region >= 1 s below full clock)"
+
+
+def flush_l2(buf):
+    buf.zero_()                      # writes more than the 126 MB L2: evicts every line
+
+
+class StepTimer:
+    """Runs `one_step` K times on `stream` with a CUDA event after every step
+    (the loop total and per-step times from the same events)."""
+
+    def __init__(self, torch, stream):
+        self.torch, self.stream = torch, stream
+
+    def run(self, one_step, steps, start=0):
+        ev = [self.torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        ev[0].record(self.stream)
+        for s in range(steps):
+            one_step(start + s)
+            ev[s + 1].record(self.stream)
+        return ev
+
+    @staticmethod
+    def times(ev):
+        return ev[0].elapsed_time(ev[-1]), [ev[i].elapsed_time(ev[i + 1]) for i in range(len(ev) - 1)]
+
+
+def gemm_roofline(prof, flops, steps, peak):
+    gemm_ms = sum(prof[k][0] for k in ("gram", "poly", "update", "update_apply"))
+    gemm_launches = sum(prof[k][1] for k in ("gram", "poly", "update", "update_apply"))
+    if not gemm_launches:
+        return None
+    per_launch = flops * steps / gemm_launches
+    us = gemm_ms / gemm_launches * 1e3
+    achieved = per_launch / (us / 1e6) / 1e12
+    return {"achieved": achieved, "flops_per_launch": per_launch, "us_per_launch": us, "launches": gemm_launches,
+            "frac": achieved / peak}
+
+
+def run_sweep(args, muon, workloads, torch, dev, stream, peaks):
+    """GEMM-kernel throughput on the 64-matrix square batches, each timed on
+    its own (>= 3 warm-up and >= 5 timed steps, every launch bracketed by
+    CUDA events), with its own clock record."""
+    out = {}
+    for n in [int(x) for x in args.sweep.split(",") if x.strip()]:
+        w = workloads.get(f"square_n{n}")
+        W = workloads.weights(w, device=dev)
+        bufs = workloads.zero_bufs(w, device=dev)
+        gsets = [workloads.grads(w, s, device=dev) for s in range(2)]
+        stepper = muon.PreparedStep(W, bufs, lr=w.lr, mu=w.mu)
+        steps, warm = max(5, args.sweep_steps), 3
+        for s in range(warm):
+            stepper(gsets[s % 2], stream=stream)
+        torch.cuda.synchronize(dev)
+        muon.profile_read()
+        muon.profile_enable(True)
+        clocks = ClockSampler(dev.index)
+        clocks.start()
+        time.sleep(0.2)
+        timer = StepTimer(torch, stream)
+        ev = timer.run(lambda s: stepper(gsets[s % 2], stream=stream), steps)
+        torch.cuda.synchronize(dev)
+        clk = clocks.stop()
+        muon.profile_enable(False)
+        prof = muon.profile_read()
+        total, per = timer.times(ev)
+        flops = ns_flops(w.shapes)
+        peak, why = pick_peak(peaks, clk, total / 1e3)
+        r = gemm_roofline(prof, flops, steps, peak)
+        burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        entry = {"matrices": w.n_matrices, "steps": steps, "warmup": warm,
+                 "ms_per_step_median": statistics.median(per), "step_tflops": flops * steps / (total / 1e3) / 1e12,
+                 "gemm_tflops": r["achieved"] if r else None,
+                 "gemm_frac_burst": r["achieved"] / burst if r else None, "clocks": clk, "peak_choice": why}
+        if peaks.get("bf16_tflops_sustained") and r:
+            entry["gemm_frac_sustained"] = r["achieved"] / float(peaks["bf16_tflops_sustained"])
+        if r and clk:
+            entry["gemm_kcycles_per_launch"] = r["us_per_launch"] * clk["sm_mhz"] / 1e3
+        out[f"n{n}"] = entry
+        if muon.sync_status(stream) != 0:
+            raise RuntimeError(f"device status after the n={n} sweep entry: " + muon.last_error())
+        del W, bufs, gsets, stepper
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args):
@@ -265,13 +375,13 @@ def run_ours(args):
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    sharded = world > 1 and not args.replicas
 
     def barrier():
         if world > 1:
             dist.barrier()
 
     w = workloads.get(args.workload)
-    n = w.n_matrices
     W = workloads.weights(w, device=dev)
     bufs = workloads.zero_bufs(w, device=dev)
     gsets = [workloads.grads(w, s, device=dev) for s in range(args.grad_sets)]
@@ -283,7 +393,7 @@ def run_ours(args):
     stepper = muon.PreparedStep(W, bufs, lr=w.lr, mu=w.mu)    # the training-loop call: same W and buf
 
     def one_step(s):
-        if args.sharded and world > 1:
+        if sharded:
             mdist.sharded_step(W, gsets[s % args.grad_sets], bufs, lr=w.lr, mu=w.mu, nbuckets=args.buckets)
         else:
             stepper(gsets[s % args.grad_sets], stream=stream)
@@ -295,25 +405,22 @@ def run_ours(args):
         raise RuntimeError("device status after warm-up: " + muon.last_error())
 
     # ---- timed region: device time with CUDA events on the launching stream
+    # (an event after every step gives the per-step times as well)
     muon.profile_read()                         # drop anything recorded so far
     clocks = ClockSampler(local_rank) if rank == 0 else None
+    timer = StepTimer(torch, stream)
     barrier()
     torch.cuda.synchronize(dev)
     if clocks:
         clocks.start()
         time.sleep(0.2)
     l0 = muon.launch_count()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for s in range(args.steps):
-        one_step(s)
-    e1.record(stream)
+    ev = timer.run(one_step, args.steps)
     torch.cuda.synchronize(dev)
     launches = muon.launch_count() - l0
     barrier()
     clk = clocks.stop() if clocks else None
-    ms = e0.elapsed_time(e1)
+    ms, per_step = timer.times(ev)
 
     # ---- second pass, same steps, every launch bracketed by CUDA events on its
     # stream: per-kernel device durations for the roofline (the events cost a
@@ -324,68 +431,72 @@ def run_ours(args):
         muon.profile_enable(True)
         barrier()
         torch.cuda.synchronize(dev)
-        p0 = torch.cuda.Event(enable_timing=True)
-        p1 = torch.cuda.Event(enable_timing=True)
-        p0.record(stream)
-        for s in range(args.steps):
-            one_step(s)
-        p1.record(stream)
+        evp = timer.run(one_step, args.steps)
         torch.cuda.synchronize(dev)
         muon.profile_enable(False)
         prof = muon.profile_read()
-        ms_prof = p0.elapsed_time(p1)
+        ms_prof, _ = timer.times(evp)
+
+    # ---- cold-L2 pass: the L2 is flushed before every step, each step timed alone
+    cold = []
+    if args.cold_steps:
+        flush = torch.empty(256 << 20, dtype=torch.float32, device=dev)     # 1 GiB
+        barrier()
+        for s in range(args.cold_steps):
+            flush_l2(flush)
+            e = timer.run(one_step, 1, start=s)
+            torch.cuda.synchronize(dev)
+            cold.append(timer.times(e)[0])
+        del flush
     if muon.sync_status(stream) != 0:
         raise RuntimeError("device status after timing: " + muon.last_error())
     ms_max = mdist.max_over_ranks(ms, device=dev)
 
     flops_step = ns_flops(w.shapes)
-    jobs = 1 if args.sharded else world          # sharded: one model split over the ranks
+    jobs = 1 if sharded else world              # sharded: one model split over the ranks
     value = flops_step * args.steps * jobs / (ms_max / 1e3) / 1e12
 
     peaks, peak_src = load_peaks()
-    fk = flops_by_kind(w.shapes)
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     kinds = {}
-    gemm_ms = sum(prof[k][0] for k in ("gram", "poly", "update", "update_apply"))
-    gemm_launches = sum(prof[k][1] for k in ("gram", "poly", "update", "update_apply"))
     for k, (tms, cnt) in prof.items():
         if cnt:
             kinds[k] = {"launches": cnt, "ms_total": tms, "us_per_launch": tms / cnt * 1e3,
                         "share_of_step": tms / ms_prof}
-    roofline = None
     # algorithmic work of this rank's own GEMM launches
     own_flops = flops_step
-    if args.sharded and world > 1:
+    if sharded:
         own_flops = ns_flops([w.shapes[i] for i in mdist.partition(w.shapes, world)[rank]])
-    if gemm_launches and args.kernel_events:
-        gemm_flops_per_launch = own_flops * args.steps / gemm_launches
-        achieved = gemm_flops_per_launch / (gemm_ms / gemm_launches / 1e3) / 1e12
-        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-        roofline = {"bound": "tensor", "kernel": "ns_gemm_kernel", "achieved": achieved, "peak": peak,
-                    "unit": "TFLOP/s", "frac": achieved / peak, "traffic": ncu_traffic(),
-                    "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)",
-                    "flops_per_launch": gemm_flops_per_launch,
-                    "us_per_launch": gemm_ms / gemm_launches * 1e3}
+    peak, peak_why = pick_peak(peaks, clk, ms / 1e3)
+    roofline = None
+    r = gemm_roofline(prof, own_flops, args.steps, peak) if args.kernel_events else None
+    if r is not None:
+        roofline = {"bound": "tensor", "kernel": "ns_gemm_kernel", "achieved": r["achieved"], "peak": peak,
+                    "unit": "TFLOP/s", "frac": r["frac"], "traffic": ncu_traffic(),
+                    "peak_source": f"{peak_src} {peak_why}", "flops_per_launch": r["flops_per_launch"],
+                    "us_per_launch": r["us_per_launch"], "frac_burst": r["achieved"] / burst}
+        if peaks.get("bf16_tflops_sustained"):
+            roofline["frac_sustained"] = r["achieved"] / float(peaks["bf16_tflops_sustained"])
+        if clk:
+            roofline["kcycles_per_launch"] = r["us_per_launch"] * clk["sm_mhz"] / 1e3
     fused = [k for k in ("small", "pair") if prof[k][1]]
-    if not gemm_launches and fused and args.kernel_events:
+    if r is None and fused and args.kernel_events:
         # every matrix ran in a fused on-chip kernel: its launches carry the whole step
         f_ms = sum(prof[k][0] for k in fused)
         f_launches = sum(prof[k][1] for k in fused)
         achieved = own_flops * args.steps / (f_ms / 1e3) / 1e12
-        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
         roofline = {"bound": "tensor", "kernel": " + ".join(f"ns_{k}_kernel" for k in fused), "achieved": achieved,
-                    "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                    "peak": burst, "unit": "TFLOP/s", "frac": achieved / burst, "traffic": None,
                     "peak_source": f"{peak_src} bf16_tflops (burst: one short launch per step)",
                     "flops_per_launch": own_flops * args.steps / f_launches,
                     "us_per_launch": f_ms / f_launches * 1e3}
-    if roofline is not None and gemm_launches:
-        if "prologue" in kinds:
-            pro_bytes = 14.0 * w.n_elements
-            pro_s = prof["prologue"][0] / prof["prologue"][1] / 1e3
-            roofline["prologue"] = {"bound": "hbm", "achieved": pro_bytes / pro_s / 1e9,
-                                    "peak": float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
-                                    "unit": "GB/s",
-                                    "frac": pro_bytes / pro_s / 1e9 / float(peaks.get("hbm_gbs", 6650.0)),
-                                    "bytes_per_launch": pro_bytes}
+    if roofline is not None and "prologue" in kinds:
+        pro_bytes = 14.0 * sum(w.shapes[i][0] * w.shapes[i][1] for i in
+                               (mdist.partition(w.shapes, world)[rank] if sharded else range(w.n_matrices)))
+        pro_s = prof["prologue"][0] / prof["prologue"][1] / 1e3
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        roofline["prologue"] = {"bound": "hbm", "achieved": pro_bytes / pro_s / 1e9, "peak": hbm, "unit": "GB/s",
+                                "frac": pro_bytes / pro_s / 1e9 / hbm, "bytes_per_launch": pro_bytes}
 
     # ---- end to end through the host-buffer entry point
     e2e = None
@@ -406,11 +517,22 @@ def run_ours(args):
                "h2d_bytes_per_step": 12 * w.n_elements, "d2h_bytes_per_step": 8 * w.n_elements,
                "ms_per_step": el / k2 * 1e3, "steps": k2,
                "path": "muon_step_host: pinned host W, g, buf -> device, step, W and buf -> host"}
+        del Wh, bh, gh
+
+    sweep = None
+    if rank == 0 and world == 1 and args.sweep:
+        del W, bufs, gsets, stepper
+        torch.cuda.empty_cache()
+        sweep = run_sweep(args, muon, workloads, torch, dev, stream, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r = cpu_oracle_rate(w, budget_s=args.ref_budget)
-        cpu = {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        r_all = cpu_oracle_rate(w, budget_s=args.ref_budget)
+        cpu = {k: r_all[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        if args.ref_budget_1core > 0:
+            r_one = cpu_oracle_rate(w, budget_s=args.ref_budget_1core, threads=1)
+            cpu["one_core"] = {"value": r_one["value"], "unit": UNIT, "cores": r_one["cores"],
+                               "sample": r_one["sample"]}
 
     if world > 1:
         dist.barrier()
@@ -420,17 +542,23 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-        "scaling": "strong" if args.sharded else "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "strong" if sharded else "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) gradients, N(0,0.02) weights, zero-initialised momentum; "
                 "GPT-2-124M hidden-matrix shapes)",
-        "config": workload_config(w, args),
+        "config": workload_config(w, args, sharded),
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk,
+        "step_times": {"ms_median": statistics.median(per_step), "ms_min": min(per_step), "ms_max": max(per_step),
+                       "ms_cold_l2_median": statistics.median(cold) if cold else None,
+                       "cold_l2_steps": len(cold),
+                       "cold_l2": "a 1 GiB buffer is written before each cold step (evicts the 126 MB L2)"},
         "kernels": kinds,
-        "frac_of_dense_peak": value / world / float(peaks.get("bf16_tflops", 1647.8)),
+        "sweep": sweep,
+        "frac_of_dense_peak": value / world / burst,
+        "frac_of_dense_spec": value / world / 2250.0,
         "peaks": {"source": peak_src, "bf16_tflops": peaks.get("bf16_tflops"),
                   "bf16_tflops_sustained": peaks.get("bf16_tflops_sustained"), "hbm_gbs": peaks.get("hbm_gbs")},
     }
@@ -452,8 +580,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-events", type=int, default=1, help="per-launch CUDA events in a second timed pass")
-    ap.add_argument("--sharded", action="store_true",
-                    help="split one model's matrices over the ranks (all_gather exchange) instead of replicas")
+    ap.add_argument("--replicas", action="store_true",
+                    help="under torchrun: an independent copy of the workload per rank instead of the sharded step")
+    ap.add_argument("--sweep", default="1024,2048,4096",
+                    help="square batch sizes n (64 matrices each) timed for the sweep object ('' to skip)")
+    ap.add_argument("--sweep-steps", type=int, default=5)
+    ap.add_argument("--cold-steps", type=int, default=5, help="steps timed one by one after an L2 flush")
+    ap.add_argument("--ref-budget-1core", type=float, default=4.0,
+                    help="seconds of single-threaded CPU oracle work (cpu_baseline.one_core)")
     ap.add_argument("--buckets", type=int, default=2,
                     help="with --sharded: runs per rank whose all_gather overlaps the next run's step")
     args = ap.parse_args()

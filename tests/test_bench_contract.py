@@ -33,7 +33,8 @@ def test_reference_arm_line():
 
 @pytest.mark.gpu
 def test_gpu_arm_line():
-    d = _run(["--steps", "20", "--warmup", "3", "--grad-sets", "2", "--e2e-steps", "2", "--ref-budget", "1"], 900)
+    d = _run(["--steps", "20", "--warmup", "3", "--grad-sets", "2", "--e2e-steps", "2", "--ref-budget", "1",
+              "--ref-budget-1core", "1", "--sweep", "1024", "--cold-steps", "2"], 900)
     assert BASE_KEYS | {"roofline", "gpu_launches", "clocks", "kernels"} <= set(d)
     assert d["n_gpus"] == 1 and d["scaling"] == "weak" and d["higher_is_better"] is True
     r = d["roofline"]
@@ -43,6 +44,11 @@ def test_gpu_arm_line():
     assert d["e2e"]["h2d_bytes_per_step"] > 0 and d["e2e"]["d2h_bytes_per_step"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle"
     assert set(d["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
+    assert 0 < r["frac_burst"] < 1.5 and d["cpu_baseline"]["one_core"]["cores"] == 1
+    st = d["step_times"]
+    assert st["cold_l2_steps"] == 2 and st["ms_cold_l2_median"] > 0 and st["ms_min"] <= st["ms_median"]
+    sw = d["sweep"]["n1024"]
+    assert sw["matrices"] == 64 and sw["steps"] >= 5 and sw["warmup"] >= 3 and 0 < sw["gemm_frac_burst"] < 1.5
 
 
 def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
@@ -110,3 +116,16 @@ def test_reference_arm_under_torchrun_prints_once_from_rank_0():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2
     assert d["cpu_baseline"]["cores"] > 1 or (os.cpu_count() or 1) == 1   # not the launcher's one thread
+
+
+def test_peak_choice_follows_the_clock_record():
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = {"bf16_tflops": 1647.8, "bf16_tflops_sustained": 1344.1}
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}
+    capped = {"sm_mhz": 1450.0, "sm_max_mhz": 1965.0}
+    assert bench.pick_peak(peaks, full, 5.0)[0] == 1647.8          # full clock: burst
+    assert bench.pick_peak(peaks, capped, 0.03)[0] == 1647.8       # short region: burst
+    assert bench.pick_peak(peaks, capped, 5.0)[0] == 1344.1        # long region under the cap: sustained
+    assert bench.pick_peak({"bf16_tflops": 1590.0}, capped, 5.0)[0] == 1590.0   # no sustained figure
+    assert "bf16_tflops_sustained" not in bench.FALLBACK_PEAKS
