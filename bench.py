@@ -277,6 +277,11 @@ def pick_peak(peaks, clk, timed_s):
     return float(sust), "bf16_tflops_sustained (timed region >= 1 s below full clock)"
 
 
+# Launch kinds of the tcgen05 GEMM kernel (ns_gemm_kernel): the chained launch
+# of every phase but the last update, and the one-phase launches.
+GEMM_KINDS = ("chain", "gram", "poly", "update", "update_apply")
+
+
 def flush_l2(buf):
     buf.zero_()                      # writes more than the 126 MB L2: evicts every line
 
@@ -302,8 +307,8 @@ class StepTimer:
 
 
 def gemm_roofline(prof, flops, steps, peak):
-    gemm_ms = sum(prof[k][0] for k in ("gram", "poly", "update", "update_apply"))
-    gemm_launches = sum(prof[k][1] for k in ("gram", "poly", "update", "update_apply"))
+    gemm_ms = sum(prof[k][0] for k in GEMM_KINDS)
+    gemm_launches = sum(prof[k][1] for k in GEMM_KINDS)
     if not gemm_launches:
         return None
     per_launch = flops * steps / gemm_launches

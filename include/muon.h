@@ -178,7 +178,8 @@ void muon_release(void);
 #define MUON_KIND_APPLY_X0 5
 #define MUON_KIND_SMALL 6        /* fused single-CTA step of small matrices */
 #define MUON_KIND_PAIR 7         /* fused CTA-pair step, 128 < short side <= 256, long side <= 256 */
-#define MUON_NUM_KINDS 8
+#define MUON_KIND_CHAIN 8        /* every Newton-Schulz phase but the last update, one chained launch */
+#define MUON_NUM_KINDS 9
 
 /* 1: bracket every kernel launch with CUDA events on its stream; 0: stop. */
 int muon_profile_enable(int enable);
@@ -196,8 +197,23 @@ int64_t muon_launch_count(void);
  * so its MMA warp's wait runs out and the call reports MUON_ERR_TIMEOUT
  * (fault injection that neither faults nor hangs the GPU).
  * flags bit 1: the same for the next CTA-pair launch, whose first product is
- * not issued, so both CTAs' waits for it run out. */
+ * not issued, so both CTAs' waits for it run out.
+ * flags bit 2 (kept until cleared): run the Newton-Schulz phases as one launch
+ * per phase instead of the chained launch (for comparisons). */
 int muon_debug_set(int flags, int64_t wait_limit_ns);
+
+/* The work lists of the chained launch for these shapes and `ns_steps`, as
+ * the library would build them for a device that holds `nclusters` clusters of
+ * two CTAs at once (host only: no device is touched).  Covers the first group
+ * of matrices (at most 320 matrices over 16 padded shapes; matrices the fused
+ * kernels run whole take no part).  Item i is items[8i .. 8i+7] = {need,
+ * matrix (the caller's index), shape class, index in class, tile row, tile
+ * column, phase (0 Gram, 1 polynomial, 2 update), iteration}; cluster c runs
+ * items [cluster_off[c], cluster_off[c + 1]) in order (cluster_off holds
+ * nclusters + 1 entries).  *nitems receives the item count;
+ * MUON_ERR_INVALID_ARG if `capacity` (in items) is smaller. */
+int muon_chain_plan(const int64_t* shapes, int n, int ns_steps, int nclusters, int32_t* items, int64_t capacity,
+                    int32_t* cluster_off, int64_t* nitems);
 
 #ifdef __cplusplus
 }

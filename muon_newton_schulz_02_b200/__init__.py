@@ -20,7 +20,7 @@ from array import array
 
 __all__ = [
     "step", "PreparedStep", "orthogonalize", "step_host", "step_noalloc", "workspace_size", "sync_status", "last_error", "release",
-    "profile_enable", "profile_read", "launch_count", "debug_set", "lib", "MuonError", "KINDS",
+    "profile_enable", "profile_read", "launch_count", "debug_set", "chain_plan", "lib", "MuonError", "KINDS",
     "NS_A", "NS_B", "NS_C", "NS_STEPS", "NS_EPS", "LIB_PATH", "header_functions",
 ]
 
@@ -29,7 +29,7 @@ LIB_PATH = os.path.join(HERE, "libmuon_b200.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "muon.h")
 
 NS_A, NS_B, NS_C, NS_STEPS, NS_EPS = 3.4445, -4.7750, 2.0315, 5, 1e-7
-KINDS = ("prologue", "gram", "poly", "update", "update_apply", "apply_x0", "small", "pair")
+KINDS = ("prologue", "gram", "poly", "update", "update_apply", "apply_x0", "small", "pair", "chain")
 
 STATUS = {0: "MUON_OK", -1: "MUON_ERR_INVALID_ARG", -2: "MUON_ERR_SHAPE", -3: "MUON_ERR_CUDA",
           -4: "MUON_ERR_NOMEM", -5: "MUON_ERR_TIMEOUT", -6: "MUON_ERR_DEVICE", -7: "MUON_ERR_UNSUPPORTED"}
@@ -90,6 +90,9 @@ def lib() -> ctypes.CDLL:
     L.muon_launch_count.restype = ctypes.c_int64
     L.muon_debug_set.argtypes = [ctypes.c_int, ctypes.c_int64]
     L.muon_debug_set.restype = ctypes.c_int
+    L.muon_chain_plan.argtypes = [_I64P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int32),
+                                  ctypes.c_int64, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64)]
+    L.muon_chain_plan.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -269,3 +272,20 @@ def launch_count() -> int:
 
 def debug_set(flags: int = 0, wait_limit_ns: int = 0):
     _check(lib().muon_debug_set(int(flags), int(wait_limit_ns)))
+
+
+def chain_plan(shapes, ns_steps: int = NS_STEPS, nclusters: int = 74):
+    """The chained launch's work lists for these shapes (host only): returns
+    (items, cluster_off) with items a list of (need, matrix, class, index,
+    tile row, tile column, phase, iteration) tuples."""
+    sh = _shapes(shapes)
+    off = (ctypes.c_int32 * (nclusters + 1))()
+    cnt = ctypes.c_int64(0)
+    rc = lib().muon_chain_plan(sh, len(shapes), int(ns_steps), int(nclusters), None, 0, off, ctypes.byref(cnt))
+    if rc not in (0, -1):
+        _check(rc)
+    buf = (ctypes.c_int32 * (8 * max(1, cnt.value)))()
+    _check(lib().muon_chain_plan(sh, len(shapes), int(ns_steps), int(nclusters), buf, cnt.value, off,
+                                 ctypes.byref(cnt)))
+    items = [tuple(buf[8 * i:8 * i + 8]) for i in range(cnt.value)]
+    return items, list(off)

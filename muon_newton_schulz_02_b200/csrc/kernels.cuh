@@ -4,8 +4,10 @@
 //
 //   prologue_kernel   buf <- mu*buf + g ; G = g + mu*buf ; per-matrix ||G||_F ;
 //                     X0 = bf16(G), stored short-side-major (k x l, padded).
-//   ns_gemm_kernel    one persistent tcgen05 GEMM launch per NS phase over all
-//                     matrices of a group:
+//   ns_gemm_kernel    persistent tcgen05 GEMM over all matrices of a group,
+//                     either one launch chaining every phase but the last
+//                     update (per-matrix completion counters order the
+//                     phases), or one launch per phase:
 //                       GRAM    A = s^2 * X X^T            (upper-triangle 256-blocks only)
 //                       POLY    B' = a*I + b*A + c*(A A)   (upper-triangle 256-blocks only)
 //                       UPDATE  X' = s*(B' X)              (last step: W -= lr*X')
@@ -85,11 +87,29 @@ struct OutMat {       // destination of the final UPDATE epilogue
   int tma;            // 1: wmaps[] holds a valid fp32 tensor map of w (needs vec)
 };
 
+// One unit of work of the chained launch: a 256 x 256 output tile of one
+// phase (Gram, polynomial or update) of one Newton-Schulz iteration of one
+// matrix.  The host lays out one list per cluster in an order in which every
+// item's inputs are produced by items that come earlier in some list (see
+// `need`), so the lists can run concurrently on all clusters.
+struct WorkItem {
+  int need;                 // tile halves of this matrix (2 per tile: one per CTA) that must have
+                            // completed before this item reads its inputs
+  unsigned short mat, b;    // matrix (group order), its index within its shape class
+  unsigned short tm, tn;    // output tile row and column (256-blocks)
+  unsigned char cls, mode;  // shape class, kModeGram / kModePoly / kModeUpdate
+  unsigned short it;        // Newton-Schulz iteration
+};
+static_assert(sizeof(WorkItem) == 16, "WorkItem layout");
+
 struct GemmArgs {
   const CUtensorMap* tmaps;
   const CUtensorMap* wmaps;   // per matrix (group order): W as fp32 [m][n]; box 32x128 (X = W) or 32x32 (X = W^T)
   const float* scale;     // per matrix (group order): 1/(||G||_F + eps)
   int* status;
+  const WorkItem* items;  // chained launch: every cluster's work list, back to back
+  const int* item_off;    // chained launch: cluster c runs items[item_off[c] .. item_off[c + 1])
+  unsigned* done;         // chained launch: per matrix, tile halves completed (zeroed by the prologue)
   unsigned long long wait_limit_ns;
   int nclasses, total_tiles;
   int mode, x_in, first, final_apply, assign, debug_flags;
@@ -114,6 +134,7 @@ struct ProArgs {
   float* partials;
   unsigned* tickets;
   float* scale;
+  unsigned* done;         // per-matrix completion counters of the chained launch that follows (or null)
   ProMat mats[kMaxMats];
 };
 
@@ -155,6 +176,8 @@ __global__ void __launch_bounds__(kProThreads) prologue_kernel(const __grid_cons
   griddep_launch_dependents();
   griddep_wait();
   const int t = blockIdx.x;
+  if (t == 0 && p.done)
+    for (int i = threadIdx.x; i < p.nmats; i += kProThreads) p.done[i] = 0u;
   const int mi = find_mat(p, t);
   const ProMat& M = p.mats[mi];
   const int local = t - M.tile_begin;
@@ -311,6 +334,17 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& p, int t, bool 
   return tc;
 }
 
+// One output tile as every role of the GEMM kernel sees it.
+struct Tile {
+  int mode;       // kModeGram / kModePoly / kModeUpdate
+  int cls, b;     // shape class, matrix within the class
+  int tm, tn;     // 256-block row and column of the output
+  int x_in;       // which ping-pong iterate holds X (iteration parity)
+  int first;      // first iteration: the normalisation scale is folded in
+  int mat;        // matrix in group order
+  int need;       // chained launch: tile halves of `mat` that must have completed first
+};
+
 // Byte offset of the 16-byte unit u (0..7) of row r inside a 128-row x 128-byte
 // box stored with the 128-byte swizzle (the pattern TMA writes / reads).
 __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t u) { return r * 128u + ((u ^ (r & 7u)) << 4); }
@@ -363,19 +397,33 @@ static_assert(sizeof(GemmCtrl) <= kSmemCtrlBytes, "GemmCtrl does not fit its sha
 static_assert(kGemmSmemBytes <= 232448, "more dynamic shared memory than a CTA may have");
 static_assert(kStgLag >= 1 && kStgLag < kStgBufs, "staging ring");
 
-// One persistent launch per Newton-Schulz phase.  A cluster of two CTAs (one
-// per SM) computes 256 x 256 output tiles with tcgen05.mma.cta_group::2: each
-// CTA loads its 128 rows of A and its 128 rows (or columns) of B per stage, the
-// even CTA issues the MMAs over both CTAs' shared memory, and each CTA's TMEM
-// holds its 128 rows x 256 fp32 columns (two accumulators, double-buffered).
-// Roles per CTA: warp 0 TMA producer; warp 1 MMA issuer (even CTA) and TMEM
-// allocator; warp 2 epilogue DMA (loads the polynomial epilogue's A slices,
-// issues the TMA stores / add-reductions of the output slices and recycles
-// their buffers); warps 3..6 epilogue math (per 64-column slice: tcgen05.ld ->
-// fp32 math -> bf16 -> 128B-swizzled smem).  The math warps hand slices to the DMA
-// warp through mbarriers and never wait on TMA latency themselves.
-template <int kMode, bool kFinal>
+// The Newton-Schulz GEMM kernel.  A cluster of two CTAs (one per SM) computes
+// 256 x 256 output tiles with tcgen05.mma.cta_group::2: each CTA loads its 128
+// rows of A and its 128 rows (or columns) of B per stage, the even CTA issues
+// the MMAs over both CTAs' shared memory, and each CTA's TMEM holds its 128
+// rows x 256 fp32 columns (two accumulators, double-buffered).  Roles per CTA:
+// warp 0 TMA producer; warp 1 MMA issuer (even CTA) and TMEM allocator; warp 2
+// epilogue DMA (loads the polynomial epilogue's A slices, issues the TMA
+// stores / add-reductions of the output slices and recycles their buffers);
+// warps 3..6 epilogue math (per 64-column slice: tcgen05.ld -> fp32 math ->
+// bf16 -> 128B-swizzled smem).  The math warps hand slices to the DMA warp
+// through mbarriers and never wait on TMA latency themselves.
+//
+// Two ways to launch it:
+//   kChain = false: one launch per phase (kMode) over all matrices of a group,
+//     persistent, tile t to cluster t mod #clusters; kFinal selects the last
+//     update, whose epilogue adds -lr*O into W.
+//   kChain = true: one launch for every phase of every iteration but the last
+//     update.  Each cluster runs its own list of work items (any phase, any
+//     matrix; the host orders the lists so that items are ready in time);
+//     before reading a matrix's Gram, polynomial or iterate it waits (bounded)
+//     for the counter of completed tiles of that matrix, and after its output
+//     stores have landed it adds one to that counter.  A matrix's phases then
+//     follow each other closely on whichever clusters are free, without a
+//     launch boundary, and its operands are still in L2 when they are read.
+template <int kMode, bool kFinal, bool kChain>
 __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ GemmArgs p) {
+  static_assert(!(kChain && kFinal), "the chained launch never runs the final update");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
@@ -386,9 +434,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();             // 0: issues the MMAs of the pair
   const int cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
-  constexpr bool sym = kMode != kModeUpdate;
-  constexpr bool has_d = kMode == kModePoly;           // the epilogue reads an input tile (A)
-  constexpr bool final_w = kMode == kModeUpdate && kFinal;
+  constexpr bool final_w = !kChain && kMode == kModeUpdate && kFinal;
   // Slice buffers: every phase but the final update uses all four 16 KB buffers
   // for its output slices (the polynomial phase loads its A input into them
   // first), with two output stores in flight.  The final update stores no bf16
@@ -398,6 +444,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   auto slice_buf = [&](int b) { return b < 2 ? dbuf + b * kSliceBytes : mbuf + (b - 2) * kSliceBytes; };
   // fp32 staging buffers of the final update
   auto stg_buf = [&](int i) { return i < 2 ? mbuf + i * kSliceBytes : dbuf + (i - 2) * kSliceBytes; };
+
+  // This cluster's tiles, in processing order.
+  const int item0 = kChain ? p.item_off[cid] : 0;
+  const int my_tiles = kChain ? p.item_off[cid + 1] - item0
+                              : (cid < p.total_tiles ? (p.total_tiles - cid + ncl - 1) / ncl : 0);
+  auto tile_of = [&](int i) {
+    Tile T;
+    if constexpr (kChain) {
+      const WorkItem w = p.items[item0 + i];
+      T.mode = w.mode; T.cls = w.cls; T.b = w.b; T.tm = w.tm; T.tn = w.tn;
+      T.x_in = w.it & 1; T.first = w.it == 0; T.mat = w.mat; T.need = w.need;
+    } else {
+      const TileCoord tc = decode_tile(p, cid + i * ncl, kMode != kModeUpdate);
+      T.mode = kMode; T.cls = tc.cls; T.b = tc.b; T.tm = tc.tm; T.tn = tc.tn;
+      T.x_in = p.x_in; T.first = p.first; T.mat = p.cls[tc.cls].mat_first + tc.b; T.need = 0;
+    }
+    return T;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
@@ -430,8 +494,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   // set-up above overlaps the previous launch; its outputs are read only below
   griddep_launch_dependents();
   griddep_wait();
-  // tiles of this cluster and their 64-column slices, in processing order
-  const int my_tiles = cid < p.total_tiles ? (p.total_tiles - cid + ncl - 1) / ncl : 0;
   const int my_slices = 4 * my_tiles;
 
   if (warp == 0) {
@@ -446,22 +508,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int it = 0;
-      for (int t = cid; t < p.total_tiles && ok; t += ncl, ++it) {
-        const TileCoord tc = decode_tile(p, t, sym);
-        const GemmClass& C = p.cls[tc.cls];
+      for (int it = 0; it < my_tiles && ok; ++it) {
+        const Tile T = tile_of(it);
+        const GemmClass& C = p.cls[T.cls];
+        const bool sym = T.mode != kModeUpdate;
+        if (kChain && T.need > 0) {
+          // this tile reads what earlier tiles of the matrix wrote
+          if (!wait_count(&p.done[T.mat], (uint32_t)T.need, wc, kDevTimeoutDep)) { ok = false; break; }
+          fence_proxy_async_global();
+        }
         const CUtensorMap* tA;
         const CUtensorMap* tB;
-        if (kMode == kModeGram) { tA = &p.tmaps[C.tmap_base + (p.x_in ? kTmX1 : kTmX0)]; tB = tA; }
-        else if (kMode == kModePoly) { tA = &p.tmaps[C.tmap_base + kTmA]; tB = tA; }
-        else { tA = &p.tmaps[C.tmap_base + kTmB]; tB = &p.tmaps[C.tmap_base + (p.x_in ? kTmX1mn : kTmX0mn)]; }
-        const int arow = tc.tm * kTile + (int)rank * kBM;     // this CTA's A rows
-        const int bidx = tc.tn * kTile + (int)rank * kBNh;    // this CTA's B rows (or columns)
+        if (T.mode == kModeGram) { tA = &p.tmaps[C.tmap_base + (T.x_in ? kTmX1 : kTmX0)]; tB = tA; }
+        else if (T.mode == kModePoly) { tA = &p.tmaps[C.tmap_base + kTmA]; tB = tA; }
+        else { tA = &p.tmaps[C.tmap_base + kTmB]; tB = &p.tmaps[C.tmap_base + (T.x_in ? kTmX1mn : kTmX0mn)]; }
+        const int arow = T.tm * kTile + (int)rank * kBM;     // this CTA's A rows
+        const int bidx = T.tn * kTile + (int)rank * kBNh;    // this CTA's B rows (or columns)
         // The Gram and polynomial matrices hold only their upper-triangle 256-blocks:
         // an operand block below the diagonal is read through its stored transpose.
-        const CUtensorMap* tAt = (kMode == kModePoly) ? &p.tmaps[C.tmap_base + kTmAmn]
-                                                      : &p.tmaps[C.tmap_base + kTmBmn];
-        for (int kb = 0; kb < C.kblocks; ++kb) {
+        const CUtensorMap* tAt = (T.mode == kModePoly) ? &p.tmaps[C.tmap_base + kTmAmn]
+                                                       : &p.tmaps[C.tmap_base + kTmBmn];
+        const int kblocks = (T.mode == kModeGram ? C.lp : C.kp) / kBK;
+        for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, wc, kDevTimeoutEmpty)) { ok = false; break; }
           uint8_t* sa = stage_base + stage * kStageBytes;
           uint8_t* sb = sa + kStageABytes;
@@ -469,25 +537,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           const bool inject_skip = (p.debug_flags & 1) && it == 0 && kb == 0;
           // on a diagonal tile of the symmetric phases a CTA's A rows are its B
           // rows: load them once, the MMA reads both operands from the A buffer
-          const bool same_ab = sym && tc.tm == tc.tn;
+          const bool same_ab = sym && T.tm == T.tn;
           if (!inject_skip) {
             if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], same_ab ? 2 * kStageABytes : 2 * kStageBytes);
-            if (kMode != kModeGram && tc.tm > (kb >> 2)) {
+            if (T.mode != kModeGram && T.tm > (kb >> 2)) {
               // A rows below the diagonal block: columns [arow, +128) of rows [kb*64, +64), MN-major
-              tma_load_3d_pair(sa, tAt, full_lead, arow, kb * kBK, tc.b);
-              tma_load_3d_pair(sa + kStageABytes / 2, tAt, full_lead, arow + 64, kb * kBK, tc.b);
+              tma_load_3d_pair(sa, tAt, full_lead, arow, kb * kBK, T.b);
+              tma_load_3d_pair(sa + kStageABytes / 2, tAt, full_lead, arow + 64, kb * kBK, T.b);
             } else {
-              tma_load_3d_pair(sa, tA, full_lead, kb * kBK, arow, tc.b);
+              tma_load_3d_pair(sa, tA, full_lead, kb * kBK, arow, T.b);
             }
             if (same_ab) {
               // nothing: B is the A block just loaded
-            } else if (kMode == kModeUpdate || (kMode == kModePoly && tc.tn > (kb >> 2))) {
+            } else if (T.mode == kModeUpdate || (T.mode == kModePoly && T.tn > (kb >> 2))) {
               // B = rows [kb*64, +64) x this CTA's 128 columns, MN-major: two 64-col boxes
-              const CUtensorMap* tBm = (kMode == kModeUpdate) ? tB : tAt;
-              tma_load_3d_pair(sb, tBm, full_lead, bidx, kb * kBK, tc.b);
-              tma_load_3d_pair(sb + kStageBBytes / 2, tBm, full_lead, bidx + 64, kb * kBK, tc.b);
+              const CUtensorMap* tBm = (T.mode == kModeUpdate) ? tB : tAt;
+              tma_load_3d_pair(sb, tBm, full_lead, bidx, kb * kBK, T.b);
+              tma_load_3d_pair(sb + kStageBBytes / 2, tBm, full_lead, bidx + 64, kb * kBK, T.b);
             } else {
-              tma_load_3d_pair(sb, tB, full_lead, kb * kBK, bidx, tc.b);
+              tma_load_3d_pair(sb, tB, full_lead, kb * kBK, bidx, T.b);
             }
           }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -500,28 +568,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int it = 0;
       bool ok = true;
       bool issued_any = false;
-      for (int t = cid; t < p.total_tiles && ok; t += ncl, ++it) {
-        const TileCoord tc = decode_tile(p, t, sym);
-        const GemmClass& C = p.cls[tc.cls];
+      for (int it = 0; it < my_tiles && ok; ++it) {
+        const Tile T = tile_of(it);
+        const GemmClass& C = p.cls[T.cls];
+        const bool sym = T.mode != kModeUpdate;
         const int acc = it & 1;
         const uint32_t acc_phase = (uint32_t)((it >> 1) & 1);
         if (!mbar_wait_cluster(&ctl->tmem_empty[acc], acc_phase ^ 1u, wc, kDevTimeoutAccum)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
-        for (int kb = 0; kb < C.kblocks; ++kb) {
+        const int kblocks = (T.mode == kModeGram ? C.lp : C.kp) / kBK;
+        for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&ctl->full[stage], phase, wc, kDevTimeoutFull)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * kStageBytes);
           // same choices as the producer: diagonal tiles of the symmetric phases
           // share one operand buffer, blocks below the diagonal arrive MN-major
-          const bool same_ab = sym && tc.tm == tc.tn;
+          const bool same_ab = sym && T.tm == T.tn;
           const uint32_t sb = same_ab ? sa : sa + kStageABytes;
-          const uint32_t a_mn = (kMode != kModeGram && tc.tm > (kb >> 2)) ? 1u : 0u;
+          const uint32_t a_mn = (T.mode != kModeGram && T.tm > (kb >> 2)) ? 1u : 0u;
           const uint32_t b_mn = same_ab ? a_mn
-                                : (kMode == kModeUpdate || (kMode == kModePoly && tc.tn > (kb >> 2))) ? 1u : 0u;
+                                : (T.mode == kModeUpdate || (T.mode == kModePoly && T.tn > (kb >> 2))) ? 1u : 0u;
           const uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN, a_mn, b_mn);
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
@@ -556,92 +625,143 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           for (int b = 0; b < p.cls[c].batch; ++b)
             if (p.out[p.cls[c].mat_first + b].tma) tmap_acquire(&p.wmaps[p.cls[c].mat_first + b]);
       int pend[4] = {-1, -1, -1, -1};              // parity of an input load not yet seen landed
-      // Make slice gs's buffer set ready: load its input slice, or just hand it over.
-      auto prepare = [&](int gs) {
-        if (gs < 0 || gs >= my_slices) return;
+      // Make slice gs's buffer set ready: load its input slice (polynomial
+      // phase: the A block the epilogue adds), or just hand it over.
+      auto prepare = [&](int gs, const Tile& T) {
         const int b = gs % nbuf;
-        if (has_d) {
-          const int t = cid + (gs >> 2) * ncl, h = gs & 3;
-          const TileCoord tc = decode_tile(p, t, sym);
-          const GemmClass& C = p.cls[tc.cls];
-          const CUtensorMap* tD = &p.tmaps[C.tmap_base + kTmA];
+        if (T.mode == kModePoly) {
+          const GemmClass& C = p.cls[T.cls];
           mbar_arrive_expect_tx(&ctl->in_full[b], kSliceBytes);
-          tma_load_3d(slice_buf(b), tD, &ctl->in_full[b], tc.tn * kTile + 64 * h,
-                      tc.tm * kTile + (int)rank * kBM, tc.b);
+          tma_load_3d(slice_buf(b), &p.tmaps[C.tmap_base + kTmA], &ctl->in_full[b], T.tn * kTile + 64 * (gs & 3),
+                      T.tm * kTile + (int)rank * kBM, T.b);
           pend[b] = (gs / nbuf) & 1;
         } else {
           mbar_arrive(&ctl->in_full[b]);
         }
       };
-      for (int g0 = 0; g0 < nbuf; ++g0) prepare(g0);
-      bool ok = true;
-      int gc = 0;                                  // fp32 chunk counter (final update)
-      int stg_freed = 0;                           // chunks whose staging buffer was handed back
-      auto release_stg = [&](int upto) {           // hand back the buffers of chunks < upto, in order
-        for (; stg_freed < upto; ++stg_freed) mbar_arrive(&ctl->stg_free[stg_freed % kStgBufs]);
+      auto output_map = [&](const Tile& T) {
+        const GemmClass& C = p.cls[T.cls];
+        if (T.mode == kModeGram) return &p.tmaps[C.tmap_base + kTmA];
+        if (T.mode == kModePoly) return &p.tmaps[C.tmap_base + kTmB];
+        return &p.tmaps[C.tmap_base + (T.x_in ? kTmX0 : kTmX1)];
       };
-      for (int gs = 0; gs < my_slices && ok; ++gs) {
-        const int b = gs % nbuf;
-        const uint32_t ph = (uint32_t)((gs / nbuf) & 1);
-        const int t = cid + (gs >> 2) * ncl, h = gs & 3;
-        const TileCoord tc = decode_tile(p, t, sym);
-        const GemmClass& C = p.cls[tc.cls];
-        const int row0 = tc.tm * kTile + (int)rank * kBM;
-        if (final_w) {
-          const int mat = C.mat_first + tc.b;
-          const OutMat& O = p.out[mat];
-          for (int sub = 0; sub < 2 && ok; ++sub, ++gc) {
-            const int s = gc % kStgBufs;
-            if (!mbar_wait(&ctl->stg_full[s], (uint32_t)((gc / kStgBufs) & 1), wc, kDevTimeoutEpi)) { ok = false; break; }
-            if (O.tma) {
-              const uint8_t* S = stg_buf(s);
-              const CUtensorMap* wm = &p.wmaps[mat];
-              const int gj0 = tc.tn * kTile + 64 * h + 32 * sub;
-              if (!O.trans) {
-                if (row0 < O.m && gj0 < O.n) {
-                  if (p.assign) tma_store_2d(wm, S, gj0, row0); else tma_reduce_add_2d(wm, S, gj0, row0);
-                }
-              } else if (gj0 < O.m) {
-                for (int hq = 0; hq < 4; ++hq) {
-                  if (row0 + 32 * hq >= O.n) continue;
-                  if (p.assign) tma_store_2d(wm, S + hq * 4096, row0 + 32 * hq, gj0);
-                  else tma_reduce_add_2d(wm, S + hq * 4096, row0 + 32 * hq, gj0);
-                }
-              }
-              tma_store_commit();                  // one bulk group per chunk
-              tma_store_wait_read<kStgLag>();      // chunks up to gc - kStgLag have been read
-              release_stg(gc + 1 - kStgLag);
-            } else {
-              tma_store_wait_read0();
-              release_stg(gc + 1);
+      bool ok = true;
+      if constexpr (kChain) {
+        // Slices of tile i use buffers 0..3 in order.  A tile's completion is
+        // published (its stores landed, then the counter) before the DMA waits
+        // for anything a later tile needs, so a cluster never waits on itself.
+        if (my_tiles > 0) {
+          const Tile T0 = tile_of(0);
+          if (T0.mode == kModePoly && T0.need > 0) {
+            ok = wait_count(&p.done[T0.mat], (uint32_t)T0.need, wc, kDevTimeoutDep);
+            fence_proxy_async_global();
+          }
+          if (ok)
+            for (int h = 0; h < 4; ++h) prepare(h, T0);
+        }
+        for (int i = 0; i < my_tiles && ok; ++i) {
+          const Tile T = tile_of(i);
+          const GemmClass& C = p.cls[T.cls];
+          const bool has_next = i + 1 < my_tiles;
+          const Tile N = tile_of(has_next ? i + 1 : i);
+          const bool next_in = has_next && N.mode == kModePoly;
+          const int row0 = T.tm * kTile + (int)rank * kBM;
+          const CUtensorMap* tO = output_map(T);
+          const int ocols = T.mode != kModeUpdate ? C.kp : C.lp;
+          for (int h = 0; h < 4; ++h) {
+            if (!mbar_wait(&ctl->out_full[h], (uint32_t)(i & 1), wc, kDevTimeoutEpi)) { ok = false; break; }
+            pend[h] = -1;                          // the math warps saw this slice's input land
+            const int x0 = T.tn * kTile + 64 * h;
+            if (row0 < C.kp && x0 < ocols) tma_store_3d(tO, slice_buf(h), x0, row0, T.b);
+            tma_store_commit();
+            if (h >= 1 && has_next && !next_in) {
+              tma_store_wait_read1();              // slice h-1's buffer has been read
+              prepare(4 * (i + 1) + h - 1, N);     // no input to load: hand it over now
             }
           }
           if (!ok) break;
-        }
-        if (!mbar_wait(&ctl->out_full[b], ph, wc, kDevTimeoutEpi)) { ok = false; break; }
-        if (has_d) pend[b] = -1;                   // the math warps saw this slice's input land
-        if (!final_w) {
-          const CUtensorMap* tO;
-          if (kMode == kModeGram) tO = &p.tmaps[C.tmap_base + kTmA];
-          else if (kMode == kModePoly) tO = &p.tmaps[C.tmap_base + kTmB];
-          else tO = &p.tmaps[C.tmap_base + (p.x_in ? kTmX0 : kTmX1)];
-          // stores start inside the tensor only (a pair tile can overhang the
-          // 128-padded edge by half; the overhang is never stored)
-          const int ocols = sym ? C.kp : C.lp;
-          const int x0 = tc.tn * kTile + 64 * h;
-          if (row0 < C.kp && x0 < ocols) tma_store_3d(tO, slice_buf(b), x0, row0, tc.b);
-          tma_store_commit();
-          if constexpr (nbuf == 4) {
-            tma_store_wait_read1();                // the previous slice's buffer is free again
-            if (gs >= 1) prepare(gs - 1 + nbuf);   // slices 0..3 were armed before the loop
-            continue;
+          tma_store_wait_all0();                   // this tile's output has landed in memory
+          fence_proxy_async_global();
+          red_release_gpu_add(&p.done[T.mat], 1u);
+          if (has_next) {
+            if (next_in) {
+              if (N.need > 0) {
+                if (!wait_count(&p.done[N.mat], (uint32_t)N.need, wc, kDevTimeoutDep)) { ok = false; break; }
+                fence_proxy_async_global();
+              }
+              for (int h = 0; h < 4; ++h) prepare(4 * (i + 1) + h, N);
+            } else {
+              prepare(4 * (i + 1) + 3, N);
+            }
           }
-          tma_store_wait_read0();                  // buffers b readable again
         }
-        prepare(gs + nbuf);
+      } else {
+        for (int g0 = 0; g0 < nbuf && g0 < my_slices; ++g0) prepare(g0, tile_of(g0 >> 2));
+        int gc = 0;                                // fp32 chunk counter (final update)
+        int stg_freed = 0;                         // chunks whose staging buffer was handed back
+        auto release_stg = [&](int upto) {         // hand back the buffers of chunks < upto, in order
+          for (; stg_freed < upto; ++stg_freed) mbar_arrive(&ctl->stg_free[stg_freed % kStgBufs]);
+        };
+        for (int gs = 0; gs < my_slices && ok; ++gs) {
+          const int b = gs % nbuf;
+          const uint32_t ph = (uint32_t)((gs / nbuf) & 1);
+          const int h = gs & 3;
+          const Tile T = tile_of(gs >> 2);
+          const GemmClass& C = p.cls[T.cls];
+          const int row0 = T.tm * kTile + (int)rank * kBM;
+          if (final_w) {
+            const OutMat& O = p.out[T.mat];
+            for (int sub = 0; sub < 2 && ok; ++sub, ++gc) {
+              const int s = gc % kStgBufs;
+              if (!mbar_wait(&ctl->stg_full[s], (uint32_t)((gc / kStgBufs) & 1), wc, kDevTimeoutEpi)) { ok = false; break; }
+              if (O.tma) {
+                const uint8_t* S = stg_buf(s);
+                const CUtensorMap* wm = &p.wmaps[T.mat];
+                const int gj0 = T.tn * kTile + 64 * h + 32 * sub;
+                if (!O.trans) {
+                  if (row0 < O.m && gj0 < O.n) {
+                    if (p.assign) tma_store_2d(wm, S, gj0, row0); else tma_reduce_add_2d(wm, S, gj0, row0);
+                  }
+                } else if (gj0 < O.m) {
+                  for (int hq = 0; hq < 4; ++hq) {
+                    if (row0 + 32 * hq >= O.n) continue;
+                    if (p.assign) tma_store_2d(wm, S + hq * 4096, row0 + 32 * hq, gj0);
+                    else tma_reduce_add_2d(wm, S + hq * 4096, row0 + 32 * hq, gj0);
+                  }
+                }
+                tma_store_commit();                  // one bulk group per chunk
+                tma_store_wait_read<kStgLag>();      // chunks up to gc - kStgLag have been read
+                release_stg(gc + 1 - kStgLag);
+              } else {
+                tma_store_wait_read0();
+                release_stg(gc + 1);
+              }
+            }
+            if (!ok) break;
+          }
+          if (!mbar_wait(&ctl->out_full[b], ph, wc, kDevTimeoutEpi)) { ok = false; break; }
+          pend[b] = -1;                              // the math warps saw this slice's input land
+          if (!final_w) {
+            // stores start inside the tensor only (a pair tile can overhang the
+            // 128-padded edge by half; the overhang is never stored)
+            const int ocols = T.mode != kModeUpdate ? C.kp : C.lp;
+            const int x0 = T.tn * kTile + 64 * h;
+            if (row0 < C.kp && x0 < ocols) tma_store_3d(output_map(T), slice_buf(b), x0, row0, T.b);
+            tma_store_commit();
+            if constexpr (nbuf == 4) {
+              tma_store_wait_read1();                // the previous slice's buffer is free again
+              const int nx = gs - 1 + nbuf;          // slices 0..3 were armed before the loop
+              if (gs >= 1 && nx < my_slices) prepare(nx, tile_of(nx >> 2));
+              continue;
+            }
+            tma_store_wait_read0();                  // buffers b readable again
+          }
+          if (gs + nbuf < my_slices) prepare(gs + nbuf, tile_of((gs + nbuf) >> 2));
+        }
+        tma_store_wait_all0();
+        release_stg(gc);
       }
       tma_store_wait_all0();
-      release_stg(gc);
       for (int b = 0; b < nbuf; ++b)
         if (pend[b] >= 0) mbar_wait(&ctl->in_full[b], (uint32_t)pend[b], wc, kDevTimeoutDrain);
       aborted = !ok;
@@ -650,19 +770,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     // ---------------------------------------------------- epilogue math
     const int q = warp & 3;                       // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;                  // tile row owned by this thread
-    int it = 0, gs = 0, gc = 0;
+    int gs = 0, gc = 0;
     bool ok = true;
-    for (int t = cid; t < p.total_tiles && ok; t += ncl, ++it) {
-      const TileCoord tc = decode_tile(p, t, sym);
-      const GemmClass& C = p.cls[tc.cls];
-      const int mat = C.mat_first + tc.b;
+    for (int it = 0; it < my_tiles && ok; ++it) {
+      const Tile T = tile_of(it);
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)((it >> 1) & 1);
       ok = __all_sync(0xffffffffu, mbar_wait(&ctl->tmem_full[acc], acc_phase, wc, kDevTimeoutAccum));
       if (!ok) break;
       tc_fence_after();
-      const float s = p.first ? p.scale[mat] : 1.0f;
-      const int row0 = tc.tm * kTile + (int)rank * kBM;
+      const float s = T.first ? p.scale[T.mat] : 1.0f;
+      const int row0 = T.tm * kTile + (int)rank * kBM;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
 #pragma unroll 1
       for (int h = 0; h < 4 && ok; ++h, ++gs) {
@@ -677,10 +795,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(mapa_shared(&ctl->tmem_empty[acc], 0));
         }
-        if (kMode != kModePoly) {
+        if (T.mode != kModePoly) {
           // Gram: s^2 X X^T.  Update: s (aI + B) X = a s X + s B X, the aI term
           // carried on the diagonal of the polynomial phase's output.
-          const float alpha = kMode == kModeGram ? s * s : s;
+          const float alpha = T.mode == kModeGram ? s * s : s;
 #pragma unroll
           for (int i = 0; i < 64; ++i) v[i] *= alpha;
         } else {
@@ -699,7 +817,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           // + a on the diagonal: on a diagonal tile, a warp's 32 rows meet the
           // slice's columns at 32 consecutive columns starting at dbase, lane by lane
           const int dbase = (int)rank * kBM + q * 32 - 64 * h;
-          if (tc.tm == tc.tn && (dbase == 0 || dbase == 32)) {
+          if (T.tm == T.tn && (dbase == 0 || dbase == 32)) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               if (j == lane) {
@@ -709,7 +827,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           }
         }
         if (final_w) {
-          const OutMat& O = p.out[mat];
+          const OutMat& O = p.out[T.mat];
 #pragma unroll
           for (int sub = 0; sub < 2; ++sub, ++gc) {
             const int sidx = gc % kStgBufs;
@@ -750,7 +868,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
                 for (int i = 0; i < 32; ++i) Sf[i * kBM + r] = vv[i];
               }
               __syncwarp();
-              store_w_slice_warp(O, Sf, row0, tc.tn * kTile + 64 * h + 32 * sub, q, lane, p.lr, p.assign);
+              store_w_slice_warp(O, Sf, row0, T.tn * kTile + 64 * h + 32 * sub, q, lane, p.lr, p.assign);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->stg_full[sidx]);

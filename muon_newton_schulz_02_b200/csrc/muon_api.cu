@@ -18,11 +18,14 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <list>
 #include <map>
 #include <memory>
 #include <mutex>
+#include <queue>
+#include <set>
 #include <string>
 #include <vector>
 
@@ -83,7 +86,7 @@ struct Group {
   std::vector<ClassDesc> classes;
   std::vector<int> pro_tile_begin;
   int pro_tiles = 0;
-  size_t off_partials = 0, off_tickets = 0, off_scale = 0, off_tmaps = 0, off_wmaps = 0;
+  size_t off_partials = 0, off_tickets = 0, off_scale = 0, off_done = 0, off_tmaps = 0, off_wmaps = 0;
   size_t data_bytes = 0;
   int sym_tiles = 0, upd_tiles = 0;
   std::vector<GemmClass> sym_cls, upd_cls;
@@ -95,6 +98,17 @@ struct Group {
 // plan may place anything else there.
 constexpr size_t kTicketBytes = 4096;
 static_assert(kMaxMats * 4 <= kTicketBytes, "ticket region too small");
+
+// Work lists of one chained launch (see ns_gemm_kernel<..., true>) for one
+// group and one iteration count, in device memory: the items of every
+// cluster back to back, then the cluster offsets.
+struct ChainTables {
+  int nclusters = 0;
+  int nitems = 0;
+  void* dev = nullptr;
+  const WorkItem* items = nullptr;
+  const int* off = nullptr;
+};
 
 struct Plan {
   std::vector<int64_t> shapes;
@@ -110,8 +124,11 @@ struct Plan {
   std::vector<std::vector<const void*>> wmap_key;
   std::vector<CUtensorMap*> wmap_host;
   cudaEvent_t wmap_copied = nullptr;
+  std::map<std::pair<size_t, int>, ChainTables> chains;   // (group, ns_steps) -> work lists
   ~Plan() {
     if (tmaps) cudaFree(tmaps);
+    for (auto& kv : chains)
+      if (kv.second.dev) cudaFree(kv.second.dev);
     for (auto h : wmap_host)
       if (h) cudaFreeHost(h);
     if (wmap_copied) cudaEventDestroy(wmap_copied);
@@ -190,6 +207,7 @@ int build_layout(const int64_t* shapes, int n, Plan& plan) {
     }
     g.off_partials = off; off = align_up(off + (size_t)g.pro_tiles * 4, 1024);
     g.off_scale = off; off = align_up(off + g.mats.size() * 4, 1024);
+    g.off_done = off; off = align_up(off + g.mats.size() * 4, 1024);
     g.data_bytes = off;
     data_max = std::max(data_max, off);
     // GEMM tile bookkeeping
@@ -228,6 +246,135 @@ int build_layout(const int64_t* shapes, int n, Plan& plan) {
   plan.tmap_bytes = off;
   plan.ws_bytes = data_max;
   return MUON_OK;
+}
+
+// ------------------------------------------------------ chained schedule ---
+// Host-side list scheduling of the chained launch.  Every matrix runs the
+// chain Gram(0), poly(0), update(0), Gram(1), ..., poly(n-1) (the last update
+// runs in its own launch); each phase's tiles may start only once all tiles of
+// the previous phase of that matrix are done.  A simulation of `ncl` clusters
+// assigns tiles greedily: a free cluster takes the next tile of the
+// highest-priority matrix whose current phase is ready (larger matrices first),
+// so a matrix's phases follow each other closely and its operands stay in L2
+// while other matrices fill the gaps.  Tile cost is modelled as its K-blocks
+// plus a fixed overhead; a finished tile is visible to dependants `lat` units
+// later (epilogue, store, and the producer running ahead of the MMAs).
+//
+// Each cluster's list is in order of simulated start time, and every item's
+// inputs come from items with strictly earlier simulated start times, so with
+// all clusters resident some list head can always proceed: the lists cannot
+// deadlock.  `need` counts tile halves (each CTA of a pair publishes its own).
+double chain_latency_units() {
+  static double lat = -1.0;
+  if (lat < 0.0) {
+    const char* e = std::getenv("MUON_CHAIN_LATENCY");
+    lat = e ? std::max(0.0, std::atof(e)) : 12.0;
+  }
+  return lat;
+}
+
+void build_chain(const Group& g, int ns_steps, int ncl, std::vector<WorkItem>& items, std::vector<int>& off) {
+  constexpr double kOverhead = 2.0;
+  const double lat = chain_latency_units();
+  const int nm = (int)g.mats.size();
+  const int nphases = 3 * ns_steps - 1;
+  struct MatState {
+    int cls = 0, b = 0, T = 0, Tn = 0;
+    int ntiles[3] = {0, 0, 0};
+    double cost[3] = {0, 0, 0};
+    int phase = 0, next = 0;
+    int need = 0;              // tile halves completed before the current phase
+    double vis = 0.0;          // latest visibility time among the current phase's tiles
+    double total = 0.0;
+  };
+  std::vector<MatState> ms(nm);
+  for (size_t ci = 0; ci < g.classes.size(); ++ci) {
+    const ClassDesc& cd = g.classes[ci];
+    for (size_t b = 0; b < cd.mats.size(); ++b) {
+      MatState& st = ms[cd.mats[b]];
+      st.cls = (int)ci;
+      st.b = (int)b;
+      st.T = (cd.kp + kTile - 1) / kTile;
+      st.Tn = (cd.lp + kTile - 1) / kTile;
+      st.ntiles[kModeGram] = st.ntiles[kModePoly] = st.T * (st.T + 1) / 2;
+      st.ntiles[kModeUpdate] = st.T * st.Tn;
+      st.cost[kModeGram] = cd.lp / kBK + kOverhead;
+      st.cost[kModePoly] = st.cost[kModeUpdate] = cd.kp / kBK + kOverhead;
+      for (int j = 0; j < nphases; ++j) st.total += st.ntiles[j % 3] * st.cost[j % 3];
+    }
+  }
+  // priority: more total work first (its long chain starts early), then group order
+  std::vector<int> by_prio(nm);
+  for (int i = 0; i < nm; ++i) by_prio[i] = i;
+  std::stable_sort(by_prio.begin(), by_prio.end(), [&](int x, int y) { return ms[x].total > ms[y].total; });
+  std::vector<int> prio(nm);
+  for (int r = 0; r < nm; ++r) prio[by_prio[r]] = r;
+
+  std::vector<std::vector<WorkItem>> lists(ncl);
+  std::priority_queue<std::pair<double, int>, std::vector<std::pair<double, int>>, std::greater<>> free_at;
+  for (int c = 0; c < ncl; ++c) free_at.push({0.0, c});
+  std::set<std::pair<double, int>> pending;   // (ready time, priority) of a matrix's next phase
+  std::set<int> avail;                        // priorities of matrices with ready, unassigned tiles
+  for (int m = 0; m < nm; ++m)
+    if (nphases > 0) avail.insert(prio[m]);
+  long long left = 0;
+  for (int m = 0; m < nm; ++m)
+    for (int j = 0; j < nphases; ++j) left += ms[m].ntiles[j % 3];
+  while (left > 0) {
+    auto [t, c] = free_at.top();
+    free_at.pop();
+    auto admit = [&](double now) {
+      while (!pending.empty() && pending.begin()->first <= now) {
+        avail.insert(pending.begin()->second);
+        pending.erase(pending.begin());
+      }
+    };
+    admit(t);
+    if (avail.empty()) {                      // this cluster idles until a phase becomes ready
+      t = std::max(t, pending.begin()->first);
+      admit(t);
+    }
+    const int m = by_prio[*avail.begin()];
+    MatState& st = ms[m];
+    const int mode = st.phase % 3;
+    int tm, tn;
+    if (mode == kModeUpdate) {
+      tm = st.next / st.Tn;
+      tn = st.next % st.Tn;
+    } else {                                  // upper-triangle 256-blocks, row by row
+      int r = st.next, row = 0, len = st.T;
+      while (r >= len) { r -= len; ++row; --len; }
+      tm = row;
+      tn = row + r;
+    }
+    WorkItem w{};
+    w.need = st.need;
+    w.mat = (unsigned short)m;
+    w.b = (unsigned short)st.b;
+    w.tm = (unsigned short)tm;
+    w.tn = (unsigned short)tn;
+    w.cls = (unsigned char)st.cls;
+    w.mode = (unsigned char)mode;
+    w.it = (unsigned short)(st.phase / 3);
+    lists[c].push_back(w);
+    const double end = t + st.cost[mode];
+    st.vis = std::max(st.vis, end + lat);
+    free_at.push({end, c});
+    --left;
+    if (++st.next == st.ntiles[mode]) {       // phase fully assigned: the next one is ready at st.vis
+      avail.erase(prio[m]);
+      st.need += 2 * st.ntiles[mode];
+      st.next = 0;
+      if (++st.phase < nphases) pending.insert({st.vis, prio[m]});
+      st.vis = 0.0;
+    }
+  }
+  items.clear();
+  off.assign(1, 0);
+  for (int c = 0; c < ncl; ++c) {
+    items.insert(items.end(), lists[c].begin(), lists[c].end());
+    off.push_back((int)items.size());
+  }
 }
 
 int encode_map(CUtensorMap* map, void* base, int cols, int rows, int batch, int box_cols, int box_rows) {
@@ -278,9 +425,11 @@ cudaError_t launch_pdl(void (*kernel)(Args), dim3 grid, dim3 block, size_t smem,
   return cudaLaunchKernelEx(&cfg, kernel, args);
 }
 
-// One NS-phase launch: persistent clusters of two CTAs (one CTA per SM).
-cudaError_t launch_gemm(cudaStream_t stream, const GemmArgs& args, int sm_count) {
-  const int pairs = std::max(1, std::min(args.total_tiles, sm_count / 2));
+// One GEMM launch: persistent clusters of two CTAs (one CTA per SM).  With
+// `chain_clusters` > 0 it is the chained launch over that many clusters (every
+// phase but the last update); otherwise one Newton-Schulz phase (args.mode).
+cudaError_t launch_gemm(cudaStream_t stream, const GemmArgs& args, int sm_count, int chain_clusters = 0) {
+  const int pairs = chain_clusters > 0 ? chain_clusters : std::max(1, std::min(args.total_tiles, sm_count / 2));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
@@ -295,12 +444,13 @@ cudaError_t launch_gemm(cudaStream_t stream, const GemmArgs& args, int sm_count)
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  if (chain_clusters > 0) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false, true>, args);
   switch (args.mode) {
-    case kModeGram: return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false>, args);
-    case kModePoly: return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModePoly, false>, args);
+    case kModeGram: return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false, false>, args);
+    case kModePoly: return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModePoly, false, false>, args);
     default:
-      return args.final_apply ? cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeUpdate, true>, args)
-                              : cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeUpdate, false>, args);
+      return args.final_apply ? cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeUpdate, true, false>, args)
+                              : cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeUpdate, false, false>, args);
   }
 }
 
@@ -341,6 +491,7 @@ struct Ctx {
 
 std::map<std::pair<int, void*>, std::unique_ptr<Ctx>> g_ctx;
 std::map<int, bool> g_dev_ready;
+std::map<int, int> g_chain_clusters;      // per device: clusters of two CTAs that can be resident at once
 
 int device_setup(int dev) {
   if (g_dev_ready[dev]) return MUON_OK;
@@ -351,14 +502,38 @@ int device_setup(int dev) {
                                      std::to_string(prop.major) + std::to_string(prop.minor));
   CUDA_TRY(cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallSmem));
   CUDA_TRY(cudaFuncSetAttribute(ns_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem));
-  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kGemmSmemBytes));
-  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModePoly, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModePoly, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kGemmSmemBytes));
-  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeUpdate, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeUpdate, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kGemmSmemBytes));
-  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeUpdate, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeUpdate, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kGemmSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kGemmSmemBytes));
+  {
+    // The chained launch's clusters wait on one another's results, so all of
+    // them must be resident at once: never launch more than the device holds.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(prop.multiProcessorCount, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = kGemmSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, (void*)ns_gemm_kernel<kModeGram, false, true>, &cfg) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      nclusters = 0;                         // chained launch unavailable: one launch per phase
+    }
+    g_chain_clusters[dev] = std::min(nclusters, prop.multiProcessorCount / 2);
+  }
   g_dev_ready[dev] = true;
   return MUON_OK;
 }
@@ -464,7 +639,8 @@ cudaEvent_t pool_event(Ctx& c) {
 // NVTX range names of the launch kinds (MUON_KIND_*), for timeline tools; the
 // ranges cost nothing when no tool is attached.
 const char* const kKindNames[MUON_NUM_KINDS] = {"muon.prologue", "muon.gram", "muon.poly", "muon.update",
-                                                "muon.update_apply", "muon.apply_x0", "muon.small", "muon.pair"};
+                                                "muon.update_apply", "muon.apply_x0", "muon.small", "muon.pair",
+                                                "muon.chain"};
 
 template <class F>
 int launch(Ctx& c, int kind, F&& f) {
@@ -532,12 +708,44 @@ int update_wmaps(Ctx& c, Plan& plan, size_t gi, const StepIO& io) {
   return MUON_OK;
 }
 
+// The chained launch's work lists for group gidx and ns_steps iterations,
+// built and uploaded on first use (a synchronous copy: make the first call for
+// a set of shapes and an iteration count outside stream capture).
+int get_chain(Ctx& c, Plan& plan, size_t gidx, int ns_steps, ChainTables** out) {
+  const auto key = std::make_pair(gidx, ns_steps);
+  auto it = plan.chains.find(key);
+  if (it == plan.chains.end()) {
+    ChainTables ct;
+    ct.nclusters = g_chain_clusters[c.dev];
+    std::vector<WorkItem> items;
+    std::vector<int> off;
+    build_chain(plan.groups[gidx], ns_steps, ct.nclusters, items, off);
+    ct.nitems = (int)items.size();
+    const size_t ib = align_up(items.size() * sizeof(WorkItem), 256), ob = off.size() * sizeof(int);
+    if (cudaMalloc(&ct.dev, ib + ob) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(MUON_ERR_NOMEM, "work-list allocation failed");
+    }
+    it = plan.chains.emplace(key, ct).first;   // owned by the plan from here on
+    CUDA_TRY(cudaMemcpy(ct.dev, items.data(), items.size() * sizeof(WorkItem), cudaMemcpyHostToDevice));
+    CUDA_TRY(cudaMemcpy((char*)ct.dev + ib, off.data(), ob, cudaMemcpyHostToDevice));
+    it->second.items = (const WorkItem*)ct.dev;
+    it->second.off = (const int*)((char*)ct.dev + ib);
+  }
+  *out = &it->second;
+  return MUON_OK;
+}
+
 int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
   const Group& g = plan.groups[gidx];
   char* base = (char*)c.ws;
   float* scale = (float*)(base + g.off_scale);
   const CUtensorMap* tmaps = (const CUtensorMap*)((char*)plan.tmaps + g.off_tmaps);
   const int nm = (int)g.mats.size();
+  unsigned* done = (unsigned*)(base + g.off_done);
+  // every phase but the last update in one chained launch, unless the device
+  // cannot hold its clusters or a test asks for one launch per phase
+  const bool chain = io.ns_steps >= 1 && g_chain_clusters[c.dev] > 0 && !(g_debug_flags & 4);
 
   // 1. prologue
   {
@@ -552,6 +760,7 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
     pa->partials = (float*)(base + g.off_partials);
     pa->tickets = (unsigned*)(base + g.off_tickets);
     pa->scale = scale;
+    pa->done = chain ? done : nullptr;
     for (const auto& cd : g.classes) {
       for (size_t b = 0; b < cd.mats.size(); ++b) {
         const int gi = cd.mats[b];
@@ -616,6 +825,32 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
   ga->a = io.a; ga->b = io.b; ga->c = io.c; ga->lr = io.lr;
   ga->assign = io.assign;
   fill_out(ga->out);
+
+  if (chain) {
+    ChainTables* ct = nullptr;
+    int rc = get_chain(c, plan, gidx, io.ns_steps, &ct);
+    if (rc) return rc;
+    for (size_t ci = 0; ci < g.sym_cls.size(); ++ci) ga->cls[ci] = g.sym_cls[ci];
+    ga->items = ct->items;
+    ga->item_off = ct->off;
+    ga->done = done;
+    ga->debug_flags = 0;
+    if (g_debug_flags & 1) { ga->debug_flags = 1; g_debug_flags &= ~1; }
+    rc = launch(c, MUON_KIND_CHAIN, [&] { launch_gemm(c.stream, *ga, c.sm_count, ct->nclusters); });
+    if (rc) return rc;
+    // the last update, with W -= lr*O fused, in its own launch
+    for (size_t ci = 0; ci < g.upd_cls.size(); ++ci) ga->cls[ci] = g.upd_cls[ci];
+    ga->items = nullptr;
+    ga->item_off = nullptr;
+    ga->done = nullptr;
+    ga->total_tiles = g.upd_tiles;
+    ga->mode = kModeUpdate;
+    ga->x_in = (io.ns_steps - 1) & 1;
+    ga->first = io.ns_steps == 1;
+    ga->final_apply = 1;
+    ga->debug_flags = 0;
+    return launch(c, MUON_KIND_UPDATE_APPLY, [&] { launch_gemm(c.stream, *ga, c.sm_count); });
+  }
 
   for (int it = 0; it < io.ns_steps; ++it) {
     for (int mode = kModeGram; mode <= kModeUpdate; ++mode) {
@@ -951,6 +1186,37 @@ int muon_profile_read(double* ms, int64_t* launches, int nkinds) {
 }
 
 int64_t muon_launch_count(void) { return g_launches.load(); }
+
+int muon_chain_plan(const int64_t* shapes, int n, int ns_steps, int nclusters, int32_t* items, int64_t capacity,
+                    int32_t* cluster_off, int64_t* nitems) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int rc = validate_common(shapes, n, ns_steps);
+  if (rc) return rc;
+  if (!nitems || !cluster_off || nclusters < 1 || nclusters > 4096)
+    return fail(MUON_ERR_INVALID_ARG, "nitems and cluster_off must be given, 1 <= nclusters <= 4096");
+  Plan plan;
+  if ((rc = build_layout(shapes, n, plan))) return rc;
+  *nitems = 0;
+  if (plan.groups.empty() || ns_steps < 1) {
+    for (int c = 0; c <= nclusters; ++c) cluster_off[c] = 0;
+    return MUON_OK;
+  }
+  std::vector<WorkItem> list;
+  std::vector<int> off;
+  build_chain(plan.groups[0], ns_steps, nclusters, list, off);
+  *nitems = (int64_t)list.size();
+  for (int c = 0; c <= nclusters; ++c) cluster_off[c] = off[c];
+  if (!items || capacity < (int64_t)list.size())
+    return fail(MUON_ERR_INVALID_ARG, "items holds fewer than " + std::to_string(list.size()) + " entries");
+  const Group& g = plan.groups[0];
+  for (size_t i = 0; i < list.size(); ++i) {
+    const WorkItem& w = list[i];
+    int32_t* o = items + 8 * i;
+    o[0] = w.need; o[1] = g.mats[w.mat].user; o[2] = w.cls; o[3] = w.b;
+    o[4] = w.tm; o[5] = w.tn; o[6] = w.mode; o[7] = w.it;
+  }
+  return MUON_OK;
+}
 
 int muon_debug_set(int flags, int64_t wait_limit_ns) {
   std::lock_guard<std::mutex> lk(g_mu);

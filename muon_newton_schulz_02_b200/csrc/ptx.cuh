@@ -24,6 +24,7 @@ enum DeviceError : int {
   kDevTimeoutAccum = 3,     // waited too long for an accumulator
   kDevTimeoutEpi = 4,       // waited too long for an epilogue input tile
   kDevTimeoutDrain = 5,     // waited too long for in-flight copies at exit
+  kDevTimeoutDep = 6,       // waited too long for another tile's results (chained launch)
 };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -189,6 +190,36 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
       : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return done != 0;
+}
+
+// ------------------------------------------ cross-CTA completion counters ---
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const unsigned* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(unsigned* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Orders this thread's generic-proxy accesses to global memory against its
+// async-proxy (TMA) accesses: after TMA stores complete, before a release that
+// publishes them; after an acquire, before TMA loads of what it published.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Wait until *ctr >= target, bounded by w.limit_ns (see mbar_wait).
+__device__ __forceinline__ bool wait_count(const unsigned* ctr, uint32_t target, const WaitCtx& w, int code) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(32);
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if (*w.abort_flag) return false;
+    if (globaltimer_ns() - t0 > w.limit_ns) {
+      raise_error(w, code);
+      return false;
+    }
+  }
 }
 
 // ------------------------------------------------------------------ TMA ---

@@ -68,7 +68,11 @@ def o_from_w(W_old, W_new, lr):
 
 def check_band(O, G, svd_device="cpu"):
     """Every singular value of O <= BAND_HI; no more values below BAND_LO than
-    normalised input singular values below X_THRESHOLD."""
+    normalised input singular values below X_THRESHOLD.  An output singular
+    value counts as below BAND_LO only if it is below it by more than the
+    parity tolerance REL_O: an input just above the threshold maps to just
+    above 0.6 in exact arithmetic, and the bf16 iteration may move it by that
+    much."""
     if svd_device == "cpu":
         so = np.linalg.svd(np.asarray(O, np.float64), compute_uv=False)
         sg = np.linalg.svd(np.asarray(G, np.float64), compute_uv=False)
@@ -77,7 +81,7 @@ def check_band(O, G, svd_device="cpu"):
         sg = torch.linalg.svdvals(torch.as_tensor(G, device=svd_device, dtype=torch.float64)).cpu().numpy()
     x = sg / (np.sqrt((sg ** 2).sum()) + 1e-7)
     n_small_in = int((x < X_THRESHOLD).sum())
-    n_low_out = int((so < BAND_LO).sum())
+    n_low_out = int((so < BAND_LO * (1 - REL_O)).sum())
     assert so.max() <= BAND_HI, f"max singular value {so.max():.5f} above {BAND_HI}"
     assert n_low_out <= n_small_in, f"{n_low_out} singular values < {BAND_LO}, only {n_small_in} inputs below threshold"
     return so

@@ -62,8 +62,9 @@ def _expect_ws(shapes):
     """Layout documented in the C source: a fixed 4 KiB region of norm
     arrival counters, then per shape class (padded short side kp, long side
     lp, both multiples of 128) two bf16 iterates [B][kp][lp] and two bf16
-    [B][kp][kp] matrices, then per-tile norm partials (64x128 tiles) and
-    per-matrix scales, each region rounded to 1 KiB.  Matrices that a fused
+    [B][kp][kp] matrices, then per-tile norm partials (64x128 tiles),
+    per-matrix scales and per-matrix completion counters (of the chained
+    launch), each region rounded to 1 KiB.  Matrices that a fused
     kernel runs whole (short side <= 128 and long side <= 512 on one CTA, or
     short side <= 256 and long side <= 256 on a CTA pair) take none."""
     up = lambda v, a: (v + a - 1) // a * a
@@ -86,6 +87,7 @@ def _expect_ws(shapes):
         tiles += b * (kp // 64) * (lp // 128)
     n = sum(len(v) for v in classes.values())
     off = up(off + tiles * 4, 1024)
+    off = up(off + n * 4, 1024)
     off = up(off + n * 4, 1024)
     return off
 

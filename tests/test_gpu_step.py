@@ -233,3 +233,28 @@ def test_nan_and_inf_propagate(poison):
         ok = [i for i in range(len(shapes)) if i != bad]
         _check_step([W[i] for i in ok], [g[i] for i in ok], [b[i] for i in ok],
                     [W_new[i] for i in ok], [b_new[i] for i in ok])
+
+
+@pytest.mark.parametrize("ns_steps", [1, 2, 5])
+def test_chained_launch_matches_one_launch_per_phase_bitwise(ns_steps):
+    # The chained launch computes every tile exactly as the per-phase launches
+    # do (same operands, same K order, same epilogue); only the order in which
+    # tiles run differs.  So both give bitwise the same weights and buffers.
+    shapes = [(768, 768)] * 3 + [(768, 3072), (3072, 768), (640, 1920), (1000, 300), (384, 384), (1600, 1600)]
+    W, g, b = _inputs(shapes, 41, gscale=0.02)
+    muon.profile_enable(True)
+    try:
+        muon.profile_read()
+        r_chain = gpu_step(W, g, b, 0.02, 0.95, ns_steps=ns_steps)
+        kinds = muon.profile_read()
+        assert kinds["chain"][1] == 1 and kinds["gram"][1] == 0     # the chained launch ran
+        muon.debug_set(4, 0)
+        r_phase = gpu_step(W, g, b, 0.02, 0.95, ns_steps=ns_steps)
+        kinds = muon.profile_read()
+        assert kinds["chain"][1] == 0 and kinds["gram"][1] == ns_steps
+    finally:
+        muon.debug_set(0, 0)
+        muon.profile_enable(False)
+    for x, y in zip(r_chain[0] + r_chain[1], r_phase[0] + r_phase[1]):
+        assert np.array_equal(x, y)
+    _check_step(W, g, b, r_chain[0], r_chain[1], steps=ns_steps)
