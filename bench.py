@@ -555,6 +555,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
+        "chain_clusters": muon.chain_clusters(),
         "clocks": clk,
         "step_times": {"ms_median": statistics.median(per_step), "ms_min": min(per_step), "ms_max": max(per_step),
                        "ms_cold_l2_median": statistics.median(cold) if cold else None,

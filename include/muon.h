@@ -34,8 +34,10 @@
  *     of shapes outside capture) and freed by muon_release().
  *   - Matrices with short side <= 128 and long side <= 512, or with both
  *     sides <= 256, run their whole step in one fused launch (one CTA, or
- *     a cluster of two CTAs, per matrix) and use no workspace; the others
- *     run as one launch per Newton-Schulz phase over all of them.
+ *     a cluster of two CTAs, per matrix) and use no workspace.  The others
+ *     run the momentum/norm/cast prologue, then every Newton-Schulz phase and
+ *     the weight update in one chained launch (short side <= 1024), or one
+ *     launch per phase (larger matrices).
  *   - Concurrent calls on different streams use different workspaces; calls
  *     on one stream are serialised by the stream.
  *   - NaN / Inf in the inputs propagate to the outputs; nothing checks them.
@@ -178,7 +180,7 @@ void muon_release(void);
 #define MUON_KIND_APPLY_X0 5
 #define MUON_KIND_SMALL 6        /* fused single-CTA step of small matrices */
 #define MUON_KIND_PAIR 7         /* fused CTA-pair step, 128 < short side <= 256, long side <= 256 */
-#define MUON_KIND_CHAIN 8        /* every Newton-Schulz phase but the last update, one chained launch */
+#define MUON_KIND_CHAIN 8        /* every Newton-Schulz phase and the weight update, one chained launch */
 #define MUON_NUM_KINDS 9
 
 /* 1: bracket every kernel launch with CUDA events on its stream; 0: stop. */
@@ -189,6 +191,9 @@ int muon_profile_enable(int enable);
 int muon_profile_read(double* ms, int64_t* launches, int nkinds);
 /* Number of kernels this library has launched since it was loaded. */
 int64_t muon_launch_count(void);
+/* Clusters of two CTAs the chained launch runs on the current device (the
+ * most that can be resident at once), or -1 if the device cannot be used. */
+int muon_chain_clusters(void);
 
 /* ---- test hooks -------------------------------------------------------- */
 
@@ -208,7 +213,8 @@ int muon_debug_set(int flags, int64_t wait_limit_ns);
  * of matrices (at most 320 matrices over 16 padded shapes; matrices the fused
  * kernels run whole take no part).  Item i is items[8i .. 8i+7] = {need,
  * matrix (the caller's index), shape class, index in class, tile row, tile
- * column, phase (0 Gram, 1 polynomial, 2 update), iteration}; cluster c runs
+ * column, phase (0 Gram, 1 polynomial, 2 update, 3 the last update with
+ * W -= lr*O), iteration}; cluster c runs
  * items [cluster_off[c], cluster_off[c + 1]) in order (cluster_off holds
  * nclusters + 1 entries).  *nitems receives the item count;
  * MUON_ERR_INVALID_ARG if `capacity` (in items) is smaller. */

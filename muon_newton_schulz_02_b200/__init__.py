@@ -20,7 +20,7 @@ from array import array
 
 __all__ = [
     "step", "PreparedStep", "orthogonalize", "step_host", "step_noalloc", "workspace_size", "sync_status", "last_error", "release",
-    "profile_enable", "profile_read", "launch_count", "debug_set", "chain_plan", "lib", "MuonError", "KINDS",
+    "profile_enable", "profile_read", "launch_count", "chain_clusters", "debug_set", "chain_plan", "lib", "MuonError", "KINDS",
     "NS_A", "NS_B", "NS_C", "NS_STEPS", "NS_EPS", "LIB_PATH", "header_functions",
 ]
 
@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
     L.muon_profile_read.restype = ctypes.c_int
     L.muon_launch_count.argtypes = []
     L.muon_launch_count.restype = ctypes.c_int64
+    L.muon_chain_clusters.argtypes = []
+    L.muon_chain_clusters.restype = ctypes.c_int
     L.muon_debug_set.argtypes = [ctypes.c_int, ctypes.c_int64]
     L.muon_debug_set.restype = ctypes.c_int
     L.muon_chain_plan.argtypes = [_I64P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int32),
@@ -268,6 +270,11 @@ def profile_read() -> dict:
 
 def launch_count() -> int:
     return int(lib().muon_launch_count())
+
+
+def chain_clusters() -> int:
+    """Clusters of two CTAs the chained launch uses on the current device."""
+    return int(lib().muon_chain_clusters())
 
 
 def debug_set(flags: int = 0, wait_limit_ns: int = 0):

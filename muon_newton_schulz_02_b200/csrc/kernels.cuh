@@ -51,7 +51,8 @@ enum TmapSlot : int {
   kTmA = 4, kTmB = 5,               // Gram / polynomial matrices, 64 x 128 boxes
   kTmAmn = 6, kTmBmn = 7            // Gram / polynomial matrices, 64 x 64 boxes (transposed operand reads)
 };
-enum GemmMode : int { kModeGram = 0, kModePoly = 1, kModeUpdate = 2 };
+enum GemmMode : int { kModeGram = 0, kModePoly = 1, kModeUpdate = 2,
+                      kModeFinal = 3 };   // work items only: the last update, with W -= lr*O
 
 constexpr uint32_t kStageABytes = kBM * kBK * 2;     // 16 KB
 constexpr uint32_t kStageBBytes = kBNh * kBK * 2;    // 16 KB
@@ -59,11 +60,6 @@ constexpr uint32_t kStageBytes = kStageABytes + kStageBBytes;
 constexpr uint32_t kSliceBytes = kBM * 64 * 2;       // 16 KB: 128 rows x 64 cols bf16 (one TMA box)
 constexpr uint32_t kSmemDataBytes = kStages * kStageBytes + 4 * kSliceBytes;
 constexpr uint32_t kSmemCtrlBytes = 512;
-// Final update: fp32 staging ring for the W add-reductions (the two slice
-// buffers plus the two the other phases use for slices 2 and 3), and how many
-// add-reductions stay in flight behind the newest one.
-constexpr int kStgBufs = 4;
-constexpr int kStgLag = 1;
 constexpr uint32_t kGemmSmemBytes = kSmemDataBytes + kSmemCtrlBytes + 1024;  // + alignment slack
 
 // ------------------------------------------------------------ arguments ---
@@ -97,7 +93,7 @@ struct WorkItem {
                             // completed before this item reads its inputs
   unsigned short mat, b;    // matrix (group order), its index within its shape class
   unsigned short tm, tn;    // output tile row and column (256-blocks)
-  unsigned char cls, mode;  // shape class, kModeGram / kModePoly / kModeUpdate
+  unsigned char cls, mode;  // shape class, kModeGram / kModePoly / kModeUpdate / kModeFinal
   unsigned short it;        // Newton-Schulz iteration
 };
 static_assert(sizeof(WorkItem) == 16, "WorkItem layout");
@@ -337,6 +333,7 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& p, int t, bool 
 // One output tile as every role of the GEMM kernel sees it.
 struct Tile {
   int mode;       // kModeGram / kModePoly / kModeUpdate
+  int fin;        // the last update: the epilogue adds -lr*O into W
   int cls, b;     // shape class, matrix within the class
   int tm, tn;     // 256-block row and column of the output
   int x_in;       // which ping-pong iterate holds X (iteration parity)
@@ -385,17 +382,14 @@ struct __align__(8) GemmCtrl {
   uint64_t empty[kStages];    // the pair MMAs reading a stage are done (both CTAs)
   uint64_t tmem_full[2];      // an accumulator is ready (both CTAs)
   uint64_t tmem_empty[2];     // even CTA: all 8 epilogue math warps of the pair drained an accumulator
-  uint64_t in_full[4];        // DMA -> math: slice buffer set ready (input slice landed, or just free)
-  uint64_t out_full[4];       // math -> DMA: slice staged (and input slice consumed)
-  uint64_t stg_full[kStgBufs];  // math -> DMA: fp32 result chunk staged (final update)
-  uint64_t stg_free[kStgBufs];  // DMA -> math: fp32 staging buffer free again
+  uint64_t in_full[4];        // DMA -> math: chunk buffer handed over (its input slice landed, if any)
+  uint64_t out_full[4];       // math -> DMA: chunk staged (and its input consumed)
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 static_assert(sizeof(GemmCtrl) <= kSmemCtrlBytes, "GemmCtrl does not fit its shared-memory slot");
 static_assert(kGemmSmemBytes <= 232448, "more dynamic shared memory than a CTA may have");
-static_assert(kStgLag >= 1 && kStgLag < kStgBufs, "staging ring");
 
 // The Newton-Schulz GEMM kernel.  A cluster of two CTAs (one per SM) computes
 // 256 x 256 output tiles with tcgen05.mma.cta_group::2: each CTA loads its 128
@@ -404,26 +398,29 @@ static_assert(kStgLag >= 1 && kStgLag < kStgBufs, "staging ring");
 // rows x 256 fp32 columns (two accumulators, double-buffered).  Roles per CTA:
 // warp 0 TMA producer; warp 1 MMA issuer (even CTA) and TMEM allocator; warp 2
 // epilogue DMA (loads the polynomial epilogue's A slices, issues the TMA
-// stores / add-reductions of the output slices and recycles their buffers);
-// warps 3..6 epilogue math (per 64-column slice: tcgen05.ld -> fp32 math ->
-// bf16 -> 128B-swizzled smem).  The math warps hand slices to the DMA warp
-// through mbarriers and never wait on TMA latency themselves.
+// stores / add-reductions of the output and recycles their buffers); warps
+// 3..6 epilogue math (tcgen05.ld -> fp32 math -> bf16 or fp32 -> 128B-swizzled
+// smem).  The math warps hand output chunks to the DMA warp through a ring of
+// four 16 KB buffers and mbarriers, and never wait on TMA latency themselves:
+// an ordinary tile is 4 chunks (bf16 64-column slices), a tile of the last
+// update 8 chunks (fp32 32-column halves of a slice, added into W in L2).
 //
 // Two ways to launch it:
 //   kChain = false: one launch per phase (kMode) over all matrices of a group,
 //     persistent, tile t to cluster t mod #clusters; kFinal selects the last
 //     update, whose epilogue adds -lr*O into W.
-//   kChain = true: one launch for every phase of every iteration but the last
-//     update.  Each cluster runs its own list of work items (any phase, any
-//     matrix; the host orders the lists so that items are ready in time);
-//     before reading a matrix's Gram, polynomial or iterate it waits (bounded)
-//     for the counter of completed tiles of that matrix, and after its output
-//     stores have landed it adds one to that counter.  A matrix's phases then
-//     follow each other closely on whichever clusters are free, without a
-//     launch boundary, and its operands are still in L2 when they are read.
+//   kChain = true: one launch for every phase of every iteration.  Each
+//     cluster runs its own list of work items (any phase, any matrix; the host
+//     orders the lists so that items are ready in time); before reading a
+//     matrix's Gram, polynomial or iterate it waits (bounded) for the counter
+//     of completed tiles of that matrix, and after its output stores have
+//     landed it adds one to that counter.  A matrix's phases then follow each
+//     other closely on whichever clusters are free, without a launch
+//     boundary, its operands are still in L2 when they are read, and the
+//     weight update of one matrix overlaps the products of others.
 template <int kMode, bool kFinal, bool kChain>
 __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ GemmArgs p) {
-  static_assert(!(kChain && kFinal), "the chained launch never runs the final update");
+  static_assert(!(kChain && kFinal), "the chained launch takes the final update from its items");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
@@ -434,16 +431,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();             // 0: issues the MMAs of the pair
   const int cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
-  constexpr bool final_w = !kChain && kMode == kModeUpdate && kFinal;
-  // Slice buffers: every phase but the final update uses all four 16 KB buffers
-  // for its output slices (the polynomial phase loads its A input into them
-  // first), with two output stores in flight.  The final update stores no bf16
-  // output and reads no input: its two slice buffers carry no data, and all
-  // four buffers serve as its fp32 staging ring for the weight update.
-  constexpr int nbuf = kFinal ? 2 : 4;
+  // The ring of four 16 KB chunk buffers: running chunk q uses buffer q % 4.
   auto slice_buf = [&](int b) { return b < 2 ? dbuf + b * kSliceBytes : mbuf + (b - 2) * kSliceBytes; };
-  // fp32 staging buffers of the final update
-  auto stg_buf = [&](int i) { return i < 2 ? mbuf + i * kSliceBytes : dbuf + (i - 2) * kSliceBytes; };
 
   // This cluster's tiles, in processing order.
   const int item0 = kChain ? p.item_off[cid] : 0;
@@ -453,11 +442,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     Tile T;
     if constexpr (kChain) {
       const WorkItem w = p.items[item0 + i];
-      T.mode = w.mode; T.cls = w.cls; T.b = w.b; T.tm = w.tm; T.tn = w.tn;
+      T.fin = w.mode == kModeFinal;
+      T.mode = T.fin ? kModeUpdate : w.mode; T.cls = w.cls; T.b = w.b; T.tm = w.tm; T.tn = w.tn;
       T.x_in = w.it & 1; T.first = w.it == 0; T.mat = w.mat; T.need = w.need;
     } else {
       const TileCoord tc = decode_tile(p, cid + i * ncl, kMode != kModeUpdate);
-      T.mode = kMode; T.cls = tc.cls; T.b = tc.b; T.tm = tc.tm; T.tn = tc.tn;
+      T.mode = kMode; T.fin = kFinal; T.cls = tc.cls; T.b = tc.b; T.tm = tc.tm; T.tn = tc.tn;
       T.x_in = p.x_in; T.first = p.first; T.mat = p.cls[tc.cls].mat_first + tc.b; T.need = 0;
     }
     return T;
@@ -468,10 +458,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl->tmem_full[s], 1);
       mbar_init(&ctl->tmem_empty[s], 8);
-    }
-    for (int s = 0; s < kStgBufs; ++s) {
-      mbar_init(&ctl->stg_full[s], 4);
-      mbar_init(&ctl->stg_free[s], 1);
     }
     for (int s = 0; s < 4; ++s) {
       mbar_init(&ctl->in_full[s], 1);
@@ -494,7 +480,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   // set-up above overlaps the previous launch; its outputs are read only below
   griddep_launch_dependents();
   griddep_wait();
-  const int my_slices = 4 * my_tiles;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -620,158 +605,117 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     if (lane == 0) {
       for (int c = 0; c < p.nclasses; ++c)
         for (int k = 0; k < kTmapsPerClass; ++k) tmap_acquire(&p.tmaps[p.cls[c].tmap_base + k]);
-      if (final_w)
+      if (p.final_apply)
         for (int c = 0; c < p.nclasses; ++c)
           for (int b = 0; b < p.cls[c].batch; ++b)
             if (p.out[p.cls[c].mat_first + b].tma) tmap_acquire(&p.wmaps[p.cls[c].mat_first + b]);
       int pend[4] = {-1, -1, -1, -1};              // parity of an input load not yet seen landed
-      // Make slice gs's buffer set ready: load its input slice (polynomial
-      // phase: the A block the epilogue adds), or just hand it over.
-      auto prepare = [&](int gs, const Tile& T) {
-        const int b = gs % nbuf;
-        if (T.mode == kModePoly) {
-          const GemmClass& C = p.cls[T.cls];
-          mbar_arrive_expect_tx(&ctl->in_full[b], kSliceBytes);
-          tma_load_3d(slice_buf(b), &p.tmaps[C.tmap_base + kTmA], &ctl->in_full[b], T.tn * kTile + 64 * (gs & 3),
-                      T.tm * kTile + (int)rank * kBM, T.b);
-          pend[b] = (gs / nbuf) & 1;
-        } else {
-          mbar_arrive(&ctl->in_full[b]);
-        }
-      };
-      auto output_map = [&](const Tile& T) {
-        const GemmClass& C = p.cls[T.cls];
-        if (T.mode == kModeGram) return &p.tmaps[C.tmap_base + kTmA];
-        if (T.mode == kModePoly) return &p.tmaps[C.tmap_base + kTmB];
-        return &p.tmaps[C.tmap_base + (T.x_in ? kTmX0 : kTmX1)];
-      };
       bool ok = true;
-      if constexpr (kChain) {
-        // Slices of tile i use buffers 0..3 in order.  A tile's completion is
-        // published (its stores landed, then the counter) before the DMA waits
-        // for anything a later tile needs, so a cluster never waits on itself.
-        if (my_tiles > 0) {
-          const Tile T0 = tile_of(0);
-          if (T0.mode == kModePoly && T0.need > 0) {
-            ok = wait_count(&p.done[T0.mat], (uint32_t)T0.need, wc, kDevTimeoutDep);
-            fence_proxy_async_global();
-          }
-          if (ok)
-            for (int h = 0; h < 4; ++h) prepare(h, T0);
-        }
-        for (int i = 0; i < my_tiles && ok; ++i) {
-          const Tile T = tile_of(i);
-          const GemmClass& C = p.cls[T.cls];
-          const bool has_next = i + 1 < my_tiles;
-          const Tile N = tile_of(has_next ? i + 1 : i);
-          const bool next_in = has_next && N.mode == kModePoly;
-          const int row0 = T.tm * kTile + (int)rank * kBM;
-          const CUtensorMap* tO = output_map(T);
-          const int ocols = T.mode != kModeUpdate ? C.kp : C.lp;
-          for (int h = 0; h < 4; ++h) {
-            if (!mbar_wait(&ctl->out_full[h], (uint32_t)(i & 1), wc, kDevTimeoutEpi)) { ok = false; break; }
-            pend[h] = -1;                          // the math warps saw this slice's input land
-            const int x0 = T.tn * kTile + 64 * h;
-            if (row0 < C.kp && x0 < ocols) tma_store_3d(tO, slice_buf(h), x0, row0, T.b);
-            tma_store_commit();
-            if (h >= 1 && has_next && !next_in) {
-              tma_store_wait_read1();              // slice h-1's buffer has been read
-              prepare(4 * (i + 1) + h - 1, N);     // no input to load: hand it over now
+      // Arming chunk q hands buffer q % 4 to the math warps: with the A block
+      // the polynomial epilogue adds loaded into it, or empty.  In the chained
+      // launch a polynomial tile's chunks are armed only once the DMA has
+      // reached that tile, after every earlier tile published its results, so
+      // waiting there for the tile's inputs never waits on this cluster.
+      int ia = 0, ha = 0, armed = 0;               // next chunk to arm: chunk ha of tile ia
+      Tile TA{};
+      if (my_tiles > 0) TA = tile_of(0);
+      auto deferred = [&](int drain_tile) { return kChain && ia < my_tiles && TA.mode == kModePoly && ia != drain_tile; };
+      auto arm_until = [&](int limit, int drain_tile) {
+        while (ok && armed < limit && ia < my_tiles && !deferred(drain_tile)) {
+          const int b = armed & 3;
+          if (TA.mode == kModePoly) {
+            if (kChain && ha == 0 && TA.need > 0) {
+              ok = wait_count(&p.done[TA.mat], (uint32_t)TA.need, wc, kDevTimeoutDep);
+              fence_proxy_async_global();
+              if (!ok) return;
             }
+            const GemmClass& C = p.cls[TA.cls];
+            mbar_arrive_expect_tx(&ctl->in_full[b], kSliceBytes);
+            tma_load_3d(slice_buf(b), &p.tmaps[C.tmap_base + kTmA], &ctl->in_full[b], TA.tn * kTile + 64 * ha,
+                        TA.tm * kTile + (int)rank * kBM, TA.b);
+            pend[b] = (armed >> 2) & 1;
+          } else {
+            mbar_arrive(&ctl->in_full[b]);
           }
-          if (!ok) break;
-          tma_store_wait_all0();                   // this tile's output has landed in memory
-          fence_proxy_async_global();
-          red_release_gpu_add(&p.done[T.mat], 1u);
-          if (has_next) {
-            if (next_in) {
-              if (N.need > 0) {
-                if (!wait_count(&p.done[N.mat], (uint32_t)N.need, wc, kDevTimeoutDep)) { ok = false; break; }
-                fence_proxy_async_global();
-              }
-              for (int h = 0; h < 4; ++h) prepare(4 * (i + 1) + h, N);
-            } else {
-              prepare(4 * (i + 1) + 3, N);
-            }
+          ++armed;
+          if (++ha == (TA.fin ? 8 : 4)) {
+            ha = 0;
+            if (++ia < my_tiles) TA = tile_of(ia);
           }
         }
-      } else {
-        for (int g0 = 0; g0 < nbuf && g0 < my_slices; ++g0) prepare(g0, tile_of(g0 >> 2));
-        int gc = 0;                                // fp32 chunk counter (final update)
-        int stg_freed = 0;                         // chunks whose staging buffer was handed back
-        auto release_stg = [&](int upto) {         // hand back the buffers of chunks < upto, in order
-          for (; stg_freed < upto; ++stg_freed) mbar_arrive(&ctl->stg_free[stg_freed % kStgBufs]);
-        };
-        for (int gs = 0; gs < my_slices && ok; ++gs) {
-          const int b = gs % nbuf;
-          const uint32_t ph = (uint32_t)((gs / nbuf) & 1);
-          const int h = gs & 3;
-          const Tile T = tile_of(gs >> 2);
-          const GemmClass& C = p.cls[T.cls];
-          const int row0 = T.tm * kTile + (int)rank * kBM;
-          if (final_w) {
+      };
+      arm_until(4, 0);
+      int q = 0;                                   // next chunk to drain
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const Tile T = tile_of(i);
+        const GemmClass& C = p.cls[T.cls];
+        const int row0 = T.tm * kTile + (int)rank * kBM;
+        const int nch = T.fin ? 8 : 4;
+        const CUtensorMap* tO = T.mode == kModeGram ? &p.tmaps[C.tmap_base + kTmA]
+                              : T.mode == kModePoly ? &p.tmaps[C.tmap_base + kTmB]
+                                                    : &p.tmaps[C.tmap_base + (T.x_in ? kTmX0 : kTmX1)];
+        for (int h = 0; h < nch; ++h, ++q) {
+          const int b = q & 3;
+          if (!mbar_wait(&ctl->out_full[b], (uint32_t)((q >> 2) & 1), wc, kDevTimeoutEpi)) { ok = false; break; }
+          pend[b] = -1;                            // the math warps saw this chunk's input land
+          const uint8_t* S = slice_buf(b);
+          if (T.fin) {
+            // -lr*O chunk: columns gj0..gj0+31 of X rows row0..row0+127
             const OutMat& O = p.out[T.mat];
-            for (int sub = 0; sub < 2 && ok; ++sub, ++gc) {
-              const int s = gc % kStgBufs;
-              if (!mbar_wait(&ctl->stg_full[s], (uint32_t)((gc / kStgBufs) & 1), wc, kDevTimeoutEpi)) { ok = false; break; }
-              if (O.tma) {
-                const uint8_t* S = stg_buf(s);
-                const CUtensorMap* wm = &p.wmaps[T.mat];
-                const int gj0 = T.tn * kTile + 64 * h + 32 * sub;
-                if (!O.trans) {
-                  if (row0 < O.m && gj0 < O.n) {
-                    if (p.assign) tma_store_2d(wm, S, gj0, row0); else tma_reduce_add_2d(wm, S, gj0, row0);
-                  }
-                } else if (gj0 < O.m) {
-                  for (int hq = 0; hq < 4; ++hq) {
-                    if (row0 + 32 * hq >= O.n) continue;
-                    if (p.assign) tma_store_2d(wm, S + hq * 4096, row0 + 32 * hq, gj0);
-                    else tma_reduce_add_2d(wm, S + hq * 4096, row0 + 32 * hq, gj0);
-                  }
+            if (O.tma) {
+              const CUtensorMap* wm = &p.wmaps[T.mat];
+              const int gj0 = T.tn * kTile + 64 * (h >> 1) + 32 * (h & 1);
+              if (!O.trans) {
+                if (row0 < O.m && gj0 < O.n) {
+                  if (p.assign) tma_store_2d(wm, S, gj0, row0); else tma_reduce_add_2d(wm, S, gj0, row0);
                 }
-                tma_store_commit();                  // one bulk group per chunk
-                tma_store_wait_read<kStgLag>();      // chunks up to gc - kStgLag have been read
-                release_stg(gc + 1 - kStgLag);
-              } else {
-                tma_store_wait_read0();
-                release_stg(gc + 1);
+              } else if (gj0 < O.m) {
+                for (int hq = 0; hq < 4; ++hq) {
+                  if (row0 + 32 * hq >= O.n) continue;
+                  if (p.assign) tma_store_2d(wm, S + hq * 4096, row0 + 32 * hq, gj0);
+                  else tma_reduce_add_2d(wm, S + hq * 4096, row0 + 32 * hq, gj0);
+                }
               }
-            }
-            if (!ok) break;
-          }
-          if (!mbar_wait(&ctl->out_full[b], ph, wc, kDevTimeoutEpi)) { ok = false; break; }
-          pend[b] = -1;                              // the math warps saw this slice's input land
-          if (!final_w) {
+            }                                      // (rows not 16-byte aligned: the math warps wrote W)
+          } else {
             // stores start inside the tensor only (a pair tile can overhang the
             // 128-padded edge by half; the overhang is never stored)
             const int ocols = T.mode != kModeUpdate ? C.kp : C.lp;
             const int x0 = T.tn * kTile + 64 * h;
-            if (row0 < C.kp && x0 < ocols) tma_store_3d(output_map(T), slice_buf(b), x0, row0, T.b);
-            tma_store_commit();
-            if constexpr (nbuf == 4) {
-              tma_store_wait_read1();                // the previous slice's buffer is free again
-              const int nx = gs - 1 + nbuf;          // slices 0..3 were armed before the loop
-              if (gs >= 1 && nx < my_slices) prepare(nx, tile_of(nx >> 2));
-              continue;
-            }
-            tma_store_wait_read0();                  // buffers b readable again
+            if (row0 < C.kp && x0 < ocols) tma_store_3d(tO, S, x0, row0, T.b);
           }
-          if (gs + nbuf < my_slices) prepare(gs + nbuf, tile_of((gs + nbuf) >> 2));
+          tma_store_commit();                      // one bulk group per chunk
+          if (armed < q + 4 && ia < my_tiles && !deferred(i)) {
+            tma_store_wait_read1();                // the previous chunk's buffer has been read
+            arm_until(q + 4, i);
+          }
         }
-        tma_store_wait_all0();
-        release_stg(gc);
+        if (!ok) break;
+        if (kChain && !T.fin) {
+          tma_store_wait_all0();                   // this tile's output has landed in memory
+          fence_proxy_async_global();
+          red_release_gpu_add(&p.done[T.mat], 1u);
+        }
+        if (armed < q + 3 && ia < my_tiles) {      // chunks held back until this tile was published
+          tma_store_wait_all0();
+          arm_until(q + 4, i + 1);
+        }
       }
       tma_store_wait_all0();
-      for (int b = 0; b < nbuf; ++b)
+      for (int b = 0; b < 4; ++b)
         if (pend[b] >= 0) mbar_wait(&ctl->in_full[b], (uint32_t)pend[b], wc, kDevTimeoutDrain);
       aborted = !ok;
     }
   } else {
     // ---------------------------------------------------- epilogue math
-    const int q = warp & 3;                       // TMEM lane quarter this warp may access
-    const int r = q * 32 + lane;                  // tile row owned by this thread
-    int gs = 0, gc = 0;
+    const int q4 = warp & 3;                      // TMEM lane quarter this warp may access
+    const int r = q4 * 32 + lane;                 // tile row owned by this thread
+    int q = 0;                                    // running chunk
     bool ok = true;
+    // waits until chunk q's buffer is handed over (and its input, if any, landed)
+    auto take = [&]() {
+      return __all_sync(0xffffffffu, mbar_wait(&ctl->in_full[q & 3], (uint32_t)((q >> 2) & 1), wc, kDevTimeoutEpi));
+    };
     for (int it = 0; it < my_tiles && ok; ++it) {
       const Tile T = tile_of(it);
       const int acc = it & 1;
@@ -781,13 +725,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       tc_fence_after();
       const float s = T.first ? p.scale[T.mat] : 1.0f;
       const int row0 = T.tm * kTile + (int)rank * kBM;
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
+      const uint32_t tbase = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * kBN);
 #pragma unroll 1
-      for (int h = 0; h < 4 && ok; ++h, ++gs) {
-        const int b = gs % nbuf;
-        uint8_t* dslice = slice_buf(b);
-        ok = __all_sync(0xffffffffu, mbar_wait(&ctl->in_full[b], (uint32_t)((gs / nbuf) & 1), wc, kDevTimeoutEpi));
-        if (!ok) break;
+      for (int h = 0; h < 4 && ok; ++h) {
+        if (!T.fin && !(ok = take())) break;
         float v[64];
         tmem_ld_32x32b_x64(tbase + (uint32_t)(h * 64), v);
         if (h == 3) {                               // accumulator fully read: hand it back to the MMA
@@ -803,6 +744,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           for (int i = 0; i < 64; ++i) v[i] *= alpha;
         } else {
           // b A + c A A
+          const uint8_t* dslice = slice_buf(q & 3);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             uint4 raw = *reinterpret_cast<const uint4*>(dslice + sw128_off((uint32_t)r, (uint32_t)u));
@@ -816,7 +758,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           }
           // + a on the diagonal: on a diagonal tile, a warp's 32 rows meet the
           // slice's columns at 32 consecutive columns starting at dbase, lane by lane
-          const int dbase = (int)rank * kBM + q * 32 - 64 * h;
+          const int dbase = (int)rank * kBM + q4 * 32 - 64 * h;
           if (T.tm == T.tn && (dbase == 0 || dbase == 32)) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -826,15 +768,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             }
           }
         }
-        if (final_w) {
+        if (T.fin) {
           const OutMat& O = p.out[T.mat];
 #pragma unroll
-          for (int sub = 0; sub < 2; ++sub, ++gc) {
-            const int sidx = gc % kStgBufs;
-            ok = __all_sync(0xffffffffu, mbar_wait(&ctl->stg_free[sidx], (uint32_t)(((gc / kStgBufs) & 1) ^ 1), wc,
-                                                   kDevTimeoutEpi));
-            if (!ok) break;
-            uint8_t* S = stg_buf(sidx);
+          for (int sub = 0; sub < 2; ++sub) {
+            if (!(ok = take())) break;
+            uint8_t* S = slice_buf(q & 3);
             const float* vv = v + 32 * sub;
             if (O.tma) {
               // -lr*O (or O), 128-byte swizzled; the DMA warp adds it to W in L2
@@ -856,7 +795,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
               fence_async_shared();
             } else {
               // rows not 16-byte aligned: the math warps update W themselves,
-              // in whole 128-byte rows through the staging buffer
+              // in whole 128-byte rows through the chunk buffer
               float* Sf = reinterpret_cast<float*>(S);
               if (!O.trans) {
 #pragma unroll
@@ -868,14 +807,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
                 for (int i = 0; i < 32; ++i) Sf[i * kBM + r] = vv[i];
               }
               __syncwarp();
-              store_w_slice_warp(O, Sf, row0, T.tn * kTile + 64 * h + 32 * sub, q, lane, p.lr, p.assign);
+              store_w_slice_warp(O, Sf, row0, T.tn * kTile + 64 * h + 32 * sub, q4, lane, p.lr, p.assign);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->stg_full[sidx]);
+            if (lane == 0) mbar_arrive(&ctl->out_full[q & 3]);
+            ++q;
           }
-          if (!ok) break;
         } else {
           // bf16 output (in place over the input slice), 128-byte swizzled for the TMA store
+          uint8_t* dslice = slice_buf(q & 3);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             uint4 o;
@@ -886,9 +826,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             *reinterpret_cast<uint4*>(dslice + sw128_off((uint32_t)r, (uint32_t)u)) = o;
           }
           fence_async_shared();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->out_full[q & 3]);
+          ++q;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->out_full[b]);
       }
     }
     aborted = !ok;
@@ -969,6 +910,15 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_small_kernel(const __grid
   }
   griddep_launch_dependents();
   griddep_wait();
+  // One SM moves all of g, buf and W: start them towards L2 now (bulk
+  // prefetches, no registers held), so that the loads below and the final
+  // read-modify-write of W find them there instead of waiting on DRAM.
+  if (M.vec && warp == 1) {
+    const size_t elems = (size_t)M.m * M.n;
+    prefetch_l2_matrix(M.g, elems, lane, 32);
+    if (p.has_buf) prefetch_l2_matrix(M.buf, elems, lane, 32);
+    if (!p.assign) prefetch_l2_matrix(M.w, elems, lane, 32);
+  }
 
   // ---- momentum, norm, X0 (bf16) into shared memory; zero padding included.
   // Each thread issues all loads of a batch before any store (one CTA per SM
@@ -1342,6 +1292,15 @@ __global__ void __launch_bounds__(kPairThreads, 1) ns_pair_kernel(const __grid_c
   tc_fence_after();
   griddep_launch_dependents();
   griddep_wait();
+  // g, buf and W towards L2 now (bulk prefetches split over the two CTAs), so
+  // that the loads below and the final read-modify-write of W find them there.
+  if (M.vec && warp == 1) {
+    const size_t elems = (size_t)M.m * M.n;
+    const int t = (int)rank * 32 + lane;
+    prefetch_l2_matrix(M.g, elems, t, 64);
+    if (p.has_buf) prefetch_l2_matrix(M.buf, elems, t, 64);
+    if (!p.assign) prefetch_l2_matrix(M.w, elems, t, 64);
+  }
 
   // Stores one bf16 quad / element of X row `xr` (global), column j into XO
   // (local row) and into the XC of the CTA that owns column j's half.

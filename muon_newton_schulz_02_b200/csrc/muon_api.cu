@@ -250,9 +250,9 @@ int build_layout(const int64_t* shapes, int n, Plan& plan) {
 
 // ------------------------------------------------------ chained schedule ---
 // Host-side list scheduling of the chained launch.  Every matrix runs the
-// chain Gram(0), poly(0), update(0), Gram(1), ..., poly(n-1) (the last update
-// runs in its own launch); each phase's tiles may start only once all tiles of
-// the previous phase of that matrix are done.  A simulation of `ncl` clusters
+// chain Gram(0), poly(0), update(0), Gram(1), ..., update(n-1) (the last
+// update adds -lr*O into W); each phase's tiles may start only once all tiles
+// of the previous phase of that matrix are done.  A simulation of `ncl` clusters
 // assigns tiles greedily: a free cluster takes the next tile of the
 // highest-priority matrix whose current phase is ready (larger matrices first),
 // so a matrix's phases follow each other closely and its operands stay in L2
@@ -268,25 +268,27 @@ double chain_latency_units() {
   static double lat = -1.0;
   if (lat < 0.0) {
     const char* e = std::getenv("MUON_CHAIN_LATENCY");
-    lat = e ? std::max(0.0, std::atof(e)) : 12.0;
+    lat = e ? std::max(0.0, std::atof(e)) : 20.0;
   }
   return lat;
 }
 
 void build_chain(const Group& g, int ns_steps, int ncl, std::vector<WorkItem>& items, std::vector<int>& off) {
   constexpr double kOverhead = 2.0;
+  constexpr double kFinalCost = 1.5;          // the last update also reads and writes W
   const double lat = chain_latency_units();
   const int nm = (int)g.mats.size();
-  const int nphases = 3 * ns_steps - 1;
+  const int nphases = 3 * ns_steps;
   struct MatState {
     int cls = 0, b = 0, T = 0, Tn = 0;
-    int ntiles[3] = {0, 0, 0};
-    double cost[3] = {0, 0, 0};
+    int ntiles[4] = {0, 0, 0, 0};
+    double cost[4] = {0, 0, 0, 0};
     int phase = 0, next = 0;
     int need = 0;              // tile halves completed before the current phase
     double vis = 0.0;          // latest visibility time among the current phase's tiles
     double total = 0.0;
   };
+  auto mode_of = [&](int j) { return j == nphases - 1 ? (int)kModeFinal : j % 3; };
   std::vector<MatState> ms(nm);
   for (size_t ci = 0; ci < g.classes.size(); ++ci) {
     const ClassDesc& cd = g.classes[ci];
@@ -297,10 +299,11 @@ void build_chain(const Group& g, int ns_steps, int ncl, std::vector<WorkItem>& i
       st.T = (cd.kp + kTile - 1) / kTile;
       st.Tn = (cd.lp + kTile - 1) / kTile;
       st.ntiles[kModeGram] = st.ntiles[kModePoly] = st.T * (st.T + 1) / 2;
-      st.ntiles[kModeUpdate] = st.T * st.Tn;
+      st.ntiles[kModeUpdate] = st.ntiles[kModeFinal] = st.T * st.Tn;
       st.cost[kModeGram] = cd.lp / kBK + kOverhead;
       st.cost[kModePoly] = st.cost[kModeUpdate] = cd.kp / kBK + kOverhead;
-      for (int j = 0; j < nphases; ++j) st.total += st.ntiles[j % 3] * st.cost[j % 3];
+      st.cost[kModeFinal] = kFinalCost * st.cost[kModeUpdate];
+      for (int j = 0; j < nphases; ++j) st.total += st.ntiles[mode_of(j)] * st.cost[mode_of(j)];
     }
   }
   // priority: more total work first (its long chain starts early), then group order
@@ -319,7 +322,7 @@ void build_chain(const Group& g, int ns_steps, int ncl, std::vector<WorkItem>& i
     if (nphases > 0) avail.insert(prio[m]);
   long long left = 0;
   for (int m = 0; m < nm; ++m)
-    for (int j = 0; j < nphases; ++j) left += ms[m].ntiles[j % 3];
+    for (int j = 0; j < nphases; ++j) left += ms[m].ntiles[mode_of(j)];
   while (left > 0) {
     auto [t, c] = free_at.top();
     free_at.pop();
@@ -336,9 +339,9 @@ void build_chain(const Group& g, int ns_steps, int ncl, std::vector<WorkItem>& i
     }
     const int m = by_prio[*avail.begin()];
     MatState& st = ms[m];
-    const int mode = st.phase % 3;
+    const int mode = mode_of(st.phase);
     int tm, tn;
-    if (mode == kModeUpdate) {
+    if (mode == kModeUpdate || mode == kModeFinal) {
       tm = st.next / st.Tn;
       tn = st.next % st.Tn;
     } else {                                  // upper-triangle 256-blocks, row by row
@@ -708,6 +711,8 @@ int update_wmaps(Ctx& c, Plan& plan, size_t gi, const StepIO& io) {
   return MUON_OK;
 }
 
+constexpr int kChainMaxK = 1024;       // largest padded short side the chained launch takes
+
 // The chained launch's work lists for group gidx and ns_steps iterations,
 // built and uploaded on first use (a synchronous copy: make the first call for
 // a set of shapes and an iteration count outside stream capture).
@@ -743,9 +748,13 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
   const CUtensorMap* tmaps = (const CUtensorMap*)((char*)plan.tmaps + g.off_tmaps);
   const int nm = (int)g.mats.size();
   unsigned* done = (unsigned*)(base + g.off_done);
-  // every phase but the last update in one chained launch, unless the device
-  // cannot hold its clusters or a test asks for one launch per phase
-  const bool chain = io.ns_steps >= 1 && g_chain_clusters[c.dev] > 0 && !(g_debug_flags & 4);
+  // every phase in one chained launch, unless the device cannot hold its
+  // clusters, a test asks for one launch per phase, or the matrices are so
+  // large that one phase of one matrix already fills the GPU (short side above
+  // kChainMaxK): there the phases gain little from overlapping, and keeping
+  // several such matrices in flight costs more L2 misses than it saves.
+  bool chain = io.ns_steps >= 1 && g_chain_clusters[c.dev] > 0 && !(g_debug_flags & 4);
+  for (const auto& cd : g.classes) chain = chain && cd.kp <= kChainMaxK;
 
   // 1. prologue
   {
@@ -836,20 +845,8 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
     ga->done = done;
     ga->debug_flags = 0;
     if (g_debug_flags & 1) { ga->debug_flags = 1; g_debug_flags &= ~1; }
-    rc = launch(c, MUON_KIND_CHAIN, [&] { launch_gemm(c.stream, *ga, c.sm_count, ct->nclusters); });
-    if (rc) return rc;
-    // the last update, with W -= lr*O fused, in its own launch
-    for (size_t ci = 0; ci < g.upd_cls.size(); ++ci) ga->cls[ci] = g.upd_cls[ci];
-    ga->items = nullptr;
-    ga->item_off = nullptr;
-    ga->done = nullptr;
-    ga->total_tiles = g.upd_tiles;
-    ga->mode = kModeUpdate;
-    ga->x_in = (io.ns_steps - 1) & 1;
-    ga->first = io.ns_steps == 1;
-    ga->final_apply = 1;
-    ga->debug_flags = 0;
-    return launch(c, MUON_KIND_UPDATE_APPLY, [&] { launch_gemm(c.stream, *ga, c.sm_count); });
+    ga->final_apply = 1;                     // its items include the last update (W -= lr*O)
+    return launch(c, MUON_KIND_CHAIN, [&] { launch_gemm(c.stream, *ga, c.sm_count, ct->nclusters); });
   }
 
   for (int it = 0; it < io.ns_steps; ++it) {
@@ -1186,6 +1183,16 @@ int muon_profile_read(double* ms, int64_t* launches, int nkinds) {
 }
 
 int64_t muon_launch_count(void) { return g_launches.load(); }
+
+int muon_chain_clusters(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || device_setup(dev) != MUON_OK) {
+    cudaGetLastError();
+    return -1;
+  }
+  return g_chain_clusters[dev];
+}
 
 int muon_chain_plan(const int64_t* shapes, int n, int ns_steps, int nclusters, int32_t* items, int64_t capacity,
                     int32_t* cluster_off, int64_t* nitems) {

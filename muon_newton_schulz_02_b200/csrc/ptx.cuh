@@ -233,6 +233,22 @@ __device__ __forceinline__ void tmap_acquire(const void* tmap) {
                : "memory");
 }
 
+// Prefetch [p, p + bytes) from global memory into L2 (no data comes to the SM;
+// p and bytes multiples of 16).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+// Prefetch a whole contiguous fp32 matrix into L2 in 32 KB pieces, the pieces
+// spread over the threads of the calling group (first thread t, stride n).
+__device__ __forceinline__ void prefetch_l2_matrix(const float* p, size_t elems, int t, int n) {
+  const size_t bytes = (elems * 4) & ~size_t(15);
+  for (size_t off = (size_t)t * 32768; off < bytes; off += (size_t)n * 32768) {
+    const size_t len = bytes - off < 32768 ? bytes - off : 32768;
+    prefetch_l2_bulk(reinterpret_cast<const char*>(p) + off, (uint32_t)len);
+  }
+}
+
 // 3-D tiled load global -> shared, completion counted on an mbarrier.
 // x (innermost) must be a multiple of 8 elements for bf16 (16 bytes).
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, uint64_t* bar, int x, int y, int z) {

@@ -1,5 +1,5 @@
 """The chained launch's work lists, checked on the host (no GPU): every tile of
-every phase but the last update appears exactly once, each item's `need`
+every phase appears exactly once, each item's `need`
 counts exactly the tile halves of the earlier phases of its matrix, and the
 lists cannot deadlock -- with every cluster running its list in order and an
 item starting only once its matrix's counter reaches `need`, all items finish
@@ -48,11 +48,13 @@ def test_lists_cover_every_tile_once_and_cannot_deadlock(name, ns_steps, ncluste
             continue
         sym, upd = _tiles(min(r, c), max(r, c))
         before = 0
-        for j in range(3 * ns_steps - 1):
+        for j in range(3 * ns_steps):
             it, mode = divmod(j, 3)
-            for t in (upd if mode == 2 else sym):
+            if j == 3 * ns_steps - 1:
+                mode = 3                                   # the last update, with W -= lr*O
+            for t in (upd if mode >= 2 else sym):
                 expect[(m, it, mode) + t] = before
-            before += 2 * len(upd if mode == 2 else sym)
+            before += 2 * len(upd if mode >= 2 else sym)
     seen = {}
     for need, m, cls, b, tm, tn, mode, it in items:
         key = (m, it, mode, tm, tn)

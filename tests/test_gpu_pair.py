@@ -100,7 +100,7 @@ def test_pair_mixed_with_small_and_gemm_paths_in_one_call():
     W_new, b_new = gpu_step(W, g, b, 0.02, 0.95)
     muon.profile_enable(False)
     prof = muon.profile_read()
-    assert prof["pair"][1] == 1 and prof["small"][1] == 1 and prof["gram"][1] == 5
+    assert prof["pair"][1] == 1 and prof["small"][1] == 1 and prof["chain"][1] == 1
     _check(W, g, b, W_new, b_new, band=False)
 
 

@@ -240,7 +240,7 @@ def test_chained_launch_matches_one_launch_per_phase_bitwise(ns_steps):
     # The chained launch computes every tile exactly as the per-phase launches
     # do (same operands, same K order, same epilogue); only the order in which
     # tiles run differs.  So both give bitwise the same weights and buffers.
-    shapes = [(768, 768)] * 3 + [(768, 3072), (3072, 768), (640, 1920), (1000, 300), (384, 384), (1600, 1600)]
+    shapes = [(768, 768)] * 3 + [(768, 3072), (3072, 768), (640, 1920), (1000, 300), (384, 384), (1024, 1280)]
     W, g, b = _inputs(shapes, 41, gscale=0.02)
     muon.profile_enable(True)
     try:
@@ -258,3 +258,18 @@ def test_chained_launch_matches_one_launch_per_phase_bitwise(ns_steps):
     for x, y in zip(r_chain[0] + r_chain[1], r_phase[0] + r_phase[1]):
         assert np.array_equal(x, y)
     _check_step(W, g, b, r_chain[0], r_chain[1], steps=ns_steps)
+
+
+def test_large_short_sides_take_one_launch_per_phase():
+    # short side above 1024: one launch per phase, still within the parity bar
+    shapes = [(1600, 1600), (1100, 2000)]
+    W, g, b = _inputs(shapes, 43, gscale=0.02)
+    muon.profile_enable(True)
+    try:
+        muon.profile_read()
+        W_new, b_new = gpu_step(W, g, b, 0.02, 0.95)
+        kinds = muon.profile_read()
+    finally:
+        muon.profile_enable(False)
+    assert kinds["chain"][1] == 0 and kinds["gram"][1] == 5 and kinds["update_apply"][1] == 1
+    _check_step(W, g, b, W_new, b_new)
