@@ -859,7 +859,9 @@ constexpr int kSmallThreads = 128;
 constexpr int kSmallMaxK = 128;
 constexpr int kSmallMaxL = 512;
 constexpr uint32_t kSmallChunk = 128 * 64 * 2;                       // 16 KB
-constexpr uint32_t kSmallSmem = (kSmallMaxL / 64 + 2 + 2) * kSmallChunk + 256 + 1024;
+// X (8 chunks), A and B (2 each), a 32 KB staging area (with A and B the
+// three 32 KB slots of the prologue's bulk-copy ring), control words
+constexpr uint32_t kSmallSmem = (kSmallMaxL / 64 + 2 + 2 + 2) * kSmallChunk + 256 + 1024;
 
 struct SmallMat {
   const float* g;
@@ -889,18 +891,20 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_small_kernel(const __grid
   uint8_t* Xs = smem;                                        // 8 chunks
   uint8_t* As = Xs + (kSmallMaxL / 64) * kSmallChunk;        // 2 chunks
   uint8_t* Bs = As + 2 * kSmallChunk;                        // 2 chunks
-  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(Bs + 2 * kSmallChunk);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
+  uint8_t* Ss = Bs + 2 * kSmallChunk;                        // 2 chunks of staging
+  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(Ss + 2 * kSmallChunk);
+  uint64_t* pro_bar = mma_bar + 1;                           // 3: prologue ring slots
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pro_bar + 3);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(abort_flag + 1);     // 4 warp partials
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const SmallMat& M = p.mats[blockIdx.x];
-  const int lp = M.lp, k = M.trans ? M.n : M.m;
-  (void)k;
+  const int lp = M.lp;
 
   if (tid == 0) {
     mbar_init(mma_bar, 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&pro_bar[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -910,22 +914,88 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_small_kernel(const __grid
   }
   griddep_launch_dependents();
   griddep_wait();
-  // One SM moves all of g, buf and W: start them towards L2 now (bulk
-  // prefetches, no registers held), so that the loads below and the final
-  // read-modify-write of W find them there instead of waiting on DRAM.
-  if (M.vec && warp == 1) {
-    const size_t elems = (size_t)M.m * M.n;
-    prefetch_l2_matrix(M.g, elems, lane, 32);
-    if (p.has_buf) prefetch_l2_matrix(M.buf, elems, lane, 32);
-    if (!p.assign) prefetch_l2_matrix(M.w, elems, lane, 32);
-  }
+  WaitCtx wc{abort_flag, p.status, p.wait_limit_ns, 0u};
 
   // ---- momentum, norm, X0 (bf16) into shared memory; zero padding included.
-  // Each thread issues all loads of a batch before any store (one CTA per SM
-  // has few warps to hide memory latency with).
   const float* __restrict__ gp = M.g;
   float* __restrict__ bp = M.buf;
   float ss = 0.f;
+  bool ok = true;
+  if (M.vec) {
+    // One SM moves all of g and buf: they stream through shared memory by 1-D
+    // bulk copies (no registers held, many bytes in flight) in pieces of whole
+    // rows of at most 16 KB each, through three (g, buf) slots in A | B | S,
+    // two pieces in flight ahead of the one being processed; the new buffer
+    // goes back by bulk store from the same slot.
+    const int kx = M.trans ? M.n : M.m, lx = M.trans ? M.m : M.n;   // X is kx x lx
+    // zero the padding of X first (rows >= kx, columns >= lx)
+    for (int u = tid; u < kSmallMaxK * (lp / 8); u += kSmallThreads) {
+      const int r = u / (lp / 8), c0 = 8 * (u % (lp / 8));
+      if (r >= kx || c0 + 8 > lx) *reinterpret_cast<uint4*>(Xs + chunk_off((uint32_t)r, (uint32_t)c0)) = make_uint4(0, 0, 0, 0);
+    }
+    uint8_t* slots = As;
+    const int rows_per = max(1, min(M.m, 4096 / M.n));
+    const int npieces = (M.m + rows_per - 1) / rows_per;
+    auto issue = [&](int pc) {
+      const int sl = pc % 3;
+      const uint32_t bytes = (uint32_t)(min(rows_per, M.m - pc * rows_per) * M.n * 4);
+      const size_t off = (size_t)pc * rows_per * M.n;
+      mbar_arrive_expect_tx(&pro_bar[sl], p.has_buf ? 2 * bytes : bytes);
+      bulk_load(slots + sl * 32768, gp + off, bytes, &pro_bar[sl]);
+      if (p.has_buf) bulk_load(slots + sl * 32768 + 16384, bp + off, bytes, &pro_bar[sl]);
+    };
+    if (tid == 0) {
+      issue(0);
+      if (npieces > 1) issue(1);
+    }
+    __syncthreads();                                         // padding zeroed before X is written
+    for (int pc = 0; pc < npieces; ++pc) {
+      const int sl = pc % 3;
+      ok = __syncthreads_and(ok && mbar_wait(&pro_bar[sl], (uint32_t)((pc / 3) & 1), wc, kDevTimeoutFull)) != 0;
+      if (!ok) break;
+      float* sg = reinterpret_cast<float*>(slots + sl * 32768);
+      float* sb = reinterpret_cast<float*>(slots + sl * 32768 + 16384);
+      const int row0 = pc * rows_per;
+      const int nel = min(rows_per, M.m - row0) * M.n;
+      for (int e = tid * 4; e < nel; e += kSmallThreads * 4) {
+        const float4 g4 = *reinterpret_cast<const float4*>(sg + e);
+        float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (p.has_buf) b4 = *reinterpret_cast<const float4*>(sb + e);
+        float gv[4] = {g4.x, g4.y, g4.z, g4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w}, G[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          G[q] = nesterov_g(gv[q], bv[q], p.mu, p.nesterov, p.has_buf);
+          ss = fmaf(G[q], G[q], ss);
+        }
+        if (p.has_buf) *reinterpret_cast<float4*>(sb + e) = make_float4(bv[0], bv[1], bv[2], bv[3]);
+        const int i = row0 + e / M.n, j = e % M.n;           // G row i, columns j..j+3
+        if (!M.trans) {
+          *reinterpret_cast<uint2*>(Xs + chunk_off((uint32_t)i, (uint32_t)j)) =
+              make_uint2(pack_bf16x2(G[0], G[1]), pack_bf16x2(G[2], G[3]));
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<__nv_bfloat16*>(Xs + chunk_off((uint32_t)(j + q), (uint32_t)i)) =
+                __float2bfloat16_rn(G[q]);
+        }
+      }
+      if (p.has_buf) fence_async_shared();                   // the new buffer values -> the bulk store
+      __syncthreads();
+      if (tid == 0) {
+        if (p.has_buf) {
+          bulk_store(bp + (size_t)row0 * M.n, sb, (uint32_t)(nel * 4));
+          tma_store_commit();
+        }
+        if (pc + 2 < npieces) {
+          tma_store_wait_read1();                            // slot (pc + 2) % 3 was stored from last time
+          issue(pc + 2);
+        }
+      }
+    }
+    if (tid == 0) tma_store_wait_all0();                     // buf written; slots free for A and B
+  } else {
+  // Rows not 16-byte aligned: plain loads.  Each thread issues all loads of a
+  // batch before any store (one CTA per SM has few warps to hide latency with).
   auto load4 = [&](size_t off, int col, int ncols, float (&gv)[4], float (&bv)[4]) {
     if (M.vec && col + 3 < ncols) {
       const float4 g4 = __ldg(reinterpret_cast<const float4*>(gp + off));
@@ -1018,6 +1088,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_small_kernel(const __grid
       }
     }
   }
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   if (lane == 0) red[warp] = ss;
@@ -1029,8 +1100,6 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_small_kernel(const __grid
   const uint32_t tmem = *tmem_slot;
   const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's 32 lanes
   const int r = warp * 32 + lane;                            // row of X / A / B owned by this thread
-  WaitCtx wc{abort_flag, p.status, p.wait_limit_ns, 0u};
-  bool ok = true;
   uint32_t phase = 0;
 
   auto wait_mma = [&]() {
@@ -1227,6 +1296,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) ns_small_kernel(const __grid
       apply_chunk(cc, v);
     }
   }
+  tma_store_wait_all0();                                     // this thread's bulk copies are done
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -1292,16 +1362,6 @@ __global__ void __launch_bounds__(kPairThreads, 1) ns_pair_kernel(const __grid_c
   tc_fence_after();
   griddep_launch_dependents();
   griddep_wait();
-  // g, buf and W towards L2 now (bulk prefetches split over the two CTAs), so
-  // that the loads below and the final read-modify-write of W find them there.
-  if (M.vec && warp == 1) {
-    const size_t elems = (size_t)M.m * M.n;
-    const int t = (int)rank * 32 + lane;
-    prefetch_l2_matrix(M.g, elems, t, 64);
-    if (p.has_buf) prefetch_l2_matrix(M.buf, elems, t, 64);
-    if (!p.assign) prefetch_l2_matrix(M.w, elems, t, 64);
-  }
-
   // Stores one bf16 quad / element of X row `xr` (global), column j into XO
   // (local row) and into the XC of the CTA that owns column j's half.
   auto put_quad = [&](int xr, int j, uint32_t lo, uint32_t hi) {

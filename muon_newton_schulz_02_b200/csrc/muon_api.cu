@@ -577,6 +577,8 @@ int ensure_workspace(Ctx& c, size_t bytes) {
   return MUON_OK;
 }
 
+constexpr size_t kMaxPlans = 48;
+
 int get_plan(Ctx& c, const int64_t* shapes, int n, Plan** out) {
   for (auto it = c.plans.begin(); it != c.plans.end(); ++it) {
     Plan& p = **it;
@@ -619,9 +621,12 @@ int get_plan(Ctx& c, const int64_t* shapes, int n, Plan** out) {
   }
   CUDA_TRY(cudaEventCreateWithFlags(&p->wmap_copied, cudaEventDisableTiming));
   c.plans.push_front(std::move(p));
-  if (c.plans.size() > 16) {
+  // Keep the most recent kMaxPlans plans: enough for the chunks of the
+  // host-buffer entry point (up to 16 shape lists) next to the device-buffer
+  // calls of the same loop, so that no steady-state call rebuilds a plan.
+  if (c.plans.size() > kMaxPlans) {
     CUDA_TRY(cudaStreamSynchronize(c.stream));
-    while (c.plans.size() > 16) c.plans.pop_back();
+    while (c.plans.size() > kMaxPlans) c.plans.pop_back();
   }
   *out = c.plans.front().get();
   return MUON_OK;
@@ -1063,7 +1068,7 @@ int muon_step_host(float* const* params, const float* const* grads, float* const
   }
   // Chunks of consecutive matrices: copies in (stream h2d), the step (caller's
   // stream) and copies out (stream d2h) of different chunks overlap.
-  const size_t chunk_bytes = std::max<size_t>(size_t(64) << 20, need / 8);
+  const size_t chunk_bytes = std::max<size_t>(size_t(32) << 20, need / 16);
   std::vector<std::pair<int, int>> chunks;
   for (int i = 0; i < n;) {
     int j = i;

@@ -233,20 +233,18 @@ __device__ __forceinline__ void tmap_acquire(const void* tmap) {
                : "memory");
 }
 
-// Prefetch [p, p + bytes) from global memory into L2 (no data comes to the SM;
-// p and bytes multiples of 16).
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+// 1-D bulk copy of `bytes` contiguous bytes global -> this CTA's shared memory,
+// completion counted on an mbarrier (addresses and size multiples of 16).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
-// Prefetch a whole contiguous fp32 matrix into L2 in 32 KB pieces, the pieces
-// spread over the threads of the calling group (first thread t, stride n).
-__device__ __forceinline__ void prefetch_l2_matrix(const float* p, size_t elems, int t, int n) {
-  const size_t bytes = (elems * 4) & ~size_t(15);
-  for (size_t off = (size_t)t * 32768; off < bytes; off += (size_t)n * 32768) {
-    const size_t len = bytes - off < 32768 ? bytes - off : 32768;
-    prefetch_l2_bulk(reinterpret_cast<const char*>(p) + off, (uint32_t)len);
-  }
+// 1-D bulk copy shared -> global, completed as a bulk group of the issuing thread.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(reinterpret_cast<uint64_t>(gdst)), "r"(smem_u32(smem_src)), "r"(bytes)
+               : "memory");
 }
 
 // 3-D tiled load global -> shared, completion counted on an mbarrier.
