@@ -64,6 +64,10 @@ def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     k = csrc / "kernels.cuh"
     k.write_text(k.read_text() + "\n// a new comment\n/* and a block\n comment */\n")
     assert bench.kernel_source_hash() == h0
+    # the fused small-matrix kernels are not part of the GEMM kernel's record
+    text = k.read_text()
+    k.write_text(text.replace(bench._FUSED_BEGIN, bench._FUSED_BEGIN + "\nconstexpr int kFusedOnly = 1;\n"))
+    assert bench.kernel_source_hash() == h0
     k.write_text(k.read_text() + "\nconstexpr int kUnused = 1;\n")
     assert bench.kernel_source_hash() != h0
 
