@@ -717,6 +717,17 @@ int update_wmaps(Ctx& c, Plan& plan, size_t gi, const StepIO& io) {
 }
 
 constexpr int kChainMaxK = 1024;       // largest padded short side the chained launch takes
+constexpr int64_t kChainMaxItems = int64_t(1) << 22;   // largest work list (64 MiB of items)
+
+// Work items of the chained launch for group g: every tile of every phase.
+int64_t chain_items(const Group& g, int ns_steps) {
+  int64_t per_iter = 0;
+  for (const auto& cd : g.classes) {
+    const int64_t T = (cd.kp + kTile - 1) / kTile, Tn = (cd.lp + kTile - 1) / kTile;
+    per_iter += (int64_t)cd.mats.size() * (T * (T + 1) + T * Tn);   // Gram + polynomial + update
+  }
+  return per_iter * ns_steps;
+}
 
 // The chained launch's work lists for group gidx and ns_steps iterations,
 // built and uploaded on first use (a synchronous copy: make the first call for
@@ -736,11 +747,15 @@ int get_chain(Ctx& c, Plan& plan, size_t gidx, int ns_steps, ChainTables** out) 
       cudaGetLastError();
       return fail(MUON_ERR_NOMEM, "work-list allocation failed");
     }
+    if (cudaMemcpy(ct.dev, items.data(), items.size() * sizeof(WorkItem), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy((char*)ct.dev + ib, off.data(), ob, cudaMemcpyHostToDevice) != cudaSuccess) {
+      const cudaError_t e = cudaGetLastError();
+      cudaFree(ct.dev);
+      return fail(MUON_ERR_CUDA, std::string("work-list upload failed: ") + cudaGetErrorString(e));
+    }
+    ct.items = (const WorkItem*)ct.dev;
+    ct.off = (const int*)((char*)ct.dev + ib);
     it = plan.chains.emplace(key, ct).first;   // owned by the plan from here on
-    CUDA_TRY(cudaMemcpy(ct.dev, items.data(), items.size() * sizeof(WorkItem), cudaMemcpyHostToDevice));
-    CUDA_TRY(cudaMemcpy((char*)ct.dev + ib, off.data(), ob, cudaMemcpyHostToDevice));
-    it->second.items = (const WorkItem*)ct.dev;
-    it->second.off = (const int*)((char*)ct.dev + ib);
   }
   *out = &it->second;
   return MUON_OK;
@@ -760,6 +775,7 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
   // several such matrices in flight costs more L2 misses than it saves.
   bool chain = io.ns_steps >= 1 && g_chain_clusters[c.dev] > 0 && !(g_debug_flags & 4);
   for (const auto& cd : g.classes) chain = chain && cd.kp <= kChainMaxK;
+  chain = chain && chain_items(g, io.ns_steps) <= kChainMaxItems;   // lists of bounded size and build time
 
   // 1. prologue
   {
