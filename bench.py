@@ -465,6 +465,23 @@ def run_ours(args):
             torch.cuda.synchronize(dev)
             cold.append(timer.times(e)[0])
         del flush
+    # ---- the reduced-precision variant (muon_step_fp8) on the same workload,
+    # timed the same way; reported beside the bf16 line, never as its value
+    fp8 = None
+    if args.fp8_iters and not sharded:
+        stepper8 = muon.PreparedStep(W, bufs, lr=w.lr, mu=w.mu, fp8_iters=args.fp8_iters)
+        for s in range(3):
+            stepper8(gsets[s % args.grad_sets], stream=stream)
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev8 = timer.run(lambda s: stepper8(gsets[s % args.grad_sets], stream=stream), args.steps)
+        torch.cuda.synchronize(dev)
+        ms8, _ = timer.times(ev8)
+        fp8 = {"fp8_iters": args.fp8_iters, "ms_per_step": ms8 / args.steps, "ms_per_step_bf16": ms / args.steps,
+               "speedup": ms / ms8, "steps": args.steps,
+               "what": "muon_step_fp8: e4m3 operands for A*A (iterations 0..F-1) and X*X^T (1..F-1); "
+                       "a reduced-precision variant, not the headline"}
+        del stepper8
     if muon.sync_status(stream) != 0:
         raise RuntimeError("device status after timing: " + muon.last_error())
     ms_max = mdist.max_over_ranks(ms, device=dev)
@@ -575,6 +592,7 @@ def run_ours(args):
                        "cold_l2": "a 1 GiB buffer is written before each cold step (evicts the 126 MB L2)"},
         "kernels": kinds,
         "sweep": sweep,
+        "fp8_variant": fp8,
         "frac_of_dense_peak": value / world / burst,
         "frac_of_dense_spec": value / world / 2250.0,
         "peaks": {"source": peak_src, "bf16_tflops": peaks.get("bf16_tflops"),
@@ -598,6 +616,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-events", type=int, default=1, help="per-launch CUDA events in a second timed pass")
+    ap.add_argument("--fp8-iters", type=int, default=2,
+                    help="also time muon_step_fp8 with this many e4m3 iterations (0: skip)")
     ap.add_argument("--replicas", action="store_true",
                     help="under torchrun: an independent copy of the workload per rank instead of the sharded step")
     ap.add_argument("--per-phase", action="store_true",

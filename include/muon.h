@@ -95,6 +95,37 @@ int muon_step_ex(float* const* params, const float* const* grads, float* const* 
                  float a, float b, float c, float eps, int nesterov, void* stream);
 
 /*
+ * muon_step_ex with e4m3 (fp8) operands in the first `fp8_iters` quintic
+ * iterations (0 <= fp8_iters <= 2; 0 is muon_step_ex).  A reduced-precision
+ * variant, not the method as the article states it (its lessons paragraph
+ * runs the iteration in bf16); the fp8 training results quoted on the
+ * Karpathy-tweets page (llm.c, tensorwise vs rowwise scaling) motivate it.
+ *   - Which products read e4m3 operands: the A A product of iterations
+ *     0 .. fp8_iters-1 and the X X^T product of iterations 1 .. fp8_iters-1.
+ *     They take e4m3 copies of their operands scaled by a power of two (fixed
+ *     per iteration from bounds on the singular values, see the source) and
+ *     accumulate in fp32; the epilogues still work in fp32 and write the bf16
+ *     results as before, plus the e4m3 copies.  The update B X keeps bf16
+ *     operands in every iteration (an e4m3 iterate would move its singular
+ *     vectors, which no later iteration corrects), and so does iteration 0's
+ *     X X^T (the first iterate is stored before the norm of G is known).
+ *   - Error: the same as the bf16 path's to within a few 1e-4 relative
+ *     Frobenius (about 1e-2 against exact NS5 on Gaussian, tall and
+ *     ill-conditioned inputs); e4m3 in a third iteration would not stay
+ *     within 3e-2.
+ *   - Applies to the tcgen05 GEMM path; matrices that the fused single-CTA
+ *     and CTA-pair kernels run whole (short side <= 128 with long side <= 512,
+ *     or both sides <= 256) keep bf16 operands.
+ *   - Workspace: the e4m3 copies take kp*lp + kp*kp more bytes per matrix
+ *     (kp, lp: short and long side rounded up to 128) than muon_workspace_size
+ *     reports.
+ * Returns MUON_ERR_INVALID_ARG for fp8_iters outside [0, 2], else as muon_step_ex.
+ */
+int muon_step_fp8(float* const* params, const float* const* grads, float* const* momentum_bufs,
+                  const int64_t* shapes, int n, float lr, float mu, int ns_steps, float a, float b, float c,
+                  float eps, int nesterov, int fp8_iters, void* stream);
+
+/*
  * NS5 alone (the zeroth_power_via_newtonschulz5 listing): O_i = NS5(G_i)
  * with the listing's defaults and `ns_steps` iterations.  G_i is read only,
  * O_i (m x n fp32, caller-owned device memory) is overwritten.

@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
     L.muon_step.restype = ctypes.c_int
     L.muon_step_ex.argtypes = step_args + [ctypes.c_float] * 4 + [ctypes.c_int, _P]
     L.muon_step_ex.restype = ctypes.c_int
+    L.muon_step_fp8.argtypes = step_args + [ctypes.c_float] * 4 + [ctypes.c_int, ctypes.c_int, _P]
+    L.muon_step_fp8.restype = ctypes.c_int
     L.muon_step_host.argtypes = step_args + [_P]
     L.muon_step_host.restype = ctypes.c_int
     L.muon_step_noalloc.argtypes = step_args + [_P]
@@ -176,11 +178,18 @@ def _marshal_step(params, grads, bufs, device_kind="cuda"):
 
 
 def step(params, grads, bufs, lr: float, mu: float, ns_steps: int = NS_STEPS, *, a: float = NS_A,
-         b: float = NS_B, c: float = NS_C, eps: float = NS_EPS, nesterov: bool = True, stream=None):
-    """One Muon step, in place on ``params`` and ``bufs`` (lists of CUDA fp32 matrices)."""
+         b: float = NS_B, c: float = NS_C, eps: float = NS_EPS, nesterov: bool = True, fp8_iters: int = 0,
+         stream=None):
+    """One Muon step, in place on ``params`` and ``bufs`` (lists of CUDA fp32 matrices).
+    ``fp8_iters`` > 0 selects the reduced-precision variant ``muon_step_fp8``
+    (e4m3 operands in the first one or two iterations)."""
     pp, gp, bp, sh, n = _marshal_step(params, grads, bufs)
-    rc = lib().muon_step_ex(pp, gp, bp, sh, n, float(lr), float(mu), int(ns_steps), float(a), float(b), float(c),
-                            float(eps), 1 if nesterov else 0, _stream(stream))
+    if fp8_iters:
+        rc = lib().muon_step_fp8(pp, gp, bp, sh, n, float(lr), float(mu), int(ns_steps), float(a), float(b),
+                                 float(c), float(eps), 1 if nesterov else 0, int(fp8_iters), _stream(stream))
+    else:
+        rc = lib().muon_step_ex(pp, gp, bp, sh, n, float(lr), float(mu), int(ns_steps), float(a), float(b),
+                                float(c), float(eps), 1 if nesterov else 0, _stream(stream))
     _check(rc)
 
 
@@ -188,12 +197,12 @@ class PreparedStep:
     """A Muon step bound to fixed ``params`` and ``bufs`` (the usual training
     loop: the same weight and momentum tensors every step).  Their checks and
     pointer arrays are built once; each call checks and marshals only the
-    gradients, then makes the same ``muon_step_ex`` call as :func:`step`.
+    gradients, then makes the same library call as :func:`step`.
     The bound tensors must keep their storage (no re-allocation) while the
     object is in use."""
 
     def __init__(self, params, bufs, lr: float, mu: float, ns_steps: int = NS_STEPS, *, a: float = NS_A,
-                 b: float = NS_B, c: float = NS_C, eps: float = NS_EPS, nesterov: bool = True):
+                 b: float = NS_B, c: float = NS_C, eps: float = NS_EPS, nesterov: bool = True, fp8_iters: int = 0):
         n = len(params)
         if len(bufs) != n or n == 0:
             raise ValueError("params and bufs must be equally long, non-empty lists")
@@ -204,13 +213,19 @@ class PreparedStep:
         self.n = n
         self.lr, self.mu, self.ns_steps = float(lr), float(mu), int(ns_steps)
         self._abc = (float(a), float(b), float(c), float(eps), 1 if nesterov else 0)
+        self.fp8_iters = int(fp8_iters)
 
     def __call__(self, grads, lr: float = None, stream=None):
         if len(grads) != self.n:
             raise ValueError("params, grads and bufs must be equally long, non-empty lists")
         gp, _ = _marshal("grads", grads, shapes=self._shp)
-        rc = lib().muon_step_ex(self._pp, gp, self._bp, self._sh, self.n, self.lr if lr is None else float(lr),
-                                self.mu, self.ns_steps, *self._abc, _stream(stream))
+        lr = self.lr if lr is None else float(lr)
+        if self.fp8_iters:
+            rc = lib().muon_step_fp8(self._pp, gp, self._bp, self._sh, self.n, lr, self.mu, self.ns_steps,
+                                     *self._abc, self.fp8_iters, _stream(stream))
+        else:
+            rc = lib().muon_step_ex(self._pp, gp, self._bp, self._sh, self.n, lr, self.mu, self.ns_steps,
+                                    *self._abc, _stream(stream))
         _check(rc)
 
 

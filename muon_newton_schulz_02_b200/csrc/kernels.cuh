@@ -44,12 +44,20 @@ constexpr int kMaxClasses = 16;
 constexpr int kMaxMats = 320;
 constexpr int kTmapsPerClass = 8;
 constexpr int kPad = 128;           // padding granule of the short and long sides
+constexpr int kBK8 = 128;           // K per pipeline stage of e4m3 operands: one 128-byte swizzle row
+constexpr int kUmmaK8 = 32;         // K of one tcgen05.mma kind::f8f6f4
+constexpr int kTmaps8PerClass = 4;
+constexpr int kMaxFp8Iters = 2;     // e4m3 operands reach at most the first two iterations
 
 enum TmapSlot : int {
   kTmX0 = 0, kTmX1 = 1,             // iterates, 64 x 128 boxes (K-major operand rows, epilogue slices, stores)
   kTmX0mn = 2, kTmX1mn = 3,         // iterates, 64 x 64 boxes (MN-major operand of the update)
   kTmA = 4, kTmB = 5,               // Gram / polynomial matrices, 64 x 128 boxes
   kTmAmn = 6, kTmBmn = 7            // Gram / polynomial matrices, 64 x 64 boxes (transposed operand reads)
+};
+enum Tmap8Slot : int {
+  kTm8X = 0, kTm8A = 1,             // e4m3 copies of X and A, 128 x 128 boxes (K-major and MN-major operand reads)
+  kTm8Xs = 2, kTm8As = 3            // the same tensors, 64 x 128 boxes with the 64-byte swizzle (epilogue stores)
 };
 enum GemmMode : int { kModeGram = 0, kModePoly = 1, kModeUpdate = 2,
                       kModeFinal = 3 };   // work items only: the last update, with W -= lr*O
@@ -100,6 +108,7 @@ static_assert(sizeof(WorkItem) == 16, "WorkItem layout");
 
 struct GemmArgs {
   const CUtensorMap* tmaps;
+  const CUtensorMap* tmaps8;  // per class kTmaps8PerClass maps of the e4m3 copies (null: no e4m3 iteration)
   const CUtensorMap* wmaps;   // per matrix (group order): W as fp32 [m][n]; box 32x128 (X = W) or 32x32 (X = W^T)
   const float* scale;     // per matrix (group order): 1/(||G||_F + eps)
   int* status;
@@ -109,6 +118,9 @@ struct GemmArgs {
   unsigned long long wait_limit_ns;
   int nclasses, total_tiles;
   int mode, x_in, first, final_apply, assign, debug_flags;
+  int iter;               // one launch per phase: the Newton-Schulz iteration
+  int fp8_iters;          // iterations whose products read e4m3 operands (see set_precision), <= kMaxFp8Iters
+  float sx8[kMaxFp8Iters], sa8[kMaxFp8Iters];   // power-of-two scales of the e4m3 copies of X_i and A_i
   float a, b, c, lr;
   GemmClass cls[kMaxClasses];
   OutMat out[kMaxMats];
@@ -340,7 +352,26 @@ struct Tile {
   int first;      // first iteration: the normalisation scale is folded in
   int mat;        // matrix in group order
   int need;       // chained launch: tile halves of `mat` that must have completed first
+  int it;         // Newton-Schulz iteration
+  int op8;        // the product reads e4m3 copies of its operands (K = 128 per stage)
+  int dual;       // besides its bf16 output, write the e4m3 copy the next product reads (A, or X)
+  int nsub;       // chunks per 64-column slice of the output: 2 (last update, dual) or 1
 };
+
+// Which products of iteration `it` read e4m3 operands, for fp8_iters = F
+// (0 <= F <= 2): the A A product of iterations 0 .. F-1 and the X X^T product
+// of iterations 1 .. F-1.  The update B' X keeps bf16 operands throughout: an
+// e4m3 rounding of the iterate itself moves its singular vectors, which no
+// later iteration corrects, while a rounding of A only perturbs the polynomial
+// that maps the singular values.  The first Gram product stays bf16 too: X0 is
+// stored before the norm of G is known, so no fixed scale fits it, while every
+// later iterate and Gram matrix is bounded through the singular values (see
+// the host's scales).
+__device__ __forceinline__ void set_precision(Tile& T, int F) {
+  T.op8 = T.mode == kModePoly ? T.it < F : (T.mode == kModeGram && T.it >= 1 && T.it < F);
+  T.dual = T.mode == kModeGram ? T.it < F : (T.mode == kModeUpdate && !T.fin && T.it + 1 < F);
+  T.nsub = (T.fin || T.dual) ? 2 : 1;
+}
 
 // Byte offset of the 16-byte unit u (0..7) of row r inside a 128-row x 128-byte
 // box stored with the 128-byte swizzle (the pattern TMA writes / reads).
@@ -444,12 +475,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       const WorkItem w = p.items[item0 + i];
       T.fin = w.mode == kModeFinal;
       T.mode = T.fin ? kModeUpdate : w.mode; T.cls = w.cls; T.b = w.b; T.tm = w.tm; T.tn = w.tn;
-      T.x_in = w.it & 1; T.first = w.it == 0; T.mat = w.mat; T.need = w.need;
+      T.x_in = w.it & 1; T.first = w.it == 0; T.mat = w.mat; T.need = w.need; T.it = w.it;
     } else {
       const TileCoord tc = decode_tile(p, cid + i * ncl, kMode != kModeUpdate);
       T.mode = kMode; T.fin = kFinal; T.cls = tc.cls; T.b = tc.b; T.tm = tc.tm; T.tn = tc.tn;
-      T.x_in = p.x_in; T.first = p.first; T.mat = p.cls[tc.cls].mat_first + tc.b; T.need = 0;
+      T.x_in = p.x_in; T.first = p.first; T.mat = p.cls[tc.cls].mat_first + tc.b; T.need = 0; T.it = p.iter;
     }
+    set_precision(T, p.fp8_iters);
     return T;
   };
 
@@ -490,6 +522,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           tmap_acquire(tm);
           tmap_prefetch(tm);
         }
+      if (p.tmaps8)
+        for (int c = 0; c < p.nclasses; ++c)
+          for (int k = kTm8X; k <= kTm8A; ++k) {
+            const CUtensorMap* tm = &p.tmaps8[c * kTmaps8PerClass + k];
+            tmap_acquire(tm);
+            tmap_prefetch(tm);
+          }
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -513,7 +552,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         // an operand block below the diagonal is read through its stored transpose.
         const CUtensorMap* tAt = (T.mode == kModePoly) ? &p.tmaps[C.tmap_base + kTmAmn]
                                                        : &p.tmaps[C.tmap_base + kTmBmn];
-        const int kblocks = (T.mode == kModeGram ? C.lp : C.kp) / kBK;
+        // e4m3 operands (Gram: X, polynomial: A): one 128 x 128 box per operand and
+        // stage, read K-major or (blocks below the diagonal) MN-major from one map
+        const CUtensorMap* t8 = T.op8 ? &p.tmaps8[T.cls * kTmaps8PerClass + (T.mode == kModeGram ? kTm8X : kTm8A)]
+                                      : nullptr;
+        const int bk = T.op8 ? kBK8 : kBK;
+        const int kbpb = kTile / bk;                          // K-blocks per 256-block
+        const int kblocks = (T.mode == kModeGram ? C.lp : C.kp) / bk;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, wc, kDevTimeoutEmpty)) { ok = false; break; }
           uint8_t* sa = stage_base + stage * kStageBytes;
@@ -523,9 +568,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           // on a diagonal tile of the symmetric phases a CTA's A rows are its B
           // rows: load them once, the MMA reads both operands from the A buffer
           const bool same_ab = sym && T.tm == T.tn;
-          if (!inject_skip) {
+          const bool a_below = T.mode != kModeGram && T.tm > kb / kbpb;
+          const bool b_mn = T.mode == kModeUpdate || (T.mode == kModePoly && T.tn > kb / kbpb);
+          if (!inject_skip && T.op8) {
             if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], same_ab ? 2 * kStageABytes : 2 * kStageBytes);
-            if (T.mode != kModeGram && T.tm > (kb >> 2)) {
+            if (a_below) tma_load_3d_pair(sa, t8, full_lead, arow, kb * kBK8, T.b);
+            else tma_load_3d_pair(sa, t8, full_lead, kb * kBK8, arow, T.b);
+            if (!same_ab) {
+              if (b_mn) tma_load_3d_pair(sb, t8, full_lead, bidx, kb * kBK8, T.b);
+              else tma_load_3d_pair(sb, t8, full_lead, kb * kBK8, bidx, T.b);
+            }
+          } else if (!inject_skip) {
+            if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], same_ab ? 2 * kStageABytes : 2 * kStageBytes);
+            if (a_below) {
               // A rows below the diagonal block: columns [arow, +128) of rows [kb*64, +64), MN-major
               tma_load_3d_pair(sa, tAt, full_lead, arow, kb * kBK, T.b);
               tma_load_3d_pair(sa + kStageABytes / 2, tAt, full_lead, arow + 64, kb * kBK, T.b);
@@ -534,7 +589,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             }
             if (same_ab) {
               // nothing: B is the A block just loaded
-            } else if (T.mode == kModeUpdate || (T.mode == kModePoly && T.tn > (kb >> 2))) {
+            } else if (b_mn) {
               // B = rows [kb*64, +64) x this CTA's 128 columns, MN-major: two 64-col boxes
               const CUtensorMap* tBm = (T.mode == kModeUpdate) ? tB : tAt;
               tma_load_3d_pair(sb, tBm, full_lead, bidx, kb * kBK, T.b);
@@ -564,7 +619,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         if (!mbar_wait_cluster(&ctl->tmem_empty[acc], acc_phase ^ 1u, wc, kDevTimeoutAccum)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
-        const int kblocks = (T.mode == kModeGram ? C.lp : C.kp) / kBK;
+        const int bk = T.op8 ? kBK8 : kBK;
+        const int kbpb = kTile / bk;
+        const int kblocks = (T.mode == kModeGram ? C.lp : C.kp) / bk;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&ctl->full[stage], phase, wc, kDevTimeoutFull)) { ok = false; break; }
           tc_fence_after();
@@ -573,17 +630,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           // share one operand buffer, blocks below the diagonal arrive MN-major
           const bool same_ab = sym && T.tm == T.tn;
           const uint32_t sb = same_ab ? sa : sa + kStageABytes;
-          const uint32_t a_mn = (T.mode != kModeGram && T.tm > (kb >> 2)) ? 1u : 0u;
+          const uint32_t a_mn = (T.mode != kModeGram && T.tm > kb / kbpb) ? 1u : 0u;
           const uint32_t b_mn = same_ab ? a_mn
-                                : (T.mode == kModeUpdate || (T.mode == kModePoly && T.tn > (kb >> 2))) ? 1u : 0u;
-          const uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN, a_mn, b_mn);
+                                : (T.mode == kModeUpdate || (T.mode == kModePoly && T.tn > kb / kbpb)) ? 1u : 0u;
+          if (T.op8) {
+            // 128 MN bytes per CTA: one swizzle atom wide, so only the K stride (SBO) matters MN-major
+            const uint32_t idesc = idesc_e4m3_f32(2 * kBM, kBN, a_mn, b_mn);
 #pragma unroll
-          for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-            const uint64_t adesc = a_mn ? smem_desc_sw128(sa + kk * (kUmmaK * 128), kStageABytes / 2, 1024)
-                                        : smem_desc_sw128(sa + kk * (kUmmaK * 2), 16, 1024);
-            const uint64_t bdesc = b_mn ? smem_desc_sw128(sb + kk * (kUmmaK * 128), kStageBBytes / 2, 1024)
-                                        : smem_desc_sw128(sb + kk * (kUmmaK * 2), 16, 1024);
-            tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < kBK8 / kUmmaK8; ++kk) {
+              const uint64_t adesc = a_mn ? smem_desc_sw128(sa + kk * (kUmmaK8 * 128), kStageABytes, 1024)
+                                          : smem_desc_sw128(sa + kk * kUmmaK8, 16, 1024);
+              const uint64_t bdesc = b_mn ? smem_desc_sw128(sb + kk * (kUmmaK8 * 128), kStageBBytes, 1024)
+                                          : smem_desc_sw128(sb + kk * kUmmaK8, 16, 1024);
+              tc_mma_e4m3_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
+          } else {
+            const uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN, a_mn, b_mn);
+#pragma unroll
+            for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+              const uint64_t adesc = a_mn ? smem_desc_sw128(sa + kk * (kUmmaK * 128), kStageABytes / 2, 1024)
+                                          : smem_desc_sw128(sa + kk * (kUmmaK * 2), 16, 1024);
+              const uint64_t bdesc = b_mn ? smem_desc_sw128(sb + kk * (kUmmaK * 128), kStageBBytes / 2, 1024)
+                                          : smem_desc_sw128(sb + kk * (kUmmaK * 2), 16, 1024);
+              tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
           }
           issued_any = true;
           tc_commit_pair(mapa_shared(&ctl->empty[stage], 0));
@@ -605,6 +675,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     if (lane == 0) {
       for (int c = 0; c < p.nclasses; ++c)
         for (int k = 0; k < kTmapsPerClass; ++k) tmap_acquire(&p.tmaps[p.cls[c].tmap_base + k]);
+      if (p.tmaps8)
+        for (int c = 0; c < p.nclasses; ++c)
+          for (int k = kTm8Xs; k <= kTm8As; ++k) tmap_acquire(&p.tmaps8[c * kTmaps8PerClass + k]);
       if (p.final_apply)
         for (int c = 0; c < p.nclasses; ++c)
           for (int b = 0; b < p.cls[c].batch; ++b)
@@ -638,7 +711,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             mbar_arrive(&ctl->in_full[b]);
           }
           ++armed;
-          if (++ha == (TA.fin ? 8 : 4)) {
+          if (++ha == 4 * TA.nsub) {
             ha = 0;
             if (++ia < my_tiles) TA = tile_of(ia);
           }
@@ -650,10 +723,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         const Tile T = tile_of(i);
         const GemmClass& C = p.cls[T.cls];
         const int row0 = T.tm * kTile + (int)rank * kBM;
-        const int nch = T.fin ? 8 : 4;
+        const int nch = 4 * T.nsub;
         const CUtensorMap* tO = T.mode == kModeGram ? &p.tmaps[C.tmap_base + kTmA]
                               : T.mode == kModePoly ? &p.tmaps[C.tmap_base + kTmB]
                                                     : &p.tmaps[C.tmap_base + (T.x_in ? kTmX0 : kTmX1)];
+        // e4m3 copy of the output (dual tiles): of A (Gram) or of the next iterate (update)
+        const CUtensorMap* tO8 = !T.dual ? nullptr
+                               : &p.tmaps8[T.cls * kTmaps8PerClass + (T.mode == kModeGram ? kTm8As : kTm8Xs)];
         for (int h = 0; h < nch; ++h, ++q) {
           const int b = q & 3;
           if (!mbar_wait(&ctl->out_full[b], (uint32_t)((q >> 2) & 1), wc, kDevTimeoutEpi)) { ok = false; break; }
@@ -681,8 +757,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             // stores start inside the tensor only (a pair tile can overhang the
             // 128-padded edge by half; the overhang is never stored)
             const int ocols = T.mode != kModeUpdate ? C.kp : C.lp;
-            const int x0 = T.tn * kTile + 64 * h;
-            if (row0 < C.kp && x0 < ocols) tma_store_3d(tO, S, x0, row0, T.b);
+            const int x0 = T.tn * kTile + 64 * (h / T.nsub);
+            const CUtensorMap* dst = (T.dual && (h & 1)) ? tO8 : tO;   // a dual tile's odd chunks: the e4m3 copy
+            if (row0 < C.kp && x0 < ocols) tma_store_3d(dst, S, x0, row0, T.b);
           }
           tma_store_commit();                      // one bulk group per chunk
           if (armed < q + 4 && ia < my_tiles && !deferred(i)) {
@@ -724,6 +801,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       if (!ok) break;
       tc_fence_after();
       const float s = T.first ? p.scale[T.mat] : 1.0f;
+      // an e4m3 product carries the (power-of-two) scales of its operand copies
+      const float pscale = !T.op8 ? 1.f
+                           : T.mode == kModeGram ? 1.f / (p.sx8[T.it] * p.sx8[T.it])
+                                                 : 1.f / (p.sa8[T.it] * p.sa8[T.it]);
+      // scale of this tile's e4m3 output copy
+      const float oscale = !T.dual ? 1.f : T.mode == kModeGram ? p.sa8[T.it] : p.sx8[T.it + 1];
       const int row0 = T.tm * kTile + (int)rank * kBM;
       const uint32_t tbase = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * kBN);
 #pragma unroll 1
@@ -739,11 +822,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         if (T.mode != kModePoly) {
           // Gram: s^2 X X^T.  Update: s (aI + B) X = a s X + s B X, the aI term
           // carried on the diagonal of the polynomial phase's output.
-          const float alpha = T.mode == kModeGram ? s * s : s;
+          const float alpha = (T.mode == kModeGram ? s * s : s) * pscale;
 #pragma unroll
           for (int i = 0; i < 64; ++i) v[i] *= alpha;
         } else {
           // b A + c A A
+          const float cm = p.c * pscale;
           const uint8_t* dslice = slice_buf(q & 3);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -752,8 +836,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               float2 f = __bfloat1622float2(hv[e]);
-              v[u * 8 + 2 * e] = fmaf(p.c, v[u * 8 + 2 * e], p.b * f.x);
-              v[u * 8 + 2 * e + 1] = fmaf(p.c, v[u * 8 + 2 * e + 1], p.b * f.y);
+              v[u * 8 + 2 * e] = fmaf(cm, v[u * 8 + 2 * e], p.b * f.x);
+              v[u * 8 + 2 * e + 1] = fmaf(cm, v[u * 8 + 2 * e + 1], p.b * f.y);
             }
           }
           // + a on the diagonal: on a diagonal tile, a warp's 32 rows meet the
@@ -824,6 +908,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
             o.z = pack_bf16x2(v[u * 8 + 4], v[u * 8 + 5]);
             o.w = pack_bf16x2(v[u * 8 + 6], v[u * 8 + 7]);
             *reinterpret_cast<uint4*>(dslice + sw128_off((uint32_t)r, (uint32_t)u)) = o;
+          }
+          if (T.dual) {
+            // the e4m3 copy goes into the next chunk: 128 rows x 64 bytes with the
+            // 64-byte swizzle (16-byte unit u of row r at unit u ^ ((r >> 1) & 3))
+            fence_async_shared();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->out_full[q & 3]);
+            ++q;
+            if (!(ok = take())) break;
+            dslice = slice_buf(q & 3);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float* w = v + 16 * u;
+              uint4 o;
+              o.x = pack_e4m3x4(oscale * w[0], oscale * w[1], oscale * w[2], oscale * w[3]);
+              o.y = pack_e4m3x4(oscale * w[4], oscale * w[5], oscale * w[6], oscale * w[7]);
+              o.z = pack_e4m3x4(oscale * w[8], oscale * w[9], oscale * w[10], oscale * w[11]);
+              o.w = pack_e4m3x4(oscale * w[12], oscale * w[13], oscale * w[14], oscale * w[15]);
+              *reinterpret_cast<uint4*>(dslice + r * 64 + ((u ^ ((r >> 1) & 3)) << 4)) = o;
+            }
           }
           fence_async_shared();
           __syncwarp();

@@ -16,6 +16,7 @@
 #include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdio>
 #include <cstdlib>
@@ -27,6 +28,7 @@
 #include <queue>
 #include <set>
 #include <string>
+#include <tuple>
 #include <vector>
 
 #include "muon.h"
@@ -79,6 +81,7 @@ struct ClassDesc {
   int kp, lp;
   std::vector<int> mats;    // group-order indices
   size_t off_x0, off_x1, off_a, off_b;
+  size_t off_x8 = 0, off_a8 = 0;   // e4m3 copies of X and A (muon_step_fp8 only), past every other region
 };
 
 struct Group {
@@ -87,6 +90,7 @@ struct Group {
   std::vector<int> pro_tile_begin;
   int pro_tiles = 0;
   size_t off_partials = 0, off_tickets = 0, off_scale = 0, off_done = 0, off_tmaps = 0, off_wmaps = 0;
+  size_t off_tmaps8 = 0;           // in Plan::tmaps8
   size_t data_bytes = 0;
   int sym_tiles = 0, upd_tiles = 0;
   std::vector<GemmClass> sym_cls, upd_cls;
@@ -116,17 +120,21 @@ struct Plan {
   std::vector<MatDesc> small;               // matrices of the fused single-CTA kernel (no workspace)
   std::vector<MatDesc> pair;                // matrices of the fused CTA-pair kernel (no workspace)
   size_t ws_bytes = 0;
+  size_t ws_bytes_fp8 = 0;                  // with the e4m3 copies of muon_step_fp8
   size_t tmap_bytes = 0;
+  size_t tmap8_bytes = 0;
   void* ws = nullptr;                       // workspace the tensor maps point into
   void* tmaps = nullptr;                    // this plan's own device copy of its tensor maps
+  void* tmaps8 = nullptr;                   // tensor maps of the e4m3 copies, encoded by the first fp8 call
   // Per group: fp32 tensor maps of the caller's output matrices, re-encoded
   // when the caller passes other pointers; host copy in pinned memory.
   std::vector<std::vector<const void*>> wmap_key;
   std::vector<CUtensorMap*> wmap_host;
   cudaEvent_t wmap_copied = nullptr;
-  std::map<std::pair<size_t, int>, ChainTables> chains;   // (group, ns_steps) -> work lists
+  std::map<std::tuple<size_t, int, int>, ChainTables> chains;   // (group, ns_steps, fp8_iters) -> work lists
   ~Plan() {
     if (tmaps) cudaFree(tmaps);
+    if (tmaps8) cudaFree(tmaps8);
     for (auto& kv : chains)
       if (kv.second.dev) cudaFree(kv.second.dev);
     for (auto h : wmap_host)
@@ -245,6 +253,22 @@ int build_layout(const int64_t* shapes, int n, Plan& plan) {
   }
   plan.tmap_bytes = off;
   plan.ws_bytes = data_max;
+  // e4m3 copies of X and A (muon_step_fp8) after everything else, so that
+  // the bf16 path's layout and size do not depend on them
+  plan.ws_bytes_fp8 = data_max;
+  off = 0;
+  for (auto& g : plan.groups) {
+    size_t o = align_up(data_max, 1024);
+    for (auto& cd : g.classes) {
+      const size_t batch = cd.mats.size();
+      cd.off_x8 = o; o = align_up(o + batch * (size_t)cd.kp * cd.lp, 1024);
+      cd.off_a8 = o; o = align_up(o + batch * (size_t)cd.kp * cd.kp, 1024);
+    }
+    plan.ws_bytes_fp8 = std::max(plan.ws_bytes_fp8, o);
+    g.off_tmaps8 = off;
+    off = align_up(off + g.classes.size() * kTmaps8PerClass * sizeof(CUtensorMap), 1024);
+  }
+  plan.tmap8_bytes = off;
   return MUON_OK;
 }
 
@@ -273,7 +297,8 @@ double chain_latency_units() {
   return lat;
 }
 
-void build_chain(const Group& g, int ns_steps, int ncl, std::vector<WorkItem>& items, std::vector<int>& off) {
+void build_chain(const Group& g, int ns_steps, int fp8_iters, int ncl, std::vector<WorkItem>& items,
+                 std::vector<int>& off) {
   constexpr double kOverhead = 2.0;
   constexpr double kFinalCost = 1.5;          // the last update also reads and writes W
   const double lat = chain_latency_units();
@@ -282,13 +307,20 @@ void build_chain(const Group& g, int ns_steps, int ncl, std::vector<WorkItem>& i
   struct MatState {
     int cls = 0, b = 0, T = 0, Tn = 0;
     int ntiles[4] = {0, 0, 0, 0};
-    double cost[4] = {0, 0, 0, 0};
+    double cost[4] = {0, 0, 0, 0};   // bf16 operands; a product with e4m3 operands has half the K-blocks
     int phase = 0, next = 0;
     int need = 0;              // tile halves completed before the current phase
     double vis = 0.0;          // latest visibility time among the current phase's tiles
     double total = 0.0;
   };
   auto mode_of = [&](int j) { return j == nphases - 1 ? (int)kModeFinal : j % 3; };
+  auto cost_of = [&](const auto& st, int j) {   // which products read e4m3 operands: as the kernel's set_precision
+    const int it = j / 3, mode = j % 3;
+    const bool op8 = mode == kModePoly ? it < fp8_iters : (mode == kModeGram && it >= 1 && it < fp8_iters);
+    const double kb = (mode == kModeGram ? st.cost[kModeGram] : st.cost[kModeUpdate]) - kOverhead;
+    const double c = (op8 ? kb / 2 : kb) + kOverhead;
+    return mode_of(j) == kModeFinal ? kFinalCost * c : c;
+  };
   std::vector<MatState> ms(nm);
   for (size_t ci = 0; ci < g.classes.size(); ++ci) {
     const ClassDesc& cd = g.classes[ci];
@@ -303,7 +335,7 @@ void build_chain(const Group& g, int ns_steps, int ncl, std::vector<WorkItem>& i
       st.cost[kModeGram] = cd.lp / kBK + kOverhead;
       st.cost[kModePoly] = st.cost[kModeUpdate] = cd.kp / kBK + kOverhead;
       st.cost[kModeFinal] = kFinalCost * st.cost[kModeUpdate];
-      for (int j = 0; j < nphases; ++j) st.total += st.ntiles[mode_of(j)] * st.cost[mode_of(j)];
+      for (int j = 0; j < nphases; ++j) st.total += st.ntiles[mode_of(j)] * cost_of(st, j);
     }
   }
   // priority: more total work first (its long chain starts early), then group order
@@ -360,7 +392,7 @@ void build_chain(const Group& g, int ns_steps, int ncl, std::vector<WorkItem>& i
     w.mode = (unsigned char)mode;
     w.it = (unsigned short)(st.phase / 3);
     lists[c].push_back(w);
-    const double end = t + st.cost[mode];
+    const double end = t + cost_of(st, st.phase);
     st.vis = std::max(st.vis, end + lat);
     free_at.push({end, c});
     --left;
@@ -380,17 +412,32 @@ void build_chain(const Group& g, int ns_steps, int ncl, std::vector<WorkItem>& i
   }
 }
 
-int encode_map(CUtensorMap* map, void* base, int cols, int rows, int batch, int box_cols, int box_rows) {
+// [batch][rows][cols] tensor of bf16 (esize 2) or e4m3 bytes (esize 1).
+int encode_map(CUtensorMap* map, void* base, int cols, int rows, int batch, int box_cols, int box_rows,
+               int esize = 2, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (!fn) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
-  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * rows * 2};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * esize, (cuuint64_t)cols * rows * esize};
   cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims,
+                  strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return MUON_OK;
+}
+
+// The tensor maps of one shape class's e4m3 copies (see Tmap8Slot).
+int encode_class_maps8(CUtensorMap* m, char* base, const ClassDesc& cd) {
+  const int batch = (int)cd.mats.size();
+  int rc;
+  if ((rc = encode_map(&m[kTm8X], base + cd.off_x8, cd.lp, cd.kp, batch, 128, 128, 1))) return rc;
+  if ((rc = encode_map(&m[kTm8A], base + cd.off_a8, cd.kp, cd.kp, batch, 128, 128, 1))) return rc;
+  if ((rc = encode_map(&m[kTm8Xs], base + cd.off_x8, cd.lp, cd.kp, batch, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_64B)))
+    return rc;
+  if ((rc = encode_map(&m[kTm8As], base + cd.off_a8, cd.kp, cd.kp, batch, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_64B)))
+    return rc;
   return MUON_OK;
 }
 
@@ -579,20 +626,49 @@ int ensure_workspace(Ctx& c, size_t bytes) {
 
 constexpr size_t kMaxPlans = 48;
 
-int get_plan(Ctx& c, const int64_t* shapes, int n, Plan** out) {
+// Tensor maps of the plan's e4m3 copies (muon_step_fp8), encoded on first use.
+int ensure_fp8_maps(Plan& p) {
+  if (p.tmaps8 || !p.tmap8_bytes) return MUON_OK;
+  void* d = nullptr;
+  if (cudaMalloc(&d, p.tmap8_bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MUON_ERR_NOMEM, "tensor-map table allocation failed");
+  }
+  for (auto& g : p.groups) {
+    std::vector<CUtensorMap> maps(g.classes.size() * kTmaps8PerClass);
+    int rc = MUON_OK;
+    for (size_t ci = 0; ci < g.classes.size() && !rc; ++ci)
+      rc = encode_class_maps8(&maps[ci * kTmaps8PerClass], (char*)p.ws, g.classes[ci]);
+    if (!rc && cudaMemcpy((char*)d + g.off_tmaps8, maps.data(), maps.size() * sizeof(CUtensorMap),
+                          cudaMemcpyHostToDevice) != cudaSuccess) {
+      const cudaError_t e = cudaGetLastError();
+      rc = fail(MUON_ERR_CUDA, std::string("tensor-map upload failed: ") + cudaGetErrorString(e));
+    }
+    if (rc) {
+      cudaFree(d);
+      return rc;
+    }
+  }
+  p.tmaps8 = d;
+  return MUON_OK;
+}
+
+// The plan of these shapes, built on first use; `fp8`: the workspace must also
+// hold the e4m3 copies and their tensor maps must exist.
+int get_plan(Ctx& c, const int64_t* shapes, int n, Plan** out, bool fp8 = false) {
   for (auto it = c.plans.begin(); it != c.plans.end(); ++it) {
     Plan& p = **it;
     if ((int)p.shapes.size() == 2 * n && std::memcmp(p.shapes.data(), shapes, sizeof(int64_t) * 2 * n) == 0 &&
-        p.ws == c.ws) {
+        p.ws == c.ws && (!fp8 || c.ws_cap >= p.ws_bytes_fp8)) {
       c.plans.splice(c.plans.begin(), c.plans, it);
       *out = c.plans.front().get();
-      return MUON_OK;
+      return fp8 ? ensure_fp8_maps(**out) : MUON_OK;
     }
   }
   auto p = std::make_unique<Plan>();
   int rc = build_layout(shapes, n, *p);
   if (rc) return rc;
-  rc = ensure_workspace(c, std::max<size_t>(p->ws_bytes, kTicketBytes));
+  rc = ensure_workspace(c, std::max<size_t>(fp8 ? p->ws_bytes_fp8 : p->ws_bytes, kTicketBytes));
   if (rc) return rc;
   p->ws = c.ws;
   char* base = (char*)c.ws;
@@ -629,7 +705,7 @@ int get_plan(Ctx& c, const int64_t* shapes, int n, Plan** out) {
     while (c.plans.size() > kMaxPlans) c.plans.pop_back();
   }
   *out = c.plans.front().get();
-  return MUON_OK;
+  return fp8 ? ensure_fp8_maps(**out) : MUON_OK;
 }
 
 // ---------------------------------------------------------------- launches ---
@@ -677,7 +753,40 @@ struct StepIO {
   float* const* buf;        // may be null (no momentum)
   float lr, mu, a, b, c, eps;
   int ns_steps, nesterov, assign;
+  int fp8_iters = 0;        // muon_step_fp8: iterations with e4m3 operands (0: bf16 throughout)
 };
+
+// Power-of-two scale that maps magnitudes up to `bound` into e4m3's finite
+// range (|x| <= 448), with a margin for the bf16 rounding of what is bounded.
+float e4m3_scale(double bound) {
+  const double e = std::floor(std::log2(448.0 / (1.0625 * std::max(bound, 1e-30))));
+  return std::ldexp(1.0f, (int)std::min(60.0, std::max(-60.0, e)));
+}
+
+// Scales of the e4m3 copies of X_i and A_i for quintic coefficients (a, b, c).
+// The normalised first iterate has singular values in [0, 1]; an iterate whose
+// singular values lie in [0, r] has a Gram matrix with eigenvalues in [0, r^2]
+// and a successor with singular values |sigma q(sigma^2)|, q(x) = a + b x +
+// c x^2.  Every entry of a matrix is at most its largest singular value, so
+// these bounds (maximised on a fine grid, with the margin above) keep the
+// copies finite.
+void e4m3_scales(float a, float b, float c, float* sx8, float* sa8) {
+  auto q = [&](double x) { return a + b * x + c * x * x; };
+  auto pmax = [&](double r) {                // max |sigma q(sigma^2)| over [0, r]
+    double m = 0.0;
+    for (int i = 0; i <= 4096; ++i) {
+      const double sg = r * i / 4096.0;
+      m = std::max(m, std::fabs(sg * q(sg * sg)));
+    }
+    return m;
+  };
+  double r = 1.0;
+  for (int i = 0; i < kMaxFp8Iters; ++i) {
+    sx8[i] = e4m3_scale(r);
+    sa8[i] = e4m3_scale(r * r);
+    r = pmax(r);
+  }
+}
 
 int check_status(Ctx& c) {
   const int s = *(volatile int*)c.status_h;
@@ -732,15 +841,15 @@ int64_t chain_items(const Group& g, int ns_steps) {
 // The chained launch's work lists for group gidx and ns_steps iterations,
 // built and uploaded on first use (a synchronous copy: make the first call for
 // a set of shapes and an iteration count outside stream capture).
-int get_chain(Ctx& c, Plan& plan, size_t gidx, int ns_steps, ChainTables** out) {
-  const auto key = std::make_pair(gidx, ns_steps);
+int get_chain(Ctx& c, Plan& plan, size_t gidx, int ns_steps, int fp8_iters, ChainTables** out) {
+  const auto key = std::make_tuple(gidx, ns_steps, fp8_iters);
   auto it = plan.chains.find(key);
   if (it == plan.chains.end()) {
     ChainTables ct;
     ct.nclusters = g_chain_clusters[c.dev];
     std::vector<WorkItem> items;
     std::vector<int> off;
-    build_chain(plan.groups[gidx], ns_steps, ct.nclusters, items, off);
+    build_chain(plan.groups[gidx], ns_steps, fp8_iters, ct.nclusters, items, off);
     ct.nitems = (int)items.size();
     const size_t ib = align_up(items.size() * sizeof(WorkItem), 256), ob = off.size() * sizeof(int);
     if (cudaMalloc(&ct.dev, ib + ob) != cudaSuccess) {
@@ -855,10 +964,16 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
   ga->a = io.a; ga->b = io.b; ga->c = io.c; ga->lr = io.lr;
   ga->assign = io.assign;
   fill_out(ga->out);
+  const int fp8_iters = std::min(io.fp8_iters, io.ns_steps);
+  if (fp8_iters > 0) {
+    ga->tmaps8 = (const CUtensorMap*)((char*)plan.tmaps8 + g.off_tmaps8);
+    ga->fp8_iters = fp8_iters;
+    e4m3_scales(io.a, io.b, io.c, ga->sx8, ga->sa8);
+  }
 
   if (chain) {
     ChainTables* ct = nullptr;
-    int rc = get_chain(c, plan, gidx, io.ns_steps, &ct);
+    int rc = get_chain(c, plan, gidx, io.ns_steps, fp8_iters, &ct);
     if (rc) return rc;
     for (size_t ci = 0; ci < g.sym_cls.size(); ++ci) ga->cls[ci] = g.sym_cls[ci];
     ga->items = ct->items;
@@ -882,6 +997,7 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
       ga->mode = mode;
       ga->x_in = it & 1;
       ga->first = it == 0;
+      ga->iter = it;
       ga->final_apply = (mode == kModeUpdate) && (it == io.ns_steps - 1);
       ga->debug_flags = 0;
       if (g_debug_flags & 1) { ga->debug_flags = 1; g_debug_flags &= ~1; }
@@ -1000,7 +1116,7 @@ int step_impl(const StepIO& io, const int64_t* shapes, int n, void* stream) {
   if (rc) return rc;
   if ((rc = check_status(*c))) return rc;
   Plan* plan = nullptr;
-  if ((rc = get_plan(*c, shapes, n, &plan))) return rc;
+  if ((rc = get_plan(*c, shapes, n, &plan, io.fp8_iters > 0 && io.ns_steps > 0))) return rc;
   if (!plan->small.empty() && (rc = run_small(c, c->stream, plan->small, io, c->status_d))) return rc;
   if (!plan->pair.empty() && (rc = run_pair(c, c->stream, plan->pair, io, c->status_d))) return rc;
   for (size_t gi = 0; gi < plan->groups.size(); ++gi)
@@ -1025,6 +1141,23 @@ int muon_step_ex(float* const* params, const float* const* grads, float* const* 
   if (nesterov != 0 && nesterov != 1) return fail(MUON_ERR_INVALID_ARG, "nesterov must be 0 or 1");
   if (!(eps >= 0.f)) return fail(MUON_ERR_INVALID_ARG, "eps must be >= 0");
   StepIO io{params, grads, momentum_bufs, lr, mu, a, b, c, eps, ns_steps, nesterov, 0};
+  return step_impl(io, shapes, n, stream);
+}
+
+int muon_step_fp8(float* const* params, const float* const* grads, float* const* momentum_bufs,
+                  const int64_t* shapes, int n, float lr, float mu, int ns_steps, float a, float b, float c,
+                  float eps, int nesterov, int fp8_iters, void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int rc = validate_common(shapes, n, ns_steps);
+  if (rc) return rc;
+  if ((rc = validate_ptrs((const void* const*)params, n, "params"))) return rc;
+  if ((rc = validate_ptrs((const void* const*)grads, n, "grads"))) return rc;
+  if ((rc = validate_ptrs((const void* const*)momentum_bufs, n, "momentum_bufs"))) return rc;
+  if (nesterov != 0 && nesterov != 1) return fail(MUON_ERR_INVALID_ARG, "nesterov must be 0 or 1");
+  if (!(eps >= 0.f)) return fail(MUON_ERR_INVALID_ARG, "eps must be >= 0");
+  if (fp8_iters < 0 || fp8_iters > kMaxFp8Iters)
+    return fail(MUON_ERR_INVALID_ARG, "fp8_iters must be in [0, " + std::to_string(kMaxFp8Iters) + "]");
+  StepIO io{params, grads, momentum_bufs, lr, mu, a, b, c, eps, ns_steps, nesterov, 0, fp8_iters};
   return step_impl(io, shapes, n, stream);
 }
 
@@ -1231,7 +1364,7 @@ int muon_chain_plan(const int64_t* shapes, int n, int ns_steps, int nclusters, i
   }
   std::vector<WorkItem> list;
   std::vector<int> off;
-  build_chain(plan.groups[0], ns_steps, nclusters, list, off);
+  build_chain(plan.groups[0], ns_steps, 0, nclusters, list, off);
   *nitems = (int64_t)list.size();
   for (int c = 0; c <= nclusters; ++c) cluster_off[c] = off[c];
   if (!items || capacity < (int64_t)list.size())

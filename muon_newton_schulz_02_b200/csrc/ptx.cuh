@@ -365,6 +365,17 @@ __device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t a_des
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The same with e4m3 operands (kind::f8f6f4, K = 32 per instruction, fp32
+// accumulation); both operands are e4m3.
+__device__ __forceinline__ void tc_mma_e4m3_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive once on the barrier at a shared::cluster address (this CTA's or the
 // peer's) when the pair MMAs issued so far by this thread complete.
 __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster_addr) {
@@ -435,6 +446,28 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, ui
          | (a_mn_major << 15) | (b_mn_major << 16)
          | ((N >> 3) << 17)
          | ((M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::f8f6f4: e4m3 A/B (format code 0), fp32 D, dense.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N, uint32_t a_mn_major,
+                                                      uint32_t b_mn_major) {
+  return (1u << 4)                  // D format fp32; A and B format fields 0: e4m3
+         | (a_mn_major << 15) | (b_mn_major << 16)
+         | ((N >> 3) << 17)
+         | ((M >> 4) << 24);
+}
+
+// Four fp32 values as four e4m3 bytes (round to nearest even, saturating to
+// +-448 instead of overflowing), v0 in the lowest byte.  cvt's e4m3x2 form
+// puts its first source in the upper byte of the 16-bit result.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float v0, float v1, float v2, float v3) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r) : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
+  return r;
 }
 
 // ------------------------------------------------------------ bf16 pack ---

@@ -51,6 +51,10 @@ def test_argument_errors_are_reported_before_any_launch(L):
     assert L.muon_step_ex(p, p, p, sh, 1, 0.02, 0.95, 5, 3.4445, -4.775, 2.0315, -1.0, 1, None) == INVALID
     assert L.muon_orthogonalize(p, _arr(1, 0), sh, 1, 5, None) == INVALID
     assert L.muon_step_host(p, None, p, sh, 1, 0.02, 0.95, 5, None) == INVALID
+    for bad_iters in (-1, 3):
+        assert L.muon_step_fp8(p, p, p, sh, 1, 0.02, 0.95, 5, 3.4445, -4.775, 2.0315, 1e-7, 1, bad_iters, None) == INVALID
+        assert "fp8_iters" in muon.last_error()
+    assert L.muon_step_fp8(p, p, p, sh, 1, 0.02, 0.95, 5, 3.4445, -4.775, 2.0315, 1e-7, 2, 1, None) == INVALID
 
 
 def _ws(shapes):

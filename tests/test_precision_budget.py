@@ -91,3 +91,90 @@ def test_fp8_operands_in_first_two_iterations_stay_inside(case):
     mixed = _rel(ns_emulated(G, fp8_iters=(0, 1)), ref)
     assert mixed < 3e-2 and abs(mixed - bf16) < 5e-3
     assert _rel(ns_emulated(G, fp8_iters=(0, 1, 2, 3)), ref) > 3e-2
+
+
+# ---- the e4m3 variant as built (muon_step_fp8) ----------------------------
+# e4m3 copies feed only the Gram product X X^T (iterations 1 .. F-1) and the
+# A A product (iterations 0 .. F-1); every update B'X keeps bf16 operands.  The
+# copies are scaled by powers of two fixed from bounds on the singular values:
+# sigma(X_0) <= 1, sigma(X_{i+1}) <= max |sigma q(sigma^2)| over the previous
+# range, entries of A_i <= sigma_max(X_i)^2.
+
+def _pow2_scale(bound):
+    return 2.0 ** np.floor(np.log2(448.0 / (1.0625 * bound)))
+
+
+def e4m3_scales(a=A_, b=B_, c=C_, iters=2):
+    grid = np.linspace(0.0, 1.0, 4097)
+    r, sx, sa = 1.0, [], []
+    for _ in range(iters):
+        sx.append(_pow2_scale(r))
+        sa.append(_pow2_scale(r * r))
+        s = grid * r
+        r = float(np.abs(s * (a + b * s ** 2 + c * s ** 4)).max())
+    return sx, sa
+
+
+def q_e4m3(x, s):
+    return (x * s).to(torch.float8_e4m3fn).to(torch.float32) / s
+
+
+def ns_fp8_scheme(G, F=2, e4m3_update_iterate=False, steps=5):
+    """The GPU's e4m3 variant: fp32 accumulation, one bf16 rounding per output
+    (aI folded into B'), e4m3 copies where the variant reads them.  With
+    e4m3_update_iterate the update also reads the e4m3 iterate (a rejected
+    design)."""
+    sx, sa = e4m3_scales(iters=max(F, 1))
+    X = torch.tensor(G, dtype=torch.float32)
+    nrm = X.norm() + 1e-7
+    t = X.shape[0] > X.shape[1]
+    if t:
+        X = X.T
+    X = q_bf16(X) / nrm
+    I = torch.eye(X.shape[0])
+    for i in range(steps):
+        e4 = 1 <= i < F
+        Xg = q_e4m3(X, sx[min(i, len(sx) - 1)]) if e4 else X
+        A = Xg @ Xg.T
+        Ao = q_e4m3(A, sa[min(i, len(sa) - 1)]) if i < F else q_bf16(A)
+        Bp = q_bf16(A_ * I + B_ * q_bf16(A) + C_ * (Ao @ Ao))
+        Xn = Bp @ (Xg if (e4 and e4m3_update_iterate) else X)
+        X = Xn if i == steps - 1 else q_bf16(Xn)
+    return (X.T if t else X).double().numpy()
+
+
+def test_fp8_variant_matches_the_bf16_error(case):
+    G, ref = case
+    bf16 = _rel(ns_fp8_scheme(G, F=0), ref)
+    for F in (1, 2):
+        assert abs(_rel(ns_fp8_scheme(G, F=F), ref) - bf16) < 1e-3
+    tall = np.random.default_rng(1).standard_normal((768, 256))
+    ref_t = orc.newton_schulz5(tall)
+    assert abs(_rel(ns_fp8_scheme(tall, F=2), ref_t) - _rel(ns_fp8_scheme(tall, F=0), ref_t)) < 1e-3
+
+
+def test_fp8_iterate_in_the_update_breaks_the_tolerance(case):
+    # why the update keeps bf16 operands
+    G, ref = case
+    assert _rel(ns_fp8_scheme(G, F=2, e4m3_update_iterate=True), ref) > 3e-2
+
+
+def test_fp8_in_a_third_iteration_costs_accuracy(case):
+    # why fp8_iters is capped at 2
+    G, ref = case
+    bf16 = _rel(ns_fp8_scheme(G, F=0), ref)
+    assert _rel(ns_fp8_scheme(G, F=3), ref) > 2 * bf16
+
+
+def test_fp8_scales_keep_the_copies_finite():
+    # a rank-one input puts all of the norm in one singular value: the bounds are tight there
+    rng = np.random.default_rng(2)
+    G = np.outer(rng.standard_normal(256), rng.standard_normal(512))
+    sx, sa = e4m3_scales()
+    X0 = torch.tensor(G / (np.linalg.norm(G) + 1e-7), dtype=torch.float32)
+    A0 = X0 @ X0.T
+    assert float(A0.abs().max()) * sa[0] <= 448.0
+    X1 = (A_ * torch.eye(256) + B_ * A0 + C_ * A0 @ A0) @ X0
+    assert float(X1.abs().max()) * sx[1] <= 448.0
+    assert float((X1 @ X1.T).abs().max()) * sa[1] <= 448.0
+    assert sx == [256.0, 256.0] and sa == [256.0, 256.0]      # the default coefficients' scales
