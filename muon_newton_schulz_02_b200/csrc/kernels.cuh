@@ -48,6 +48,7 @@ constexpr int kBK8 = 128;           // K per pipeline stage of e4m3 operands: on
 constexpr int kUmmaK8 = 32;         // K of one tcgen05.mma kind::f8f6f4
 constexpr int kTmaps8PerClass = 4;
 constexpr int kMaxFp8Iters = 2;     // e4m3 operands reach at most the first two iterations
+static_assert(kTile == 256 && kBK == 64 && kBK8 == 128, "K-block shifts in ns_gemm_kernel assume these sizes");
 
 enum TmapSlot : int {
   kTmX0 = 0, kTmX1 = 1,             // iterates, 64 x 128 boxes (K-major operand rows, epilogue slices, stores)
@@ -367,9 +368,16 @@ struct Tile {
 // stored before the norm of G is known, so no fixed scale fits it, while every
 // later iterate and Gram matrix is bounded through the singular values (see
 // the host's scales).
+// kFp8 = false (every launch of a bf16 step) compiles the e4m3 paths out.
+template <bool kFp8>
 __device__ __forceinline__ void set_precision(Tile& T, int F) {
-  T.op8 = T.mode == kModePoly ? T.it < F : (T.mode == kModeGram && T.it >= 1 && T.it < F);
-  T.dual = T.mode == kModeGram ? T.it < F : (T.mode == kModeUpdate && !T.fin && T.it + 1 < F);
+  if constexpr (kFp8) {
+    T.op8 = T.mode == kModePoly ? T.it < F : (T.mode == kModeGram && T.it >= 1 && T.it < F);
+    T.dual = T.mode == kModeGram ? T.it < F : (T.mode == kModeUpdate && !T.fin && T.it + 1 < F);
+  } else {
+    T.op8 = 0;
+    T.dual = 0;
+  }
   T.nsub = (T.fin || T.dual) ? 2 : 1;
 }
 
@@ -449,7 +457,7 @@ static_assert(kGemmSmemBytes <= 232448, "more dynamic shared memory than a CTA m
 //     other closely on whichever clusters are free, without a launch
 //     boundary, its operands are still in L2 when they are read, and the
 //     weight update of one matrix overlaps the products of others.
-template <int kMode, bool kFinal, bool kChain>
+template <int kMode, bool kFinal, bool kChain, bool kFp8 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ GemmArgs p) {
   static_assert(!(kChain && kFinal), "the chained launch takes the final update from its items");
   extern __shared__ uint8_t smem_raw[];
@@ -481,7 +489,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       T.mode = kMode; T.fin = kFinal; T.cls = tc.cls; T.b = tc.b; T.tm = tc.tm; T.tn = tc.tn;
       T.x_in = p.x_in; T.first = p.first; T.mat = p.cls[tc.cls].mat_first + tc.b; T.need = 0; T.it = p.iter;
     }
-    set_precision(T, p.fp8_iters);
+    set_precision<kFp8>(T, p.fp8_iters);
     return T;
   };
 
@@ -522,7 +530,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           tmap_acquire(tm);
           tmap_prefetch(tm);
         }
-      if (p.tmaps8)
+      if (kFp8 && p.tmaps8)
         for (int c = 0; c < p.nclasses; ++c)
           for (int k = kTm8X; k <= kTm8A; ++k) {
             const CUtensorMap* tm = &p.tmaps8[c * kTmaps8PerClass + k];
@@ -556,9 +564,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         // stage, read K-major or (blocks below the diagonal) MN-major from one map
         const CUtensorMap* t8 = T.op8 ? &p.tmaps8[T.cls * kTmaps8PerClass + (T.mode == kModeGram ? kTm8X : kTm8A)]
                                       : nullptr;
-        const int bk = T.op8 ? kBK8 : kBK;
-        const int kbpb = kTile / bk;                          // K-blocks per 256-block
-        const int kblocks = (T.mode == kModeGram ? C.lp : C.kp) / bk;
+        const int kbsh = T.op8 ? 1 : 2;                       // K-block kb lies in 256-block kb >> kbsh
+        const int kblocks = (T.mode == kModeGram ? C.lp : C.kp) >> (8 - kbsh);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, wc, kDevTimeoutEmpty)) { ok = false; break; }
           uint8_t* sa = stage_base + stage * kStageBytes;
@@ -568,8 +575,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           // on a diagonal tile of the symmetric phases a CTA's A rows are its B
           // rows: load them once, the MMA reads both operands from the A buffer
           const bool same_ab = sym && T.tm == T.tn;
-          const bool a_below = T.mode != kModeGram && T.tm > kb / kbpb;
-          const bool b_mn = T.mode == kModeUpdate || (T.mode == kModePoly && T.tn > kb / kbpb);
+          const bool a_below = T.mode != kModeGram && T.tm > (kb >> kbsh);
+          const bool b_mn = T.mode == kModeUpdate || (T.mode == kModePoly && T.tn > (kb >> kbsh));
           if (!inject_skip && T.op8) {
             if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], same_ab ? 2 * kStageABytes : 2 * kStageBytes);
             if (a_below) tma_load_3d_pair(sa, t8, full_lead, arow, kb * kBK8, T.b);
@@ -619,9 +626,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         if (!mbar_wait_cluster(&ctl->tmem_empty[acc], acc_phase ^ 1u, wc, kDevTimeoutAccum)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
-        const int bk = T.op8 ? kBK8 : kBK;
-        const int kbpb = kTile / bk;
-        const int kblocks = (T.mode == kModeGram ? C.lp : C.kp) / bk;
+        const int kbsh = T.op8 ? 1 : 2;
+        const int kblocks = (T.mode == kModeGram ? C.lp : C.kp) >> (8 - kbsh);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&ctl->full[stage], phase, wc, kDevTimeoutFull)) { ok = false; break; }
           tc_fence_after();
@@ -630,9 +636,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           // share one operand buffer, blocks below the diagonal arrive MN-major
           const bool same_ab = sym && T.tm == T.tn;
           const uint32_t sb = same_ab ? sa : sa + kStageABytes;
-          const uint32_t a_mn = (T.mode != kModeGram && T.tm > kb / kbpb) ? 1u : 0u;
+          const uint32_t a_mn = (T.mode != kModeGram && T.tm > (kb >> kbsh)) ? 1u : 0u;
           const uint32_t b_mn = same_ab ? a_mn
-                                : (T.mode == kModeUpdate || (T.mode == kModePoly && T.tn > kb / kbpb)) ? 1u : 0u;
+                                : (T.mode == kModeUpdate || (T.mode == kModePoly && T.tn > (kb >> kbsh))) ? 1u : 0u;
           if (T.op8) {
             // 128 MN bytes per CTA: one swizzle atom wide, so only the K stride (SBO) matters MN-major
             const uint32_t idesc = idesc_e4m3_f32(2 * kBM, kBN, a_mn, b_mn);
@@ -675,7 +681,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     if (lane == 0) {
       for (int c = 0; c < p.nclasses; ++c)
         for (int k = 0; k < kTmapsPerClass; ++k) tmap_acquire(&p.tmaps[p.cls[c].tmap_base + k]);
-      if (p.tmaps8)
+      if (kFp8 && p.tmaps8)
         for (int c = 0; c < p.nclasses; ++c)
           for (int k = kTm8Xs; k <= kTm8As; ++k) tmap_acquire(&p.tmaps8[c * kTmaps8PerClass + k]);
       if (p.final_apply)

@@ -494,13 +494,22 @@ cudaError_t launch_gemm(cudaStream_t stream, const GemmArgs& args, int sm_count,
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (chain_clusters > 0) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false, true>, args);
+  // e4m3 instantiations only for launches that use them (the last update never does)
+  const bool f8 = args.fp8_iters > 0 && (chain_clusters > 0 || args.iter < args.fp8_iters);
+  if (chain_clusters > 0)
+    return f8 ? cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false, true, true>, args)
+              : cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false, true>, args);
   switch (args.mode) {
-    case kModeGram: return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false, false>, args);
-    case kModePoly: return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModePoly, false, false>, args);
+    case kModeGram:
+      return f8 ? cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false, false, true>, args)
+                : cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false, false>, args);
+    case kModePoly:
+      return f8 ? cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModePoly, false, false, true>, args)
+                : cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModePoly, false, false>, args);
     default:
-      return args.final_apply ? cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeUpdate, true, false>, args)
-                              : cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeUpdate, false, false>, args);
+      if (args.final_apply) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeUpdate, true, false>, args);
+      return f8 ? cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeUpdate, false, false, true>, args)
+                : cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeUpdate, false, false>, args);
   }
 }
 
@@ -562,6 +571,14 @@ int device_setup(int dev) {
                                 (int)kGemmSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kGemmSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false, false, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModePoly, false, false, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeUpdate, false, false, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false, true, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
   {
     // The chained launch's clusters wait on one another's results, so all of
     // them must be resident at once: never launch more than the device holds.
@@ -576,12 +593,15 @@ int device_setup(int dev) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int nclusters = 0;
+    int nclusters = 0, nclusters8 = 0;      // both instantiations of the chained launch (bf16, e4m3)
     if (cudaOccupancyMaxActiveClusters(&nclusters, (void*)ns_gemm_kernel<kModeGram, false, true>, &cfg) !=
-        cudaSuccess) {
+            cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&nclusters8, (void*)ns_gemm_kernel<kModeGram, false, true, true>, &cfg) !=
+            cudaSuccess) {
       cudaGetLastError();
       nclusters = 0;                         // chained launch unavailable: one launch per phase
     }
+    nclusters = std::min(nclusters, nclusters8);
     g_chain_clusters[dev] = std::min(nclusters, prop.multiProcessorCount / 2);
   }
   g_dev_ready[dev] = true;
