@@ -269,8 +269,9 @@ def workload_config(w, args, sharded=False):
     return {"workload": w.name, "matrices": w.n_matrices, "shapes": shapes, "ns_steps": 5,
             "mu": w.mu, "lr": w.lr, "nesterov": True, "grad_sets": args.grad_sets,
             "l2": f"inputs larger than L2: W, g, buf are {w.n_elements * 12 / 1e9:.2f} GB per step",
-            "parallelism": (f"matrices sharded over {args.gpus} ranks + all_gather in {args.buckets} run(s)"
-                            if sharded else f"independent replicas x{args.gpus}")}
+            "parallelism": (f"matrices sharded over {args.gpus} ranks + all_gather of "
+                            f"{'the bf16 update' if args.exchange == 'o16' else 'the fp32 weights'} in "
+                            f"{args.buckets} run(s)" if sharded else f"independent replicas x{args.gpus}")}
 
 
 def pick_peak(peaks, clk, timed_s):
@@ -411,7 +412,8 @@ def run_ours(args):
 
     def one_step(s):
         if sharded:
-            mdist.sharded_step(W, gsets[s % args.grad_sets], bufs, lr=w.lr, mu=w.mu, nbuckets=args.buckets)
+            mdist.sharded_step(W, gsets[s % args.grad_sets], bufs, lr=w.lr, mu=w.mu, nbuckets=args.buckets,
+                               exchange=args.exchange)
         else:
             stepper(gsets[s % args.grad_sets], stream=stream)
 
@@ -631,6 +633,8 @@ def main():
                     help="seconds of single-threaded CPU oracle work (cpu_baseline.one_core)")
     ap.add_argument("--buckets", type=int, default=2,
                     help="with --sharded: runs per rank whose all_gather overlaps the next run's step")
+    ap.add_argument("--exchange", choices=("w32", "o16"), default="w32",
+                    help="sharded step: all_gather the updated fp32 weights, or the bf16 update (every rank applies)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -126,6 +126,37 @@ int muon_step_fp8(float* const* params, const float* const* grads, float* const*
                   float eps, int nesterov, int fp8_iters, void* stream);
 
 /*
+ * The two halves of a Muon step for a data-parallel run that exchanges the
+ * orthogonalised update in bf16 instead of the fp32 weights (half the bytes
+ * on the interconnect; the speedrun of the Modded-NanoGPT article trains on 8
+ * GPUs).  Every rank computes O for the matrices it owns with
+ * muon_update_bf16, the ranks all-gather the bf16 O, and every rank applies
+ * all of them with muon_apply_bf16, so that every replica of W receives the
+ * same update.  (A deployment variant: the article has no exchange.)
+ *
+ * muon_update_bf16: momentum and NS5 as in muon_step_ex, W untouched.
+ *   grads[i]         in      g_i (fp32, m x n), read only.
+ *   momentum_bufs[i] in/out  buf_i, updated in place as by muon_step_ex.
+ *   O[i]             out     NS5(G_i) rounded to bf16 (round to nearest
+ *                            even), m x n row-major, 2-byte bf16 bit
+ *                            patterns, caller-owned device memory.
+ * The update goes through a library-held fp32 scratch of sum(m*n) floats
+ * (allocated by the first call that needs it, freed by muon_release) before
+ * its rounding to bf16.
+ */
+int muon_update_bf16(const float* const* grads, float* const* momentum_bufs, uint16_t* const* O,
+                     const int64_t* shapes, int n, float mu, int ns_steps, float a, float b, float c,
+                     float eps, int nesterov, void* stream);
+
+/*
+ * muon_apply_bf16: W_i <- W_i - lr * O_i for bf16 O_i (m x n row-major,
+ * 2-byte bf16 bit patterns, read only), one fused multiply-add in fp32 per
+ * element.  params[i] in/out: W_i, updated in place.
+ */
+int muon_apply_bf16(float* const* params, const uint16_t* const* O, const int64_t* shapes, int n, float lr,
+                    void* stream);
+
+/*
  * NS5 alone (the zeroth_power_via_newtonschulz5 listing): O_i = NS5(G_i)
  * with the listing's defaults and `ns_steps` iterations.  G_i is read only,
  * O_i (m x n fp32, caller-owned device memory) is overwritten.
@@ -212,7 +243,8 @@ void muon_release(void);
 #define MUON_KIND_SMALL 6        /* fused single-CTA step of small matrices */
 #define MUON_KIND_PAIR 7         /* fused CTA-pair step, 128 < short side <= 256, long side <= 256 */
 #define MUON_KIND_CHAIN 8        /* every Newton-Schulz phase and the weight update, one chained launch */
-#define MUON_NUM_KINDS 9
+#define MUON_KIND_O16 9          /* bf16 update exchange: fp32 -> bf16 rounding of O, or W -= lr * O */
+#define MUON_NUM_KINDS 10
 
 /* 1: bracket every kernel launch with CUDA events on its stream; 0: stop. */
 int muon_profile_enable(int enable);

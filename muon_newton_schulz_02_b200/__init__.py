@@ -21,6 +21,7 @@ from array import array
 __all__ = [
     "step", "PreparedStep", "orthogonalize", "step_host", "step_noalloc", "workspace_size", "sync_status", "last_error", "release",
     "profile_enable", "profile_read", "launch_count", "chain_clusters", "debug_set", "chain_plan", "lib", "MuonError", "KINDS",
+    "update_bf16", "apply_bf16",
     "NS_A", "NS_B", "NS_C", "NS_STEPS", "NS_EPS", "LIB_PATH", "header_functions",
 ]
 
@@ -29,7 +30,7 @@ LIB_PATH = os.path.join(HERE, "libmuon_b200.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "muon.h")
 
 NS_A, NS_B, NS_C, NS_STEPS, NS_EPS = 3.4445, -4.7750, 2.0315, 5, 1e-7
-KINDS = ("prologue", "gram", "poly", "update", "update_apply", "apply_x0", "small", "pair", "chain")
+KINDS = ("prologue", "gram", "poly", "update", "update_apply", "apply_x0", "small", "pair", "chain", "o16")
 
 STATUS = {0: "MUON_OK", -1: "MUON_ERR_INVALID_ARG", -2: "MUON_ERR_SHAPE", -3: "MUON_ERR_CUDA",
           -4: "MUON_ERR_NOMEM", -5: "MUON_ERR_TIMEOUT", -6: "MUON_ERR_DEVICE", -7: "MUON_ERR_UNSUPPORTED"}
@@ -74,6 +75,11 @@ def lib() -> ctypes.CDLL:
     L.muon_step_host.restype = ctypes.c_int
     L.muon_step_noalloc.argtypes = step_args + [_P]
     L.muon_step_noalloc.restype = ctypes.c_int
+    L.muon_update_bf16.argtypes = [_PP, _PP, _PP, _I64P, ctypes.c_int, ctypes.c_float, ctypes.c_int] + \
+        [ctypes.c_float] * 4 + [ctypes.c_int, _P]
+    L.muon_update_bf16.restype = ctypes.c_int
+    L.muon_apply_bf16.argtypes = [_PP, _PP, _I64P, ctypes.c_int, ctypes.c_float, _P]
+    L.muon_apply_bf16.restype = ctypes.c_int
     L.muon_orthogonalize.argtypes = [_PP, _PP, _I64P, ctypes.c_int, ctypes.c_int, _P]
     L.muon_orthogonalize.restype = ctypes.c_int
     L.muon_workspace_size.argtypes = [_I64P, ctypes.c_int]
@@ -124,28 +130,30 @@ def _stream(stream):
     return ctypes.c_void_p(int(stream))
 
 
-def _bad(name, i, t, device_kind):
+def _bad(name, i, t, device_kind, dtype=None):
     """The error for a tensor that failed the quick check (slow path, only on failure)."""
     import torch
+    dtype = dtype or torch.float32
     if t.dim() != 2:
         return ValueError(f"{name}[{i}] must be 2-D (the method is defined for matrices)")
-    if t.dtype != torch.float32 or not t.is_contiguous():
-        return ValueError(f"{name}[{i}] must be contiguous float32")
+    if t.dtype != dtype or not t.is_contiguous():
+        return ValueError(f"{name}[{i}] must be contiguous {str(dtype).replace('torch.', '')}")
     return ValueError(f"{name}[{i}] must live on {device_kind}")
 
 
-def _marshal(name, ts, device_kind="cuda", shapes=None):
-    """One pass over a tensor list: checks (2-D, contiguous fp32, device kind
-    -- for CUDA, the current device, where the library launches -- and equal
-    shapes to `shapes` when given) and returns (pointer array, list of
-    shapes).  The arrays are ctypes views of array('q') buffers."""
+def _marshal(name, ts, device_kind="cuda", shapes=None, dtype=None):
+    """One pass over a tensor list: checks (2-D, contiguous, of `dtype` --
+    fp32 by default -- on the device kind -- for CUDA, the current device,
+    where the library launches -- and equal shapes to `shapes` when given)
+    and returns (pointer array, list of shapes).  The arrays are ctypes
+    views of array('q') buffers."""
     import torch
-    f32, on_cuda = torch.float32, device_kind == "cuda"
+    f32, on_cuda = dtype or torch.float32, device_kind == "cuda"
     dev = None
     ptrs, shp = array("q"), []
     for i, t in enumerate(ts):
         if t.dtype is not f32 or t.is_cuda is not on_cuda or not t.is_contiguous() or t.dim() != 2:
-            raise _bad(name, i, t, device_kind)
+            raise _bad(name, i, t, device_kind, f32)
         if on_cuda:
             if dev is None:
                 dev = torch.cuda.current_device()
@@ -227,6 +235,39 @@ class PreparedStep:
             rc = lib().muon_step_ex(self._pp, gp, self._bp, self._sh, self.n, lr, self.mu, self.ns_steps,
                                     *self._abc, _stream(stream))
         _check(rc)
+
+
+def update_bf16(grads, bufs, mu: float, ns_steps: int = NS_STEPS, O=None, *, a: float = NS_A, b: float = NS_B,
+                c: float = NS_C, eps: float = NS_EPS, nesterov: bool = True, stream=None):
+    """Momentum and NS5 without the weight update: returns the orthogonalised
+    updates O_i as CUDA bfloat16 matrices (written into ``O`` when given) and
+    updates ``bufs`` in place.  With :func:`apply_bf16`, the two halves of a
+    step whose update is exchanged in bf16 between data-parallel ranks."""
+    import torch
+    n = len(grads)
+    if len(bufs) != n or n == 0:
+        raise ValueError("grads and bufs must be equally long, non-empty lists")
+    gp, shp = _marshal("grads", grads)
+    bp, _ = _marshal("bufs", bufs, shapes=shp)
+    if O is None:
+        O = [torch.empty(s, dtype=torch.bfloat16, device=g.device) for s, g in zip(shp, grads)]
+    if len(O) != n:
+        raise ValueError("O must have one matrix per gradient")
+    op, _ = _marshal("O", O, shapes=shp, dtype=torch.bfloat16)
+    rc = lib().muon_update_bf16(gp, bp, op, _shape_array(shp), n, float(mu), int(ns_steps), float(a), float(b),
+                                float(c), float(eps), 1 if nesterov else 0, _stream(stream))
+    _check(rc)
+    return O
+
+
+def apply_bf16(params, O, lr: float, stream=None):
+    """W_i -= lr * O_i for CUDA fp32 ``params`` and bfloat16 ``O`` (in place)."""
+    import torch
+    if len(params) != len(O) or not params:
+        raise ValueError("params and O must be equally long, non-empty lists")
+    pp, shp = _marshal("params", params)
+    op, _ = _marshal("O", O, shapes=shp, dtype=torch.bfloat16)
+    _check(lib().muon_apply_bf16(pp, op, _shape_array(shp), len(params), float(lr), _stream(stream)))
 
 
 def orthogonalize(G, O=None, ns_steps: int = NS_STEPS, stream=None):

@@ -1807,6 +1807,61 @@ __global__ void __launch_bounds__(kPairThreads, 1) ns_pair_kernel(const __grid_c
   }
 }
 
+// ==================================================== bf16 update exchange ===
+// For a data-parallel step that exchanges the orthogonalised update O in bf16
+// (half the bytes of fp32 weights): `convert` rounds O (fp32, written by a
+// step in assign mode) to bf16; `apply` adds -lr * O (bf16) into W.  One CTA
+// row per matrix, grid-stride over its elements, 8 elements per thread and
+// iteration where both pointers are 16-byte aligned and the count is a
+// multiple of 8.
+struct O16Args {
+  int nmats, apply;
+  float lr;
+  const float* src[kMaxMats];      // convert: O in fp32
+  __nv_bfloat16* o16[kMaxMats];    // convert: destination; apply: O in bf16 (read only)
+  float* w[kMaxMats];              // apply: W, updated in place
+  long long count[kMaxMats];
+  int vec[kMaxMats];
+};
+
+__global__ void o16_kernel(const __grid_constant__ O16Args p) {
+  griddep_wait();
+  const int mi = blockIdx.y;
+  if (mi >= p.nmats) return;
+  const long long n = p.count[mi];
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  const long long t0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  __nv_bfloat16* o = p.o16[mi];
+  if (p.vec[mi]) {
+    for (long long e = t0 * 8; e < n; e += stride * 8) {
+      if (!p.apply) {
+        const float4 a = *reinterpret_cast<const float4*>(p.src[mi] + e);
+        const float4 b = *reinterpret_cast<const float4*>(p.src[mi] + e + 4);
+        *reinterpret_cast<uint4*>(o + e) = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w),
+                                                      pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+      } else {
+        const uint4 raw = *reinterpret_cast<const uint4*>(o + e);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        float4* wp = reinterpret_cast<float4*>(p.w[mi] + e);
+        float4 a = wp[0], b = wp[1];
+        const float2 h0 = __bfloat1622float2(h[0]), h1 = __bfloat1622float2(h[1]);
+        const float2 h2 = __bfloat1622float2(h[2]), h3 = __bfloat1622float2(h[3]);
+        a.x = fmaf(-p.lr, h0.x, a.x); a.y = fmaf(-p.lr, h0.y, a.y);
+        a.z = fmaf(-p.lr, h1.x, a.z); a.w = fmaf(-p.lr, h1.y, a.w);
+        b.x = fmaf(-p.lr, h2.x, b.x); b.y = fmaf(-p.lr, h2.y, b.y);
+        b.z = fmaf(-p.lr, h3.x, b.z); b.w = fmaf(-p.lr, h3.y, b.w);
+        wp[0] = a;
+        wp[1] = b;
+      }
+    }
+  } else {
+    for (long long e = t0; e < n; e += stride) {
+      if (!p.apply) o[e] = __float2bfloat16_rn(p.src[mi][e]);
+      else p.w[mi][e] = fmaf(-p.lr, __bfloat162float(o[e]), p.w[mi][e]);
+    }
+  }
+}
+
 // ======================================================= ns_steps == 0 ===
 __global__ void apply_x0_kernel(const __grid_constant__ ApplyArgs p) {
   griddep_wait();

@@ -540,6 +540,8 @@ struct Ctx {
   int* status_h = nullptr;
   int* status_d = nullptr;
   float* stage = nullptr;                   // device staging of muon_step_host
+  float* o32 = nullptr;                     // fp32 O of muon_update_bf16 before its rounding to bf16
+  size_t o32_cap = 0;
   size_t stage_cap = 0;
   std::vector<ProfRec> prof;
   std::vector<cudaEvent_t> event_pool;
@@ -744,7 +746,7 @@ cudaEvent_t pool_event(Ctx& c) {
 // ranges cost nothing when no tool is attached.
 const char* const kKindNames[MUON_NUM_KINDS] = {"muon.prologue", "muon.gram", "muon.poly", "muon.update",
                                                 "muon.update_apply", "muon.apply_x0", "muon.small", "muon.pair",
-                                                "muon.chain"};
+                                                "muon.chain", "muon.o16"};
 
 template <class F>
 int launch(Ctx& c, int kind, F&& f) {
@@ -1144,10 +1146,91 @@ int step_impl(const StepIO& io, const int64_t* shapes, int n, void* stream) {
   return MUON_OK;
 }
 
+// One launch of o16_kernel per kMaxMats matrices: apply = 0 rounds src (fp32)
+// into o16, apply = 1 adds -lr * o16 into w.
+int run_o16(Ctx& c, int apply, float lr, const float* const* src, __nv_bfloat16* const* o16, float* const* w,
+            const int64_t* shapes, int n) {
+  for (int base = 0; base < n; base += kMaxMats) {
+    const int nm = std::min(kMaxMats, n - base);
+    auto oa = std::make_unique<O16Args>();
+    std::memset(oa.get(), 0, sizeof(O16Args));
+    oa->nmats = nm;
+    oa->apply = apply;
+    oa->lr = lr;
+    long long most = 0;
+    for (int i = 0; i < nm; ++i) {
+      const int u = base + i;
+      const long long cnt = (long long)shapes[2 * u] * shapes[2 * u + 1];
+      oa->count[i] = cnt;
+      oa->o16[i] = o16[u];
+      if (apply) oa->w[i] = w[u]; else oa->src[i] = src[u];
+      oa->vec[i] = cnt % 8 == 0 && aligned16(o16[u]) && aligned16(apply ? (const void*)w[u] : (const void*)src[u]);
+      most = std::max(most, cnt);
+    }
+    // about 8 elements per thread per pass, and some 1200 CTAs over the launch
+    const long long want = (most + 2047) / 2048;
+    const int gx = (int)std::max<long long>(1, std::min<long long>(want, std::max(4, 1184 / nm)));
+    int rc = launch(c, MUON_KIND_O16,
+                    [&] { launch_pdl(o16_kernel, dim3(gx, nm), dim3(256), 0, c.stream, *oa); });
+    if (rc) return rc;
+  }
+  return MUON_OK;
+}
+
 }  // namespace
 
 // =================================================================== C ABI ===
 extern "C" {
+
+int muon_update_bf16(const float* const* grads, float* const* momentum_bufs, uint16_t* const* O, const int64_t* shapes,
+                     int n, float mu, int ns_steps, float a, float b, float c, float eps, int nesterov, void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int rc = validate_common(shapes, n, ns_steps);
+  if (rc) return rc;
+  if ((rc = validate_ptrs((const void* const*)grads, n, "grads"))) return rc;
+  if ((rc = validate_ptrs((const void* const*)momentum_bufs, n, "momentum_bufs"))) return rc;
+  if ((rc = validate_ptrs((const void* const*)O, n, "O"))) return rc;
+  if (nesterov != 0 && nesterov != 1) return fail(MUON_ERR_INVALID_ARG, "nesterov must be 0 or 1");
+  if (!(eps >= 0.f)) return fail(MUON_ERR_INVALID_ARG, "eps must be >= 0");
+  Ctx* ctx = nullptr;
+  if ((rc = get_ctx(stream, &ctx))) return rc;
+  std::vector<size_t> off(n);
+  size_t total = 0;
+  for (int i = 0; i < n; ++i) {
+    off[i] = total;
+    total += align_up((size_t)(shapes[2 * i] * shapes[2 * i + 1]), 64);
+  }
+  if (ctx->o32_cap < total) {
+    CUDA_TRY(cudaStreamSynchronize(ctx->stream));
+    if (ctx->o32) cudaFree(ctx->o32);
+    ctx->o32 = nullptr;
+    ctx->o32_cap = 0;
+    if (cudaMalloc((void**)&ctx->o32, total * sizeof(float)) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(MUON_ERR_NOMEM, "fp32 update scratch allocation failed");
+    }
+    ctx->o32_cap = total;
+  }
+  std::vector<float*> o32(n);
+  for (int i = 0; i < n; ++i) o32[i] = ctx->o32 + off[i];
+  // the step in assign mode writes O (fp32) where it would update W
+  StepIO io{o32.data(), grads, momentum_bufs, 0.f, mu, a, b, c, eps, ns_steps, nesterov, 1};
+  if ((rc = step_impl(io, shapes, n, stream))) return rc;
+  return run_o16(*ctx, 0, 0.f, o32.data(), (__nv_bfloat16* const*)O, nullptr, shapes, n);
+}
+
+int muon_apply_bf16(float* const* params, const uint16_t* const* O, const int64_t* shapes, int n, float lr,
+                    void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int rc = validate_common(shapes, n, 0);
+  if (rc) return rc;
+  if ((rc = validate_ptrs((const void* const*)params, n, "params"))) return rc;
+  if ((rc = validate_ptrs((const void* const*)O, n, "O"))) return rc;
+  Ctx* ctx = nullptr;
+  if ((rc = get_ctx(stream, &ctx))) return rc;
+  if ((rc = check_status(*ctx))) return rc;
+  return run_o16(*ctx, 1, lr, nullptr, (__nv_bfloat16* const*)O, params, shapes, n);
+}
 
 int muon_step_ex(float* const* params, const float* const* grads, float* const* momentum_bufs,
                  const int64_t* shapes, int n, float lr, float mu, int ns_steps,
@@ -1320,6 +1403,7 @@ void muon_release(void) {
     cudaStreamSynchronize(c.stream);
     if (c.ws) cudaFree(c.ws);
     if (c.stage) cudaFree(c.stage);
+    if (c.o32) cudaFree(c.o32);
     if (c.status_h) cudaFreeHost(c.status_h);
     for (auto& r : c.prof) { cudaEventDestroy(r.a); cudaEventDestroy(r.b); }
     for (auto e : c.event_pool) cudaEventDestroy(e);

@@ -97,3 +97,57 @@ def test_sharded_step_matches_single_process(world, nbuckets):
             assert np.array_equal(W[i], W_ref[i].numpy()), (rank, i)   # every rank has every update
         for i in owned[rank]:
             assert np.array_equal(b[i], b_ref[i].numpy()), (rank, i)   # own momentum updated
+
+
+# ---- the bf16-update exchange: the owner computes O, every rank applies it --
+def _oracle_local_update(grads, bufs, O, mu, ns_steps):
+    from oracle import muon_oracle
+    for g, b, o in zip(grads, bufs, O):
+        b_new, G = muon_oracle.momentum_update(g.numpy(), b.numpy(), mu)
+        o.copy_(torch.from_numpy(muon_oracle.newton_schulz5(G, steps=ns_steps)).to(torch.bfloat16))
+        b.copy_(torch.from_numpy(b_new))
+
+
+def _cpu_apply(params, O, lr):
+    for W, o in zip(params, O):
+        W.sub_(o.float() * lr)
+
+
+def _worker_o16(rank, world, port, shapes, q, nbuckets):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        W, g, b = _inputs(shapes=shapes)
+        owned = mdist.sharded_step(W, g, b, lr=0.02, mu=0.95, nbuckets=nbuckets, exchange="o16",
+                                   local_update=_oracle_local_update, local_apply=_cpu_apply)
+        q.put((rank, [w.numpy() for w in W], [x.numpy() for x in b], owned))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,nbuckets", [(2, 1), (3, 2)])
+def test_bf16_update_exchange_gives_every_rank_the_same_weights(world, nbuckets):
+    shapes = SHAPES[4:]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_o16, args=(r, world, port, shapes, q, nbuckets)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=300) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # one process doing the same: update every matrix, then apply every bf16 O
+    W_ref, g_ref, b_ref = _inputs(shapes=shapes)
+    O = [torch.empty(s, dtype=torch.bfloat16) for s in shapes]
+    _oracle_local_update(g_ref, b_ref, O, 0.95, 5)
+    _cpu_apply(W_ref, O, 0.02)
+    for rank, W, b, owned in results:
+        for i in range(len(shapes)):
+            assert np.array_equal(W[i], W_ref[i].numpy()), (rank, i)
+        for i in owned[rank]:
+            assert np.array_equal(b[i], b_ref[i].numpy()), (rank, i)
+    with pytest.raises(ValueError):
+        mdist.sharded_step(W_ref, g_ref, b_ref, 0.02, 0.95, exchange="fp8")

@@ -97,3 +97,70 @@ def test_sharded_step_with_the_cuda_step_on_two_ranks(nbuckets):
         owner = [r for r in range(2) if i in partition[r]][0]
         b_owner = [b for r, _, b, _ in results if r == owner][0]
         assert relF(b_owner[i], b_ref) <= REL_BUF
+
+
+# ---- the bf16-update exchange with the CUDA library's two halves -----------
+def _cuda_local_update(grads, bufs, O, mu, ns_steps):
+    import muon_newton_schulz_02_b200 as muon
+    dev = torch.device("cuda:0")
+    gd = [x.to(dev) for x in grads]
+    bd = [x.to(dev) for x in bufs]
+    Od = [torch.empty(o.shape, dtype=torch.bfloat16, device=dev) for o in O]
+    muon.update_bf16(gd, bd, mu, ns_steps=ns_steps, O=Od)
+    torch.cuda.synchronize()
+    assert muon.sync_status() == 0, muon.last_error()
+    for h, d in zip(bufs + O, bd + Od):
+        h.copy_(d.cpu())
+
+
+def _cuda_apply(params, O, lr):
+    import muon_newton_schulz_02_b200 as muon
+    dev = torch.device("cuda:0")
+    Wd = [x.to(dev) for x in params]
+    muon.apply_bf16(Wd, [o.to(dev) for o in O], lr)
+    torch.cuda.synchronize()
+    for h, d in zip(params, Wd):
+        h.copy_(d.cpu())
+
+
+def _worker_o16(rank, world, port, q):
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from muon_newton_schulz_02_b200 import distributed as mdist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        W, g, b = _inputs()
+        owned = mdist.sharded_step(W, g, b, lr=0.02, mu=0.95, nbuckets=2, exchange="o16",
+                                   local_update=_cuda_local_update, local_apply=_cuda_apply)
+        q.put((rank, [w.numpy() for w in W], [x.numpy() for x in b], owned))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bf16_update_exchange_with_the_cuda_halves_on_two_ranks():
+    import __graft_entry__
+    __graft_entry__.build()
+    from oracle import muon_oracle
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_o16, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=600) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    W0, g0, b0 = _inputs()
+    partition = results[0][3]
+    for i in range(len(SHAPES)):
+        assert np.array_equal(results[0][1][i], results[1][1][i]), i      # identical replicas
+    for i in range(len(SHAPES)):
+        W_ref, b_ref, O_ref = muon_oracle.muon_update(W0[i].numpy(), g0[i].numpy(), b0[i].numpy(), 0.02, 0.95)
+        check_o(o_from_w(W0[i].numpy(), results[0][1][i], 0.02), O_ref, f"matrix {i} {SHAPES[i]}")
+        owner = [r for r in range(2) if i in partition[r]][0]
+        b_owner = [b for r, _, b, _ in results if r == owner][0]
+        assert relF(b_owner[i], b_ref) <= REL_BUF
