@@ -278,9 +278,11 @@ int build_layout(const int64_t* shapes, int n, Plan& plan) {
 // update adds -lr*O into W); each phase's tiles may start only once all tiles
 // of the previous phase of that matrix are done.  A simulation of `ncl` clusters
 // assigns tiles greedily: a free cluster takes the next tile of the
-// highest-priority matrix whose current phase is ready (larger matrices first),
-// so a matrix's phases follow each other closely and its operands stay in L2
-// while other matrices fill the gaps.  Tile cost is modelled as its K-blocks
+// highest-priority matrix whose current phase is ready (longest remaining
+// critical path first), so a matrix's phases follow each other closely, its
+// operands stay in L2 while other matrices fill the gaps, and the matrices
+// finish together instead of leaving a tail of dependent phases with too few
+// tiles to keep every cluster busy.  Tile cost is modelled as its K-blocks
 // plus a fixed overhead; a finished tile is visible to dependants `lat` units
 // later (epilogue, store, and the producer running ahead of the MMAs).
 //
@@ -295,6 +297,15 @@ double chain_latency_units() {
     lat = e ? std::max(0.0, std::atof(e)) : 20.0;
   }
   return lat;
+}
+
+bool chain_static_priority() {
+  static int rule = -1;
+  if (rule < 0) {
+    const char* e = std::getenv("MUON_CHAIN_PRIORITY");
+    rule = (e && std::strcmp(e, "static") == 0) ? 1 : 0;
+  }
+  return rule == 1;
 }
 
 void build_chain(const Group& g, int ns_steps, int fp8_iters, int ncl, std::vector<WorkItem>& items,
@@ -338,20 +349,35 @@ void build_chain(const Group& g, int ns_steps, int fp8_iters, int ncl, std::vect
       for (int j = 0; j < nphases; ++j) st.total += st.ntiles[mode_of(j)] * cost_of(st, j);
     }
   }
-  // priority: more total work first (its long chain starts early), then group order
+  // Priority of a matrix whose next phase is ready: by default the longest
+  // remaining critical path (one tile plus the visibility latency per phase
+  // still to run) first, so that the matrices finish together and no long
+  // chain is left alone at the end; "static": more total work first.
   std::vector<int> by_prio(nm);
   for (int i = 0; i < nm; ++i) by_prio[i] = i;
   std::stable_sort(by_prio.begin(), by_prio.end(), [&](int x, int y) { return ms[x].total > ms[y].total; });
   std::vector<int> prio(nm);
   for (int r = 0; r < nm; ++r) prio[by_prio[r]] = r;
+  const bool static_rule = chain_static_priority();
+  std::vector<double> key(nm, 0.0);           // the key a matrix holds while its phase is available
+  auto key_of = [&](int m) {
+    if (static_rule) return (double)prio[m];
+    double path = 0.0;
+    for (int q = ms[m].phase; q < nphases; ++q) path += cost_of(ms[m], q) + lat;
+    return -path;
+  };
 
   std::vector<std::vector<WorkItem>> lists(ncl);
   std::priority_queue<std::pair<double, int>, std::vector<std::pair<double, int>>, std::greater<>> free_at;
   for (int c = 0; c < ncl; ++c) free_at.push({0.0, c});
-  std::set<std::pair<double, int>> pending;   // (ready time, priority) of a matrix's next phase
-  std::set<int> avail;                        // priorities of matrices with ready, unassigned tiles
+  std::set<std::pair<double, int>> pending;   // (ready time, matrix) of a matrix's next phase
+  std::set<std::pair<double, int>> avail;     // (key, matrix): matrices with ready, unassigned tiles, best first
+  auto make_avail = [&](int m) {
+    key[m] = key_of(m);
+    avail.insert({key[m], m});
+  };
   for (int m = 0; m < nm; ++m)
-    if (nphases > 0) avail.insert(prio[m]);
+    if (nphases > 0) make_avail(m);
   long long left = 0;
   for (int m = 0; m < nm; ++m)
     for (int j = 0; j < nphases; ++j) left += ms[m].ntiles[mode_of(j)];
@@ -360,7 +386,7 @@ void build_chain(const Group& g, int ns_steps, int fp8_iters, int ncl, std::vect
     free_at.pop();
     auto admit = [&](double now) {
       while (!pending.empty() && pending.begin()->first <= now) {
-        avail.insert(pending.begin()->second);
+        make_avail(pending.begin()->second);
         pending.erase(pending.begin());
       }
     };
@@ -369,7 +395,7 @@ void build_chain(const Group& g, int ns_steps, int fp8_iters, int ncl, std::vect
       t = std::max(t, pending.begin()->first);
       admit(t);
     }
-    const int m = by_prio[*avail.begin()];
+    const int m = avail.begin()->second;
     MatState& st = ms[m];
     const int mode = mode_of(st.phase);
     int tm, tn;
@@ -397,10 +423,10 @@ void build_chain(const Group& g, int ns_steps, int fp8_iters, int ncl, std::vect
     free_at.push({end, c});
     --left;
     if (++st.next == st.ntiles[mode]) {       // phase fully assigned: the next one is ready at st.vis
-      avail.erase(prio[m]);
+      avail.erase({key[m], m});
       st.need += 2 * st.ntiles[mode];
       st.next = 0;
-      if (++st.phase < nphases) pending.insert({st.vis, prio[m]});
+      if (++st.phase < nphases) pending.insert({st.vis, m});
       st.vis = 0.0;
     }
   }

@@ -78,15 +78,21 @@ def test_lists_cover_every_tile_once_and_cannot_deadlock(name, ns_steps, ncluste
     assert heads == off[1:], "the work lists can deadlock"
 
 
-def test_lists_keep_a_matrix_phases_close_together():
-    # The point of the lists: a matrix's phases follow each other instead of
-    # waiting for every other matrix (which a launch per phase forces).  On the
-    # GPT-2-124M set a 768x3072 matrix (the largest, scheduled first) is done
-    # with all its phases before the last 768x768 matrix has started, judged
-    # by the positions of their items in the clusters' lists.
+def test_lists_let_the_matrices_finish_together():
+    # The lists follow the longest remaining critical path first: every matrix
+    # starts early and all of them finish near the end, so the last phases
+    # (few tiles each) of many matrices fill the clusters together instead of
+    # one long chain running alone at the end.  Judged on the GPT-2-124M set by
+    # the positions of the items in the clusters' lists.
     items, off = muon.chain_plan(GPT2, ns_steps=5, nclusters=74)
-    pos = {}
+    first, last = {}, {}
     for c in range(74):
-        for k, it in enumerate(items[off[c]:off[c + 1]]):
-            pos.setdefault(it[1], []).append(k)
-    assert max(pos[48]) < min(pos[47])
+        n = off[c + 1] - off[c]
+        for k, (need, m, cls, b, tm, tn, mode, it) in enumerate(items[off[c]:off[c + 1]]):
+            if it == 0 and mode == 0:
+                first[m] = max(first.get(m, 0.0), k / n)
+            if mode == 3:
+                last[m] = min(last.get(m, 1.0), k / n)
+    assert len(first) == len(last) == len(GPT2)
+    assert max(first.values()) < 0.2          # every matrix's first Gram tiles early in the lists
+    assert min(last.values()) > 0.8           # every matrix's last update late in the lists
