@@ -329,6 +329,28 @@ def gemm_roofline(prof, flops, steps, peak):
             "frac": achieved / peak}
 
 
+def alternate_fp8(args, muon, torch, dev, stream, w, W, bufs, gsets, stepper, blocks, per):
+    """The reduced-precision variant (muon_step_fp8) against the bf16 step on
+    the same workload, in alternating blocks so that both see the same clock
+    and power state; the medians of the block means compare them."""
+    stepper8 = muon.PreparedStep(W, bufs, lr=w.lr, mu=w.mu, fp8_iters=args.fp8_iters)
+    for s in range(2):
+        stepper8(gsets[s % len(gsets)], stream=stream)
+    torch.cuda.synchronize(dev)
+    timer = StepTimer(torch, stream)
+    t16, t8 = [], []
+    for _ in range(blocks):
+        for st_, acc in ((stepper, t16), (stepper8, t8)):
+            e = timer.run(lambda s: st_(gsets[s % len(gsets)], stream=stream), per)
+            torch.cuda.synchronize(dev)
+            acc.append(timer.times(e)[0] / per)
+    m16, m8 = statistics.median(t16), statistics.median(t8)
+    return {"fp8_iters": args.fp8_iters, "ms_per_step": m8, "ms_per_step_bf16": m16, "speedup": m16 / m8,
+            "protocol": f"{blocks} alternating blocks of {per} bf16 and {per} e4m3 steps, medians of block means",
+            "what": "muon_step_fp8: e4m3 operands for A*A (iterations 0..F-1) and X*X^T (1..F-1) in the "
+                    "per-phase launches; a reduced-precision variant, not the headline"}
+
+
 def run_sweep(args, muon, workloads, torch, dev, stream, peaks):
     """GEMM-kernel throughput on the 64-matrix square batches, each timed on
     its own (>= 3 warm-up and >= 5 timed steps, every launch bracketed by
@@ -368,6 +390,9 @@ def run_sweep(args, muon, workloads, torch, dev, stream, peaks):
             entry["gemm_frac_sustained"] = r["achieved"] / float(peaks["bf16_tflops_sustained"])
         if r and clk:
             entry["gemm_kcycles_per_launch"] = r["us_per_launch"] * clk["sm_mhz"] / 1e3
+        if args.fp8_iters and n > 1024:
+            entry["fp8_variant"] = alternate_fp8(args, muon, torch, dev, stream, w, W, bufs, gsets, stepper,
+                                                 blocks=2, per=2)
         out[f"n{n}"] = entry
         if muon.sync_status(stream) != 0:
             raise RuntimeError(f"device status after the n={n} sweep entry: " + muon.last_error())
@@ -469,28 +494,6 @@ def run_ours(args):
         del flush
     # ---- the reduced-precision variant (muon_step_fp8) on the same workload,
     # timed the same way; reported beside the bf16 line, never as its value
-    fp8 = None
-    if args.fp8_iters and not sharded:
-        # alternating blocks of bf16 and e4m3 steps, so that both see the same
-        # clock and power state; the medians of the per-block times compare them
-        stepper8 = muon.PreparedStep(W, bufs, lr=w.lr, mu=w.mu, fp8_iters=args.fp8_iters)
-        for s in range(3):
-            stepper8(gsets[s % args.grad_sets], stream=stream)
-        barrier()
-        torch.cuda.synchronize(dev)
-        blocks, per = 4, max(2, args.steps // 4)
-        t16, t8 = [], []
-        for _ in range(blocks):
-            for st_, acc in ((stepper, t16), (stepper8, t8)):
-                e = timer.run(lambda s: st_(gsets[s % args.grad_sets], stream=stream), per)
-                torch.cuda.synchronize(dev)
-                acc.append(timer.times(e)[0] / per)
-        m16, m8 = statistics.median(t16), statistics.median(t8)
-        fp8 = {"fp8_iters": args.fp8_iters, "ms_per_step": m8, "ms_per_step_bf16": m16, "speedup": m16 / m8,
-               "protocol": f"{blocks} alternating blocks of {per} bf16 and {per} e4m3 steps, medians of block means",
-               "what": "muon_step_fp8: e4m3 operands for A*A (iterations 0..F-1) and X*X^T (1..F-1); "
-                       "a reduced-precision variant, not the headline"}
-        del stepper8
     if muon.sync_status(stream) != 0:
         raise RuntimeError("device status after timing: " + muon.last_error())
     ms_max = mdist.max_over_ranks(ms, device=dev)
@@ -601,7 +604,6 @@ def run_ours(args):
                        "cold_l2": "a 1 GiB buffer is written before each cold step (evicts the 126 MB L2)"},
         "kernels": kinds,
         "sweep": sweep,
-        "fp8_variant": fp8,
         "frac_of_dense_peak": value / world / burst,
         "frac_of_dense_spec": value / world / 2250.0,
         "peaks": {"source": peak_src, "bf16_tflops": peaks.get("bf16_tflops"),
@@ -626,7 +628,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-events", type=int, default=1, help="per-launch CUDA events in a second timed pass")
     ap.add_argument("--fp8-iters", type=int, default=2,
-                    help="also time muon_step_fp8 with this many e4m3 iterations (0: skip)")
+                    help="also time muon_step_fp8 (this many e4m3 iterations; 0: skip) beside the bf16 step on "
+                         "the sweep's sizes above 1024, where it applies")
     ap.add_argument("--replicas", action="store_true",
                     help="under torchrun: an independent copy of the workload per rank instead of the sharded step")
     ap.add_argument("--per-phase", action="store_true",

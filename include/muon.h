@@ -113,9 +113,13 @@ int muon_step_ex(float* const* params, const float* const* grads, float* const* 
  *     Frobenius (about 1e-2 against exact NS5 on Gaussian, tall and
  *     ill-conditioned inputs); e4m3 in a third iteration would not stay
  *     within 3e-2.
- *   - Applies to the tcgen05 GEMM path; matrices that the fused single-CTA
- *     and CTA-pair kernels run whole (short side <= 128 with long side <= 512,
- *     or both sides <= 256) keep bf16 operands.
+ *   - Applies where the phases run as separate launches (groups with a
+ *     short side above 1024), where it is faster (3-7 % on the GPT-2-XL set and
+ *     the 2048 / 4096 square batches).  Groups that run in the chained launch
+ *     (short side <= 1024) and the matrices the fused single-CTA and CTA-pair
+ *     kernels run whole keep bf16 operands: there the e4m3 copies cost more
+ *     than the shorter products save (measured slower on every such set), so
+ *     for them this call is muon_step_ex.
  *   - Workspace: the e4m3 copies take kp*lp + kp*kp more bytes per matrix
  *     (kp, lp: short and long side rounded up to 128) than muon_workspace_size
  *     reports.

@@ -460,6 +460,7 @@ static_assert(kGemmSmemBytes <= 232448, "more dynamic shared memory than a CTA m
 template <int kMode, bool kFinal, bool kChain, bool kFp8 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ GemmArgs p) {
   static_assert(!(kChain && kFinal), "the chained launch takes the final update from its items");
+  static_assert(!(kChain && kFp8), "e4m3 operands run only in the per-phase launches");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;

@@ -28,7 +28,6 @@
 #include <queue>
 #include <set>
 #include <string>
-#include <tuple>
 #include <vector>
 
 #include "muon.h"
@@ -131,7 +130,7 @@ struct Plan {
   std::vector<std::vector<const void*>> wmap_key;
   std::vector<CUtensorMap*> wmap_host;
   cudaEvent_t wmap_copied = nullptr;
-  std::map<std::tuple<size_t, int, int>, ChainTables> chains;   // (group, ns_steps, fp8_iters) -> work lists
+  std::map<std::pair<size_t, int>, ChainTables> chains;   // (group, ns_steps) -> work lists
   ~Plan() {
     if (tmaps) cudaFree(tmaps);
     if (tmaps8) cudaFree(tmaps8);
@@ -308,8 +307,7 @@ bool chain_static_priority() {
   return rule == 1;
 }
 
-void build_chain(const Group& g, int ns_steps, int fp8_iters, int ncl, std::vector<WorkItem>& items,
-                 std::vector<int>& off) {
+void build_chain(const Group& g, int ns_steps, int ncl, std::vector<WorkItem>& items, std::vector<int>& off) {
   constexpr double kOverhead = 2.0;
   constexpr double kFinalCost = 1.5;          // the last update also reads and writes W
   const double lat = chain_latency_units();
@@ -318,20 +316,14 @@ void build_chain(const Group& g, int ns_steps, int fp8_iters, int ncl, std::vect
   struct MatState {
     int cls = 0, b = 0, T = 0, Tn = 0;
     int ntiles[4] = {0, 0, 0, 0};
-    double cost[4] = {0, 0, 0, 0};   // bf16 operands; a product with e4m3 operands has half the K-blocks
+    double cost[4] = {0, 0, 0, 0};
     int phase = 0, next = 0;
     int need = 0;              // tile halves completed before the current phase
     double vis = 0.0;          // latest visibility time among the current phase's tiles
     double total = 0.0;
   };
   auto mode_of = [&](int j) { return j == nphases - 1 ? (int)kModeFinal : j % 3; };
-  auto cost_of = [&](const auto& st, int j) {   // which products read e4m3 operands: as the kernel's set_precision
-    const int it = j / 3, mode = j % 3;
-    const bool op8 = mode == kModePoly ? it < fp8_iters : (mode == kModeGram && it >= 1 && it < fp8_iters);
-    const double kb = (mode == kModeGram ? st.cost[kModeGram] : st.cost[kModeUpdate]) - kOverhead;
-    const double c = (op8 ? kb / 2 : kb) + kOverhead;
-    return mode_of(j) == kModeFinal ? kFinalCost * c : c;
-  };
+  auto cost_of = [&](const auto& st, int j) { return st.cost[mode_of(j)]; };
   std::vector<MatState> ms(nm);
   for (size_t ci = 0; ci < g.classes.size(); ++ci) {
     const ClassDesc& cd = g.classes[ci];
@@ -520,11 +512,9 @@ cudaError_t launch_gemm(cudaStream_t stream, const GemmArgs& args, int sm_count,
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  // e4m3 instantiations only for launches that use them (the last update never does)
-  const bool f8 = args.fp8_iters > 0 && (chain_clusters > 0 || args.iter < args.fp8_iters);
-  if (chain_clusters > 0)
-    return f8 ? cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false, true, true>, args)
-              : cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false, true>, args);
+  // e4m3 instantiations only for the per-phase launches that use them (the last update never does)
+  const bool f8 = args.fp8_iters > 0 && args.iter < args.fp8_iters;
+  if (chain_clusters > 0) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false, true>, args);
   switch (args.mode) {
     case kModeGram:
       return f8 ? cudaLaunchKernelEx(&cfg, ns_gemm_kernel<kModeGram, false, false, true>, args)
@@ -605,8 +595,7 @@ int device_setup(int dev) {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeUpdate, false, false, true>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
-  CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false, true, true>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+
   {
     // The chained launch's clusters wait on one another's results, so all of
     // them must be resident at once: never launch more than the device holds.
@@ -621,15 +610,12 @@ int device_setup(int dev) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int nclusters = 0, nclusters8 = 0;      // both instantiations of the chained launch (bf16, e4m3)
+    int nclusters = 0;
     if (cudaOccupancyMaxActiveClusters(&nclusters, (void*)ns_gemm_kernel<kModeGram, false, true>, &cfg) !=
-            cudaSuccess ||
-        cudaOccupancyMaxActiveClusters(&nclusters8, (void*)ns_gemm_kernel<kModeGram, false, true, true>, &cfg) !=
-            cudaSuccess) {
+        cudaSuccess) {
       cudaGetLastError();
       nclusters = 0;                         // chained launch unavailable: one launch per phase
     }
-    nclusters = std::min(nclusters, nclusters8);
     g_chain_clusters[dev] = std::min(nclusters, prop.multiProcessorCount / 2);
   }
   g_dev_ready[dev] = true;
@@ -889,15 +875,15 @@ int64_t chain_items(const Group& g, int ns_steps) {
 // The chained launch's work lists for group gidx and ns_steps iterations,
 // built and uploaded on first use (a synchronous copy: make the first call for
 // a set of shapes and an iteration count outside stream capture).
-int get_chain(Ctx& c, Plan& plan, size_t gidx, int ns_steps, int fp8_iters, ChainTables** out) {
-  const auto key = std::make_tuple(gidx, ns_steps, fp8_iters);
+int get_chain(Ctx& c, Plan& plan, size_t gidx, int ns_steps, ChainTables** out) {
+  const auto key = std::make_pair(gidx, ns_steps);
   auto it = plan.chains.find(key);
   if (it == plan.chains.end()) {
     ChainTables ct;
     ct.nclusters = g_chain_clusters[c.dev];
     std::vector<WorkItem> items;
     std::vector<int> off;
-    build_chain(plan.groups[gidx], ns_steps, fp8_iters, ct.nclusters, items, off);
+    build_chain(plan.groups[gidx], ns_steps, ct.nclusters, items, off);
     ct.nitems = (int)items.size();
     const size_t ib = align_up(items.size() * sizeof(WorkItem), 256), ob = off.size() * sizeof(int);
     if (cudaMalloc(&ct.dev, ib + ob) != cudaSuccess) {
@@ -1012,7 +998,10 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
   ga->a = io.a; ga->b = io.b; ga->c = io.c; ga->lr = io.lr;
   ga->assign = io.assign;
   fill_out(ga->out);
-  const int fp8_iters = std::min(io.fp8_iters, io.ns_steps);
+  // e4m3 operands only where the phases run as separate launches: in the
+  // chained launch the extra e4m3 copies the epilogues write cost more than
+  // the halved K-loops save (measured slower on every chained workload)
+  const int fp8_iters = chain ? 0 : std::min(io.fp8_iters, io.ns_steps);
   if (fp8_iters > 0) {
     ga->tmaps8 = (const CUtensorMap*)((char*)plan.tmaps8 + g.off_tmaps8);
     ga->fp8_iters = fp8_iters;
@@ -1021,7 +1010,7 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
 
   if (chain) {
     ChainTables* ct = nullptr;
-    int rc = get_chain(c, plan, gidx, io.ns_steps, fp8_iters, &ct);
+    int rc = get_chain(c, plan, gidx, io.ns_steps, &ct);
     if (rc) return rc;
     for (size_t ci = 0; ci < g.sym_cls.size(); ++ci) ga->cls[ci] = g.sym_cls[ci];
     ga->items = ct->items;
@@ -1494,7 +1483,7 @@ int muon_chain_plan(const int64_t* shapes, int n, int ns_steps, int nclusters, i
   }
   std::vector<WorkItem> list;
   std::vector<int> off;
-  build_chain(plan.groups[0], ns_steps, 0, nclusters, list, off);
+  build_chain(plan.groups[0], ns_steps, nclusters, list, off);
   *nitems = (int64_t)list.size();
   for (int c = 0; c <= nclusters; ++c) cluster_off[c] = off[c];
   if (!items || capacity < (int64_t)list.size())
