@@ -426,6 +426,7 @@ struct __align__(8) GemmCtrl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
+  int prod_passed;            // chained launch: items whose inputs the producer has seen complete
 };
 static_assert(sizeof(GemmCtrl) <= kSmemCtrlBytes, "GemmCtrl does not fit its shared-memory slot");
 static_assert(kGemmSmemBytes <= 232448, "more dynamic shared memory than a CTA may have");
@@ -506,6 +507,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort_flag = 0;
+    ctl->prod_passed = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -550,6 +552,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           if (!wait_count(&p.done[T.mat], (uint32_t)T.need, wc, kDevTimeoutDep)) { ok = false; break; }
           fence_proxy_async_global();
         }
+        if (kChain) st_release_cta_shared(&ctl->prod_passed, it + 1);   // inputs of items 0..it are complete
         const CUtensorMap* tA;
         const CUtensorMap* tB;
         if (T.mode == kModeGram) { tA = &p.tmaps[C.tmap_base + (T.x_in ? kTmX1 : kTmX0)]; tB = tA; }
@@ -693,13 +696,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       bool ok = true;
       // Arming chunk q hands buffer q % 4 to the math warps: with the A block
       // the polynomial epilogue adds loaded into it, or empty.  In the chained
-      // launch a polynomial tile's chunks are armed only once the DMA has
-      // reached that tile, after every earlier tile published its results, so
-      // waiting there for the tile's inputs never waits on this cluster.
+      // launch a polynomial tile's chunks are armed only once its inputs are
+      // known to be complete -- the producer has passed the tile's dependency
+      // wait -- or once the DMA has reached that tile, after every earlier
+      // tile published its results; so waiting there for the tile's inputs
+      // never waits on this cluster, and the A slices usually load while the
+      // previous tile is still draining.
       int ia = 0, ha = 0, armed = 0;               // next chunk to arm: chunk ha of tile ia
       Tile TA{};
       if (my_tiles > 0) TA = tile_of(0);
-      auto deferred = [&](int drain_tile) { return kChain && ia < my_tiles && TA.mode == kModePoly && ia != drain_tile; };
+      auto deferred = [&](int drain_tile) {
+        return kChain && ia < my_tiles && TA.mode == kModePoly && ia != drain_tile &&
+               ld_acquire_cta_shared(&ctl->prod_passed) <= ia;
+      };
       auto arm_until = [&](int limit, int drain_tile) {
         while (ok && armed < limit && ia < my_tiles && !deferred(drain_tile)) {
           const int b = armed & 3;
