@@ -79,19 +79,22 @@ def load_peaks():
 # they are not part of the GEMM kernel whose DRAM traffic the summary records.
 _FUSED_BEGIN = "// ================================================ small matrices, fused ==="
 _FUSED_END = "// ======================================================= ns_steps == 0 ==="
+_PRO_BEGIN = "// ============================================================ prologue ==="
+_PRO_END = "// ====================================================== NS GEMM kernel ==="
 
 
 def kernel_source_hash() -> str:
     """Hash of the device code the GEMM kernel's ncu figures were taken on:
-    ptx.cuh and kernels.cuh without the fused small-matrix kernels, comments
-    and whitespace removed (a comment edit keeps it)."""
+    ptx.cuh and kernels.cuh without the prologue and the fused small-matrix
+    kernels, comments and whitespace removed (a comment edit keeps it)."""
     h = hashlib.sha256()
     for f in ("kernels.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "muon_newton_schulz_02_b200", "csrc", f)) as fh:
             text = fh.read()
-        a, b = text.find(_FUSED_BEGIN), text.find(_FUSED_END)
-        if a >= 0 and b > a:
-            text = text[:a] + text[b:]
+        for begin, end in ((_FUSED_BEGIN, _FUSED_END), (_PRO_BEGIN, _PRO_END)):
+            a, b = text.find(begin), text.find(end)
+            if a >= 0 and b > a:
+                text = text[:a] + text[b:]
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
         text = re.sub(r"//[^\n]*", " ", text)
         h.update(" ".join(text.split()).encode())

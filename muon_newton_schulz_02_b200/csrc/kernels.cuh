@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kProThreads) prologue_kernel(const __grid_cons
 
   if (!M.trans) {
     // X[xr][xc] = G[xr][xc]: each warp walks one row segment of 128 columns.
-#pragma unroll 2
+#pragma unroll
     for (int pass = 0; pass < kProRows / 8; ++pass) {
       const int row = xr0 + pass * 8 + warp;
       const int col = xc0 + lane * 4;
@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kProThreads) prologue_kernel(const __grid_cons
     }
   } else {
     // X[xr][xc] = G[xc][xr]: read a 128 (G rows) x 64 (G cols) block, transpose in shared memory.
-#pragma unroll 2
+#pragma unroll
     for (int pass = 0; pass < kProCols / 16; ++pass) {
       const int gi_l = pass * 16 + (tid >> 4);      // 0..127: G row within block = X col
       const int gj_l = (tid & 15) * 4;              // 0..60 : G col within block = X row

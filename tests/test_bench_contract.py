@@ -72,6 +72,10 @@ def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     text = k.read_text()
     k.write_text(text.replace(bench._FUSED_BEGIN, bench._FUSED_BEGIN + "\nconstexpr int kFusedOnly = 1;\n"))
     assert bench.kernel_source_hash() == h0
+    # nor is the prologue
+    text = k.read_text()
+    k.write_text(text.replace(bench._PRO_BEGIN, bench._PRO_BEGIN + "\nconstexpr int kPrologueOnly = 1;\n"))
+    assert bench.kernel_source_hash() == h0
     k.write_text(k.read_text() + "\nconstexpr int kUnused = 1;\n")
     assert bench.kernel_source_hash() != h0
 
