@@ -5,7 +5,7 @@
 //   prologue_kernel   buf <- mu*buf + g ; G = g + mu*buf ; per-matrix ||G||_F ;
 //                     X0 = bf16(G), stored short-side-major (k x l, padded).
 //   ns_gemm_kernel    persistent tcgen05 GEMM over all matrices of a group,
-//                     either one launch chaining every phase but the last
+//                     either one launch chaining every phase and the weight
 //                     update (per-matrix completion counters order the
 //                     phases), or one launch per phase:
 //                       GRAM    A = s^2 * X X^T            (upper-triangle 256-blocks only)
@@ -17,10 +17,14 @@
 //                     diagonal of B' and the update reads no second copy of X.
 //                     (256 x 256 output tiles per cluster of two CTAs,
 //                     tcgen05.mma.cta_group::2; a template per phase.)
+//                     In the per-phase launches the A A and X X^T products of
+//                     the first iterations may read e4m3 copies of their
+//                     operands (kind::f8f6f4, muon_step_fp8).
 //   ns_small_kernel   the whole step of a small matrix (short side <= 128,
 //                     long side <= 512) in one CTA, everything on chip.
 //   ns_pair_kernel    the same for 128 < short side <= 256, long side <= 256,
 //                     on a cluster of two CTAs (cta_group::2 products).
+//   o16_kernel        bf16 update exchange: O (fp32) -> bf16, or W -= lr * O.
 //   apply_x0_kernel   ns_steps == 0: W -= lr * s * X0.
 #pragma once
 

@@ -4,12 +4,13 @@
 // classes (same padded short side kp and long side lp), each class gets
 // contiguous [batch][kp][lp] bf16 iterates and [batch][kp][kp] Gram /
 // polynomial buffers in the workspace, and one TMA descriptor per buffer and
-// box shape.  A step is then 1 + 3*ns_steps kernel launches on the caller's
-// stream: the fused momentum/norm/cast prologue, then per NS iteration one
-// persistent tcgen05 GEMM launch per phase over all matrices of the group.
-// Small matrices (short side <= 128, long side <= 512; or short side <= 256
-// and long side <= 256, run by CTA pairs) need no workspace:
-// one launch of the fused single-CTA kernel runs their whole step.
+// box shape.  A step of a group is then the fused momentum/norm/cast prologue
+// and either one chained persistent tcgen05 GEMM launch that runs every
+// Newton-Schulz phase and the weight update from host-built work lists (short
+// sides up to 1024), or one launch per phase (3 * ns_steps launches), all on
+// the caller's stream.  Small matrices (short side <= 128, long side <= 512;
+// or both sides <= 256, run by CTA pairs) need no workspace: one launch of a
+// fused kernel runs their whole step.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
