@@ -114,6 +114,8 @@ struct ChainTables {
   const int* off = nullptr;
 };
 
+constexpr int kWmapRing = 4;
+
 struct Plan {
   std::vector<int64_t> shapes;
   std::vector<Group> groups;
@@ -127,10 +129,13 @@ struct Plan {
   void* tmaps = nullptr;                    // this plan's own device copy of its tensor maps
   void* tmaps8 = nullptr;                   // tensor maps of the e4m3 copies, encoded by the first fp8 call
   // Per group: fp32 tensor maps of the caller's output matrices, re-encoded
-  // when the caller passes other pointers; host copy in pinned memory.
+  // when the caller passes other pointers; host copies in a ring of
+  // kWmapRing pinned staging slots, so that re-encoding does not wait for the
+  // upload of the previous call (the chunks of muon_step_host reuse plans).
   std::vector<std::vector<const void*>> wmap_key;
-  std::vector<CUtensorMap*> wmap_host;
-  cudaEvent_t wmap_copied = nullptr;
+  std::vector<CUtensorMap*> wmap_host;      // per group: kWmapRing slots of its matrices' maps
+  cudaEvent_t wmap_copied[kWmapRing] = {};  // per slot: its last upload has been read
+  int wmap_next = 0;
   std::map<std::pair<size_t, int>, ChainTables> chains;   // (group, ns_steps) -> work lists
   ~Plan() {
     if (tmaps) cudaFree(tmaps);
@@ -139,7 +144,8 @@ struct Plan {
       if (kv.second.dev) cudaFree(kv.second.dev);
     for (auto h : wmap_host)
       if (h) cudaFreeHost(h);
-    if (wmap_copied) cudaEventDestroy(wmap_copied);
+    for (auto e : wmap_copied)
+      if (e) cudaEventDestroy(e);
   }
 };
 
@@ -723,14 +729,14 @@ int get_plan(Ctx& c, const int64_t* shapes, int n, Plan** out, bool fp8 = false)
   p->wmap_key.resize(p->groups.size());
   p->wmap_host.assign(p->groups.size(), nullptr);
   for (size_t gi = 0; gi < p->groups.size(); ++gi) {
-    if (cudaHostAlloc((void**)&p->wmap_host[gi], p->groups[gi].mats.size() * sizeof(CUtensorMap),
+    if (cudaHostAlloc((void**)&p->wmap_host[gi], kWmapRing * p->groups[gi].mats.size() * sizeof(CUtensorMap),
                       cudaHostAllocDefault) != cudaSuccess) {
       cudaGetLastError();
       p->wmap_host[gi] = nullptr;
       return fail(MUON_ERR_NOMEM, "pinned tensor-map staging allocation failed");
     }
   }
-  CUDA_TRY(cudaEventCreateWithFlags(&p->wmap_copied, cudaEventDisableTiming));
+  for (auto& e : p->wmap_copied) CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
   c.plans.push_front(std::move(p));
   // Keep the most recent kMaxPlans plans: enough for the chunks of the
   // host-buffer entry point (up to 16 shape lists) next to the device-buffer
@@ -842,8 +848,10 @@ int update_wmaps(Ctx& c, Plan& plan, size_t gi, const StepIO& io) {
   std::vector<const void*> key(g.mats.size());
   for (size_t i = 0; i < g.mats.size(); ++i) key[i] = io.W[g.mats[i].user];
   if (key == plan.wmap_key[gi]) return MUON_OK;
-  CUDA_TRY(cudaEventSynchronize(plan.wmap_copied));       // the staging buffer is free
-  CUtensorMap* h = plan.wmap_host[gi];
+  const int slot = plan.wmap_next;
+  plan.wmap_next = (slot + 1) % kWmapRing;
+  CUDA_TRY(cudaEventSynchronize(plan.wmap_copied[slot]));   // this slot's previous upload was read
+  CUtensorMap* h = plan.wmap_host[gi] + (size_t)slot * g.mats.size();
   std::memset(h, 0, g.mats.size() * sizeof(CUtensorMap));
   for (size_t i = 0; i < g.mats.size(); ++i) {
     const MatDesc& d = g.mats[i];
@@ -855,7 +863,7 @@ int update_wmaps(Ctx& c, Plan& plan, size_t gi, const StepIO& io) {
   }
   CUDA_TRY(cudaMemcpyAsync((char*)plan.tmaps + g.off_wmaps, h, g.mats.size() * sizeof(CUtensorMap),
                            cudaMemcpyHostToDevice, c.stream));
-  CUDA_TRY(cudaEventRecord(plan.wmap_copied, c.stream));
+  CUDA_TRY(cudaEventRecord(plan.wmap_copied[slot], c.stream));
   plan.wmap_key[gi] = key;
   return MUON_OK;
 }
