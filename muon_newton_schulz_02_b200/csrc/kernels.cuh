@@ -39,7 +39,8 @@ constexpr int kBN = 256;            // columns of the pair tile (TMEM fp32 colum
 constexpr int kBNh = 128;           // B-operand rows / columns loaded by one CTA (half of kBN)
 constexpr int kBK = 64;             // K per pipeline stage: one 128-byte swizzle row of bf16
 constexpr int kUmmaK = 16;          // K of one tcgen05.mma kind::f16
-constexpr int kStages = 5;
+constexpr int kStages = 5;          // operand stages of the per-phase launches
+constexpr int kChainStages = 4;     // of the chained launch (measured faster there, slower per phase)
 constexpr int kGemmThreads = 224;   // warp 0 TMA, warp 1 MMA (+TMEM alloc), warp 2 epilogue DMA, warps 3..6 epilogue math
 constexpr int kEpiThreads = 128;
 constexpr int kEpiWarp0 = 3;        // first epilogue math warp
@@ -71,9 +72,14 @@ constexpr uint32_t kStageABytes = kBM * kBK * 2;     // 16 KB
 constexpr uint32_t kStageBBytes = kBNh * kBK * 2;    // 16 KB
 constexpr uint32_t kStageBytes = kStageABytes + kStageBBytes;
 constexpr uint32_t kSliceBytes = kBM * 64 * 2;       // 16 KB: 128 rows x 64 cols bf16 (one TMA box)
-constexpr uint32_t kSmemDataBytes = kStages * kStageBytes + 4 * kSliceBytes;
 constexpr uint32_t kSmemCtrlBytes = 512;
-constexpr uint32_t kGemmSmemBytes = kSmemDataBytes + kSmemCtrlBytes + 1024;  // + alignment slack
+// dynamic shared memory of a GEMM launch with `stages` operand stages: the
+// stages, the four 16 KB chunk buffers, the control block, alignment slack
+constexpr uint32_t gemm_smem_bytes(int stages) {
+  return stages * kStageBytes + 4 * kSliceBytes + kSmemCtrlBytes + 1024;
+}
+constexpr uint32_t kGemmSmemBytes = gemm_smem_bytes(kStages);
+constexpr uint32_t kChainSmemBytes = gemm_smem_bytes(kChainStages);
 
 // ------------------------------------------------------------ arguments ---
 struct GemmClass {
@@ -433,7 +439,8 @@ struct __align__(8) GemmCtrl {
   int prod_passed;            // chained launch: items whose inputs the producer has seen complete
 };
 static_assert(sizeof(GemmCtrl) <= kSmemCtrlBytes, "GemmCtrl does not fit its shared-memory slot");
-static_assert(kGemmSmemBytes <= 232448, "more dynamic shared memory than a CTA may have");
+static_assert(kGemmSmemBytes <= 232448 && kChainSmemBytes <= 232448, "more dynamic shared memory than a CTA may have");
+static_assert(kChainStages <= kStages, "GemmCtrl holds kStages barriers per ring");
 
 // The Newton-Schulz GEMM kernel.  A cluster of two CTAs (one per SM) computes
 // 256 x 256 output tiles with tcgen05.mma.cta_group::2: each CTA loads its 128
@@ -469,7 +476,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  uint8_t* dbuf = smem + kStages * kStageBytes;        // 2 x 16 KB: slice buffers 0, 1 / fp32 staging 2, 3
+  constexpr int kSt = kChain ? kChainStages : kStages;
+  uint8_t* dbuf = smem + kSt * kStageBytes;            // 2 x 16 KB: slice buffers 0, 1 / fp32 staging 2, 3
   uint8_t* mbuf = dbuf + 2 * kSliceBytes;              // 2 x 16 KB: slice buffers 2, 3 / fp32 staging 0, 1
   GemmCtrl* ctl = reinterpret_cast<GemmCtrl*>(mbuf + 2 * kSliceBytes);
 
@@ -500,7 +508,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
+    for (int s = 0; s < kSt; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl->tmem_full[s], 1);
       mbar_init(&ctl->tmem_empty[s], 8);
@@ -613,7 +621,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
               tma_load_3d_pair(sb, tB, full_lead, kb * kBK, bidx, T.b);
             }
           }
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          if (++stage == kSt) { stage = 0; phase ^= 1u; }
         }
       }
       aborted = !ok;
@@ -672,7 +680,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
           issued_any = true;
           tc_commit_pair(mapa_shared(&ctl->empty[stage], 0));
           tc_commit_pair(mapa_shared(&ctl->empty[stage], 1));
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          if (++stage == kSt) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         tc_commit_pair(mapa_shared(&ctl->tmem_full[acc], 0));

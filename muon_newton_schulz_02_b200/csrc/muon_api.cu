@@ -502,13 +502,13 @@ cudaError_t launch_pdl(void (*kernel)(Args), dim3 grid, dim3 block, size_t smem,
 
 // One GEMM launch: persistent clusters of two CTAs (one CTA per SM).  With
 // `chain_clusters` > 0 it is the chained launch over that many clusters (every
-// phase but the last update); otherwise one Newton-Schulz phase (args.mode).
+// phase and the weight update); otherwise one Newton-Schulz phase (args.mode).
 cudaError_t launch_gemm(cudaStream_t stream, const GemmArgs& args, int sm_count, int chain_clusters = 0) {
   const int pairs = chain_clusters > 0 ? chain_clusters : std::max(1, std::min(args.total_tiles, sm_count / 2));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
-  cfg.dynamicSmemBytes = kGemmSmemBytes;
+  cfg.dynamicSmemBytes = chain_clusters > 0 ? kChainSmemBytes : kGemmSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -595,7 +595,7 @@ int device_setup(int dev) {
   CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeUpdate, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kGemmSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kGemmSmemBytes));
+                                (int)kChainSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false, false, true>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModePoly, false, false, true>,
@@ -609,7 +609,7 @@ int device_setup(int dev) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(prop.multiProcessorCount, 1, 1);
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
-    cfg.dynamicSmemBytes = kGemmSmemBytes;
+    cfg.dynamicSmemBytes = kChainSmemBytes;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
