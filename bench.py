@@ -528,7 +528,7 @@ def run_ours(args):
             roofline["frac_sustained"] = r["achieved"] / float(peaks["bf16_tflops_sustained"])
         if clk:
             roofline["kcycles_per_launch"] = r["us_per_launch"] * clk["sm_mhz"] / 1e3
-    fused = [k for k in ("small", "pair") if prof[k][1]]
+    fused = [k for k in ("small", "pair", "quad") if prof[k][1]]
     if r is None and fused and args.kernel_events:
         # every matrix ran in a fused on-chip kernel: its launches carry the whole step
         f_ms = sum(prof[k][0] for k in fused)

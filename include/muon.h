@@ -248,7 +248,8 @@ void muon_release(void);
 #define MUON_KIND_PAIR 7         /* fused CTA-pair step, 128 < short side <= 256, long side <= 256 */
 #define MUON_KIND_CHAIN 8        /* every Newton-Schulz phase and the weight update, one chained launch */
 #define MUON_KIND_O16 9          /* bf16 update exchange: fp32 -> bf16 rounding of O, or W -= lr * O */
-#define MUON_NUM_KINDS 10
+#define MUON_KIND_QUAD 10        /* fused step on a cluster of four CTAs, short side <= 128, 256 < long side <= 512 */
+#define MUON_NUM_KINDS 11
 
 /* 1: bracket every kernel launch with CUDA events on its stream; 0: stop. */
 int muon_profile_enable(int enable);

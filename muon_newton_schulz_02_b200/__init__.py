@@ -30,7 +30,7 @@ LIB_PATH = os.path.join(HERE, "libmuon_b200.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "muon.h")
 
 NS_A, NS_B, NS_C, NS_STEPS, NS_EPS = 3.4445, -4.7750, 2.0315, 5, 1e-7
-KINDS = ("prologue", "gram", "poly", "update", "update_apply", "apply_x0", "small", "pair", "chain", "o16")
+KINDS = ("prologue", "gram", "poly", "update", "update_apply", "apply_x0", "small", "pair", "chain", "o16", "quad")
 
 STATUS = {0: "MUON_OK", -1: "MUON_ERR_INVALID_ARG", -2: "MUON_ERR_SHAPE", -3: "MUON_ERR_CUDA",
           -4: "MUON_ERR_NOMEM", -5: "MUON_ERR_TIMEOUT", -6: "MUON_ERR_DEVICE", -7: "MUON_ERR_UNSUPPORTED"}

@@ -1829,6 +1829,439 @@ __global__ void __launch_bounds__(kPairThreads, 1) ns_pair_kernel(const __grid_c
   }
 }
 
+// ============================================= small matrices, four CTAs ===
+// The whole step of one small matrix (short side k <= 128, long side
+// 256 < l <= 512) on a cluster of four CTAs, each holding 128 columns of X (a
+// quarter of the long side), so that the memory phases (g, buf and W) and the
+// quarter-sized products run on four SMs instead of one.  The Gram matrix is a
+// sum over the quarters: every CTA computes its partial X_q X_q^T in TMEM and
+// sends row block r of it (32 rows, fp32) into CTA r's shared memory; CTA r
+// adds the four partials of its rows in a fixed order and writes those rows of
+// A (bf16) into every CTA.  Each CTA then forms the whole polynomial matrix
+// B = b A + c A A (128 x 128, from its own copy of A) and the update of its
+// own quarter, X_q' = a s X_q + s B X_q.  Cluster barriers separate the
+// exchanges; every CTA takes every barrier on every path (a CTA that gave up
+// on a bounded wait only stops issuing and waiting).
+// 16-byte asynchronous copy global -> shared memory (bypassing L1) and the
+// wait for all of this thread's copies.
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+constexpr int kQuadThreads = 128;
+constexpr int kQuadCols = 128;                 // columns of X held by one CTA
+constexpr int kQuadMaxMats = 37;               // four CTAs each: one wave of 148 SMs
+// [sender][row rr of this CTA's block][16-byte unit] fp32, unit u of row rr
+// stored at (u + rr) mod 32 so that the 32 rows' writes and reads hit
+// different banks
+constexpr uint32_t kQuadInbox = 4 * 32 * 128 * 4;
+__device__ __forceinline__ uint32_t quad_inbox_off(uint32_t q, uint32_t rr, uint32_t u) {
+  return ((q * 32u + rr) * 32u + ((u + rr) & 31u)) * 16u;
+}
+constexpr uint32_t kQuadSmem = 6 * kSmallChunk + kQuadInbox + 256 + 1024;
+
+__global__ void __launch_bounds__(kQuadThreads, 1) ns_quad_kernel(const __grid_constant__ SmallArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Xs = smem;                                        // 2 chunks: this CTA's 128 columns of X
+  uint8_t* As = Xs + 2 * kSmallChunk;                        // 2 chunks: A; the apply's staging at the end
+  uint8_t* Bs = As + 2 * kSmallChunk;                        // 2 chunks: B
+  float* inbox = reinterpret_cast<float*>(Bs + 2 * kSmallChunk);
+  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(inbox) + kQuadInbox);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(abort_flag + 1);    // [0..3] warp partials, [4..7] the CTAs' partials
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const SmallMat& M = p.mats[cluster_id_x()];
+  const int c0 = (int)rank * kQuadCols;                      // first X column of this CTA
+
+  if (tid == 0) {
+    mbar_init(mma_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  cluster_sync_all();                                        // every CTA initialised before any remote write
+  tc_fence_after();
+  griddep_launch_dependents();
+  griddep_wait();
+  WaitCtx wc{abort_flag, p.status, p.wait_limit_ns, 0u};
+
+  // ---- momentum, norm partial, this CTA's quarter of X0 (bf16, padding zero)
+  const float* __restrict__ gp = M.g;
+  float* __restrict__ bp = M.buf;
+  auto load4 = [&](size_t off, int col, int ncols, float (&gv)[4], float (&bv)[4]) {
+    if (M.vec && col + 3 < ncols) {
+      const float4 g4 = __ldg(reinterpret_cast<const float4*>(gp + off));
+      gv[0] = g4.x; gv[1] = g4.y; gv[2] = g4.z; gv[3] = g4.w;
+      if (p.has_buf) {
+        const float4 b4 = *reinterpret_cast<const float4*>(bp + off);
+        bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (col + q < ncols) {
+          gv[q] = gp[off + q];
+          if (p.has_buf) bv[q] = bp[off + q];
+        }
+    }
+  };
+  auto store4 = [&](size_t off, int col, int ncols, const float (&bv)[4]) {
+    if (!p.has_buf) return;
+    if (M.vec && col + 3 < ncols) {
+      *reinterpret_cast<float4*>(bp + off) = make_float4(bv[0], bv[1], bv[2], bv[3]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (col + q < ncols) bp[off + q] = bv[q];
+    }
+  };
+  float ss = 0.f;
+  // Aligned rows: the CTA's 128 x 128 blocks of g and buf land in shared
+  // memory by asynchronous copies, all in flight at once (g in the inbox,
+  // buf in A | B, both free until the first product), then each warp walks
+  // rows of them.  Otherwise: plain loads, eight rows per batch.
+  const bool staged = M.vec;
+  const int gr0 = M.trans ? c0 : 0, gc0 = M.trans ? 0 : c0;  // block origin in g: G rows, G columns
+  float* Sg = inbox;
+  float* Sb = reinterpret_cast<float*>(As);
+  if (staged) {
+    for (int e = tid; e < 128 * 32; e += kQuadThreads) {
+      const int i = e >> 5, u = e & 31;                      // block row, 16-byte unit
+      const int gi = gr0 + i, gj = gc0 + 4 * u;
+      if (gi < M.m && gj < M.n) {
+        const size_t off = (size_t)gi * M.n + gj;
+        cp_async_16(Sg + i * 128 + 4 * u, gp + off);
+        if (p.has_buf) cp_async_16(Sb + i * 128 + 4 * u, bp + off);
+      }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+  }
+  // G[i][j] for G row i = i0 + 4 t (eight per batch, all loads first), G columns
+  // j .. j+3 with j = jb + 4 lane
+  auto batch = [&](int i0, int jb, auto&& put) {
+    if (staged) {
+      const int j = jb + 4 * lane;
+#pragma unroll 2
+      for (int t = 0; t < 8; ++t) {
+        const int i = i0 + 4 * t;
+        float G[4] = {0.f, 0.f, 0.f, 0.f};
+        if (i < M.m && j < M.n) {
+          const int so = (i - gr0) * 128 + (j - gc0);
+          const float4 g4 = *reinterpret_cast<const float4*>(Sg + so);
+          float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (p.has_buf) b4 = *reinterpret_cast<const float4*>(Sb + so);
+          float gv[4] = {g4.x, g4.y, g4.z, g4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) G[q] = nesterov_g(gv[q], bv[q], p.mu, p.nesterov, p.has_buf);
+          if (p.has_buf) *reinterpret_cast<float4*>(bp + (size_t)i * M.n + j) = make_float4(bv[0], bv[1], bv[2], bv[3]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) ss = fmaf(G[q], G[q], ss);
+        put(i, j, G);
+      }
+      return;
+    }
+    float gv[8][4], bv[8][4];
+    const int j = jb + 4 * lane;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) { gv[t][q] = 0.f; bv[t][q] = 0.f; }
+      const int i = i0 + 4 * t;
+      if (i < M.m && j < M.n) load4((size_t)i * M.n + j, j, M.n, gv[t], bv[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int i = i0 + 4 * t;
+      float G[4] = {0.f, 0.f, 0.f, 0.f};
+      if (i < M.m && j < M.n) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (j + q < M.n) G[q] = nesterov_g(gv[t][q], bv[t][q], p.mu, p.nesterov, p.has_buf);
+        store4((size_t)i * M.n + j, j, M.n, bv[t]);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ss = fmaf(G[q], G[q], ss);
+      put(i, j, G);
+    }
+  };
+  if (!M.trans) {
+    // X = G: rows 0..127 of this CTA's columns c0 .. c0+127
+    for (int i0 = warp; i0 < kSmallMaxK; i0 += 32)
+      batch(i0, c0, [&](int i, int j, const float (&G)[4]) {
+        *reinterpret_cast<uint2*>(Xs + chunk_off((uint32_t)i, (uint32_t)(j - c0))) =
+            make_uint2(pack_bf16x2(G[0], G[1]), pack_bf16x2(G[2], G[3]));
+      });
+  } else {
+    // X = G^T: G rows c0 .. c0+127 are this CTA's X columns, G's (<= 128) columns its rows
+    for (int i0 = c0 + warp; i0 < c0 + kQuadCols; i0 += 32)
+      batch(i0, 0, [&](int i, int j, const float (&G)[4]) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<__nv_bfloat16*>(Xs + chunk_off((uint32_t)(j + q), (uint32_t)(i - c0))) =
+              __float2bfloat16_rn(G[q]);
+      });
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  if (tid < 4) {                                             // this CTA's partial into every CTA's slot
+    const float part = red[0] + red[1] + red[2] + red[3];
+    st_cluster_u32(mapa_shared(&red[4 + rank], (uint32_t)tid), __float_as_uint(part));
+  }
+  auto publish = [&]() {                                     // this phase's writes (local and remote) -> next phase
+    fence_async_all();
+    tc_fence_before();
+    cluster_sync_all();
+    tc_fence_after();
+  };
+  auto publish_local = [&]() {                               // this CTA's writes -> its next MMAs
+    fence_async_shared();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  };
+  publish();
+  const float scale =
+      1.0f / ((float)sqrt((double)red[4] + (double)red[5] + (double)red[6] + (double)red[7]) + p.eps);
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's 32 lanes
+  const int r = warp * 32 + lane;                            // row of X / A / B owned by this thread
+  bool ok = true;
+  uint32_t phase = 0;
+  auto wait_mma = [&]() {
+    bool got = ok && mbar_wait(mma_bar, phase, wc, kDevTimeoutAccum);
+    phase ^= 1u;
+    ok = __syncthreads_and(got) != 0;
+    tc_fence_after();
+  };
+  // W -= lr * O (or O = result) for X columns c0 + 32 cc .. +31 of this thread's
+  // row r, staged in the A buffer (free by then), then read-modified-written in
+  // whole 128-byte rows
+  auto apply_chunk = [&](int cc, const float* v) {
+    float* S = reinterpret_cast<float*>(As);
+    if (!M.trans) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float4*>(S + r * 32 + ((j ^ (r & 7)) << 2)) =
+            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 32; ++q) S[q * 128 + r] = v[q];
+    }
+    __syncthreads();
+    float4 o[8], w4[8];
+    float* wp[8];
+    bool okw[8], full[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int idx = tid + kQuadThreads * t;
+      int wi, wj;
+      if (!M.trans) {
+        const int row = idx >> 3, qd = idx & 7;
+        wi = row; wj = c0 + cc * 32 + 4 * qd;
+        o[t] = *reinterpret_cast<const float4*>(S + row * 32 + ((qd ^ (row & 7)) << 2));
+      } else {
+        const int c = idx >> 5, qd = idx & 31;
+        wi = c0 + cc * 32 + c; wj = 4 * qd;
+        o[t] = *reinterpret_cast<const float4*>(S + c * 128 + 4 * qd);
+      }
+      okw[t] = wi < M.m && wj < M.n;
+      full[t] = M.vec && wj + 3 < M.n;
+      wp[t] = M.w + (size_t)wi * M.n + wj;
+      w4[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (okw[t] && full[t] && !p.assign) w4[t] = *reinterpret_cast<const float4*>(wp[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (!okw[t]) continue;
+      if (full[t]) {
+        float4 r4 = w4[t];
+        if (p.assign) r4 = o[t];
+        else { r4.x -= p.lr * o[t].x; r4.y -= p.lr * o[t].y; r4.z -= p.lr * o[t].z; r4.w -= p.lr * o[t].w; }
+        *reinterpret_cast<float4*>(wp[t]) = r4;
+      } else {
+        const float ov[4] = {o[t].x, o[t].y, o[t].z, o[t].w};
+        const int wj = (int)((wp[t] - M.w) % M.n);
+        for (int e = 0; e < 4 && wj + e < M.n; ++e) wp[t][e] = p.assign ? ov[e] : wp[t][e] - p.lr * ov[e];
+      }
+    }
+    __syncthreads();
+  };
+
+  const uint32_t idesc_kk = idesc_bf16_f32(128, 128, 0, 0);
+  for (int it = 0; it < p.ns_steps; ++it) {
+    const float s = it == 0 ? scale : 1.0f;
+    const bool last = it == p.ns_steps - 1;
+    // ---- partial Gram of this quarter: P = X_q X_q^T (K = 128 columns)
+    if (tid == 0 && ok) {
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t d = smem_desc_sw128(smem_u32(Xs) + (kk >> 2) * kSmallChunk + (kk & 3) * 32, 16, 1024);
+        tc_mma_bf16(tmem, d, d, idesc_kk, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(mma_bar);
+    }
+    wait_mma();
+    if (ok) {
+      // row r of P goes to CTA warp (the owner of rows 32 warp .. +31), slot `rank`
+      const uint32_t dst = mapa_shared(inbox, (uint32_t)warp);
+#pragma unroll 1
+      for (int c64 = 0; c64 < 2; ++c64) {
+        float v[64];
+        tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v);
+#pragma unroll
+        for (int q = 0; q < 64; q += 4)
+          st_cluster_v4(dst + quad_inbox_off(rank, (uint32_t)lane, (uint32_t)((c64 * 64 + q) >> 2)),
+                        make_uint4(__float_as_uint(v[q]), __float_as_uint(v[q + 1]), __float_as_uint(v[q + 2]),
+                                   __float_as_uint(v[q + 3])));
+      }
+    }
+    publish();
+    // ---- rows 32 rank .. +31 of A = s^2 * (P_0 + P_1 + P_2 + P_3), to every CTA
+    if (ok) {
+      // this thread: row rr of the block, columns 8 j .. 8 j + 7 for j = (tid & 3) + 4 k
+      const int rr = tid >> 2;
+      const uint8_t* ib = reinterpret_cast<const uint8_t*>(inbox);
+      float acc[4][8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)                            // senders in a fixed order
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t j = (uint32_t)((tid & 3) + 4 * k);
+          const float4 f0 = *reinterpret_cast<const float4*>(ib + quad_inbox_off((uint32_t)q, (uint32_t)rr, 2 * j));
+          const float4 f1 = *reinterpret_cast<const float4*>(ib + quad_inbox_off((uint32_t)q, (uint32_t)rr, 2 * j + 1));
+          acc[k][0] += f0.x; acc[k][1] += f0.y; acc[k][2] += f0.z; acc[k][3] += f0.w;
+          acc[k][4] += f1.x; acc[k][5] += f1.y; acc[k][6] += f1.z; acc[k][7] += f1.w;
+        }
+      const int row = (int)rank * 32 + rr;
+      const float s2 = s * s;
+      uint4 pk[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        pk[k] = make_uint4(pack_bf16x2(s2 * acc[k][0], s2 * acc[k][1]), pack_bf16x2(s2 * acc[k][2], s2 * acc[k][3]),
+                           pack_bf16x2(s2 * acc[k][4], s2 * acc[k][5]), pack_bf16x2(s2 * acc[k][6], s2 * acc[k][7]));
+#pragma unroll
+      for (int d = 0; d < 4; ++d) {
+        const uint32_t abase = mapa_shared(As, (uint32_t)d);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          st_cluster_v4(abase + chunk_off((uint32_t)row, (uint32_t)(8 * ((tid & 3) + 4 * k))), pk[k]);
+      }
+    }
+    publish();
+    // ---- B = b A + c A A (A symmetric: both operands K-major rows of A)
+    if (tid == 0 && ok) {
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t d = smem_desc_sw128(smem_u32(As) + (kk >> 2) * kSmallChunk + (kk & 3) * 32, 16, 1024);
+        tc_mma_bf16(tmem, d, d, idesc_kk, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(mma_bar);
+    }
+    wait_mma();
+#pragma unroll 1
+    for (int c64 = 0; c64 < 2 && ok; ++c64) {
+      float v[64];
+      tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v);
+#pragma unroll
+      for (int q = 0; q < 64; q += 8) {
+        const uint4 araw = *reinterpret_cast<const uint4*>(As + chunk_off((uint32_t)r, (uint32_t)(c64 * 64 + q)));
+        const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&araw);
+        float o8[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(ah[e]);
+          o8[2 * e] = fmaf(p.c, v[q + 2 * e], p.b * f.x);
+          o8[2 * e + 1] = fmaf(p.c, v[q + 2 * e + 1], p.b * f.y);
+        }
+        *reinterpret_cast<uint4*>(Bs + chunk_off((uint32_t)r, (uint32_t)(c64 * 64 + q))) =
+            make_uint4(pack_bf16x2(o8[0], o8[1]), pack_bf16x2(o8[2], o8[3]), pack_bf16x2(o8[4], o8[5]),
+                       pack_bf16x2(o8[6], o8[7]));
+      }
+    }
+    publish_local();
+    // ---- X_q' = a s X_q + s B X_q : M = N = K = 128, X read MN-major
+    if (tid == 0 && ok) {
+      const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 1);
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t a = smem_u32(Bs) + (kk >> 2) * kSmallChunk + (kk & 3) * 32;
+        const uint32_t b = smem_u32(Xs) + kk * (16 * 128);
+        tc_mma_bf16(tmem, smem_desc_sw128(a, 16, 1024), smem_desc_sw128(b, kSmallChunk, 1024), idesc,
+                    kk > 0 ? 1u : 0u);
+      }
+      tc_commit(mma_bar);
+    }
+    wait_mma();
+#pragma unroll 1
+    for (int c64 = 0; c64 < 2 && ok; ++c64) {
+      float v64[64];
+      tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v64);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int cc = 2 * c64 + half;
+        float* v = v64 + 32 * half;
+#pragma unroll
+        for (int q = 0; q < 32; q += 8) {
+          const uint32_t xo = chunk_off((uint32_t)r, (uint32_t)(cc * 32 + q));
+          const uint4 xraw = *reinterpret_cast<const uint4*>(Xs + xo);
+          const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xraw);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(xh[e]);
+            v[q + 2 * e] = fmaf(s, v[q + 2 * e], p.a * s * f.x);
+            v[q + 2 * e + 1] = fmaf(s, v[q + 2 * e + 1], p.a * s * f.y);
+          }
+          if (!last)
+            *reinterpret_cast<uint4*>(Xs + xo) =
+                make_uint4(pack_bf16x2(v[q], v[q + 1]), pack_bf16x2(v[q + 2], v[q + 3]),
+                           pack_bf16x2(v[q + 4], v[q + 5]), pack_bf16x2(v[q + 6], v[q + 7]));
+        }
+        if (last) apply_chunk(cc, v);
+      }
+    }
+    if (!last) publish_local();
+  }
+  if (p.ns_steps == 0 && ok) {
+    // O = s * X0 (the listing with an empty loop)
+#pragma unroll 1
+    for (int cc = 0; cc < kQuadCols / 32; ++cc) {
+      float v[32];
+#pragma unroll
+      for (int q = 0; q < 32; q += 8) {
+        const uint4 xraw = *reinterpret_cast<const uint4*>(Xs + chunk_off((uint32_t)r, (uint32_t)(cc * 32 + q)));
+        const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xraw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(xh[e]);
+          v[q + 2 * e] = scale * f.x;
+          v[q + 2 * e + 1] = scale * f.y;
+        }
+      }
+      apply_chunk(cc, v);
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 // ==================================================== bf16 update exchange ===
 // For a data-parallel step that exchanges the orthogonalised update O in bf16
 // (half the bytes of fp32 weights): `convert` rounds O (fp32, written by a

@@ -121,6 +121,7 @@ struct Plan {
   std::vector<Group> groups;
   std::vector<MatDesc> small;               // matrices of the fused single-CTA kernel (no workspace)
   std::vector<MatDesc> pair;                // matrices of the fused CTA-pair kernel (no workspace)
+  std::vector<MatDesc> quad;                // matrices of the fused four-CTA kernel (no workspace)
   size_t ws_bytes = 0;
   size_t ws_bytes_fp8 = 0;                  // with the e4m3 copies of muon_step_fp8
   size_t tmap_bytes = 0;
@@ -178,6 +179,16 @@ int build_layout(const int64_t* shapes, int n, Plan& plan) {
       else big.push_back(d);
     }
     all.swap(big);
+    // A few such matrices with a long side above 256 leave most SMs idle under
+    // one CTA each: they take a cluster of four CTAs (a quarter of the long
+    // side each) instead.  Many of them fill the GPU one CTA each already.
+    int longer = 0;
+    for (const auto& d : plan.small) longer += d.l > 256;
+    if (longer > 0 && longer <= kQuadMaxMats) {
+      std::vector<MatDesc> keep;
+      for (const auto& d : plan.small) (d.l > 256 ? plan.quad : keep).push_back(d);
+      plan.small.swap(keep);
+    }
   }
   // greedy grouping in caller order, respecting kMaxMats and kMaxClasses
   std::vector<std::vector<MatDesc>> raw;
@@ -586,6 +597,7 @@ int device_setup(int dev) {
                                      std::to_string(prop.major) + std::to_string(prop.minor));
   CUDA_TRY(cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallSmem));
   CUDA_TRY(cudaFuncSetAttribute(ns_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem));
+  CUDA_TRY(cudaFuncSetAttribute(ns_quad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQuadSmem));
   CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModeGram, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kGemmSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(ns_gemm_kernel<kModePoly, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -765,7 +777,7 @@ cudaEvent_t pool_event(Ctx& c) {
 // ranges cost nothing when no tool is attached.
 const char* const kKindNames[MUON_NUM_KINDS] = {"muon.prologue", "muon.gram", "muon.poly", "muon.update",
                                                 "muon.update_apply", "muon.apply_x0", "muon.small", "muon.pair",
-                                                "muon.chain", "muon.o16"};
+                                                "muon.chain", "muon.o16", "muon.quad"};
 
 template <class F>
 int launch(Ctx& c, int kind, F&& f) {
@@ -1136,6 +1148,29 @@ int run_pair(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& mats, cons
   return MUON_OK;
 }
 
+// One launch of the fused four-CTA kernel over every matrix routed to it (a cluster each).
+int run_quad(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& mats, const StepIO& io, int* status) {
+  const int nm = (int)mats.size();
+  auto sa = fused_args(mats, 0, nm, io, status, false);
+  return launch_fused(c, MUON_KIND_QUAD, [&] {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(4 * nm, 1, 1);
+    cfg.blockDim = dim3(kQuadThreads, 1, 1);
+    cfg.dynamicSmemBytes = kQuadSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 4;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaLaunchKernelEx(&cfg, ns_quad_kernel, *sa);
+  });
+}
+
 int validate_common(const int64_t* shapes, int n, int ns_steps) {
   if (!shapes) return fail(MUON_ERR_INVALID_ARG, "shapes is null");
   if (n <= 0) return fail(MUON_ERR_INVALID_ARG, "n must be > 0");
@@ -1165,6 +1200,7 @@ int step_impl(const StepIO& io, const int64_t* shapes, int n, void* stream) {
   if ((rc = get_plan(*c, shapes, n, &plan, io.fp8_iters > 0 && io.ns_steps > 0))) return rc;
   if (!plan->small.empty() && (rc = run_small(c, c->stream, plan->small, io, c->status_d))) return rc;
   if (!plan->pair.empty() && (rc = run_pair(c, c->stream, plan->pair, io, c->status_d))) return rc;
+  if (!plan->quad.empty() && (rc = run_quad(c, c->stream, plan->quad, io, c->status_d))) return rc;
   for (size_t gi = 0; gi < plan->groups.size(); ++gi)
     if ((rc = run_group(*c, *plan, gi, io))) return rc;
   return MUON_OK;
@@ -1382,6 +1418,7 @@ int muon_step_host(float* const* params, const float* const* grads, float* const
               MUON_NS_C, MUON_NS_EPS, ns_steps, 1, 0};
     if (!plan->small.empty() && (rc = run_small(c, c->stream, plan->small, io, c->status_d))) return rc;
     if (!plan->pair.empty() && (rc = run_pair(c, c->stream, plan->pair, io, c->status_d))) return rc;
+    if (!plan->quad.empty() && (rc = run_quad(c, c->stream, plan->quad, io, c->status_d))) return rc;
     for (size_t gi = 0; gi < plan->groups.size(); ++gi)
       if ((rc = run_group(*c, *plan, gi, io))) return rc;
     CUDA_TRY(cudaEventRecord(ev[2 * ci + 1], c->stream));
@@ -1703,6 +1740,7 @@ extern "C" int muon_step_noalloc(float* const* params, const float* const* grads
   }
   if (!plan.small.empty() && (rc = run_small(nullptr, (cudaStream_t)stream, plan.small, io, status))) return rc;
   if (!plan.pair.empty() && (rc = run_pair(nullptr, (cudaStream_t)stream, plan.pair, io, status))) return rc;
+  if (!plan.quad.empty() && (rc = run_quad(nullptr, (cudaStream_t)stream, plan.quad, io, status))) return rc;
   if (plan.groups.empty()) return MUON_OK;
   return noalloc_launch((cudaStream_t)stream, (char*)base, plan, io, sm_count);
 }
