@@ -33,8 +33,10 @@
  *     not allowed during stream capture: make the first call for a given set
  *     of shapes outside capture) and freed by muon_release().
  *   - Matrices with short side <= 128 and long side <= 512, or with both
- *     sides <= 256, run their whole step in one fused launch (one CTA, or
- *     a cluster of two CTAs, per matrix) and use no workspace.  The others
+ *     sides <= 256, run their whole step in one fused launch (one CTA per
+ *     matrix, a cluster of two CTAs per matrix for both sides <= 256, or -- for
+ *     at most 37 matrices with short side <= 128 and long side above 256 -- a
+ *     cluster of four CTAs per matrix) and use no workspace.  The others
  *     run the momentum/norm/cast prologue, then every Newton-Schulz phase and
  *     the weight update in one chained launch (short side <= 1024), or one
  *     launch per phase (larger matrices).
