@@ -1834,14 +1834,21 @@ __global__ void __launch_bounds__(kPairThreads, 1) ns_pair_kernel(const __grid_c
 // 256 < l <= 512) on a cluster of four CTAs, each holding 128 columns of X (a
 // quarter of the long side), so that the memory phases (g, buf and W) and the
 // quarter-sized products run on four SMs instead of one.  The Gram matrix is a
-// sum over the quarters: every CTA computes its partial X_q X_q^T in TMEM and
-// sends row block r of it (32 rows, fp32) into CTA r's shared memory; CTA r
-// adds the four partials of its rows in a fixed order and writes those rows of
-// A (bf16) into every CTA.  Each CTA then forms the whole polynomial matrix
-// B = b A + c A A (128 x 128, from its own copy of A) and the update of its
-// own quarter, X_q' = a s X_q + s B X_q.  Cluster barriers separate the
-// exchanges; every CTA takes every barrier on every path (a CTA that gave up
-// on a bounded wait only stops issuing and waiting).
+// sum over the quarters: every CTA computes its partial X_q X_q^T in TMEM, and
+// warp r stages row block r of it (32 rows, fp32) in shared memory and sends it
+// by one bulk copy into CTA r's inbox, counted on an mbarrier there; CTA r
+// adds the four partials of its rows in a fixed order and sends those rows of
+// A (bf16) by bulk copies into every other CTA, counted on a second mbarrier.
+// Each CTA then forms the whole polynomial matrix B = b A + c A A (128 x 128,
+// from its own copy of A) and the update of its own quarter,
+// X_q' = a s X_q + s B X_q.  No cluster barrier separates the iterations:
+// every copy into a buffer follows, through this chain of waits, the
+// receiver's last read of it (a partial of iteration i+1 is sent only after
+// its sender received every A row of iteration i, which each owner sends only
+// after summing its inbox; A rows of i+1 leave their owner only after every
+// CTA's partial of i+1, sent after that CTA's last read of A of iteration i).
+// Waits are bounded; a CTA that gave up stops sending and waiting, and the
+// cluster barriers at the start and the end are taken on every path.
 // 16-byte asynchronous copy global -> shared memory (bypassing L1) and the
 // wait for all of this thread's copies.
 __device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc) {
@@ -1855,21 +1862,28 @@ constexpr int kQuadMaxMats = 37;               // four CTAs each: one wave of 14
 // [sender][row rr of this CTA's block][16-byte unit] fp32, unit u of row rr
 // stored at (u + rr) mod 32 so that the 32 rows' writes and reads hit
 // different banks
-constexpr uint32_t kQuadInbox = 4 * 32 * 128 * 4;
+constexpr uint32_t kQuadSlot = 32 * 128 * 4;                 // one sender's 32 rows of a partial (fp32)
+constexpr uint32_t kQuadInbox = 4 * kQuadSlot;
+constexpr uint32_t kQuadOutbox = 3 * kQuadSlot;               // this CTA's rows for the other three CTAs
+constexpr uint32_t kQuadARows = 32 * 64 * 2;                  // 32 rows of one 64-column chunk of A (bf16)
 __device__ __forceinline__ uint32_t quad_inbox_off(uint32_t q, uint32_t rr, uint32_t u) {
   return ((q * 32u + rr) * 32u + ((u + rr) & 31u)) * 16u;
 }
-constexpr uint32_t kQuadSmem = 6 * kSmallChunk + kQuadInbox + 256 + 1024;
+constexpr uint32_t kQuadSmem = 6 * kSmallChunk + kQuadInbox + kQuadOutbox + 256 + 1024;
+static_assert(kQuadSmem <= 232448, "more dynamic shared memory than a CTA may have");
 
 __global__ void __launch_bounds__(kQuadThreads, 1) ns_quad_kernel(const __grid_constant__ SmallArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* Xs = smem;                                        // 2 chunks: this CTA's 128 columns of X
-  uint8_t* As = Xs + 2 * kSmallChunk;                        // 2 chunks: A; the apply's staging at the end
+  uint8_t* As = Xs + 2 * kSmallChunk;                        // 2 chunks: A
   uint8_t* Bs = As + 2 * kSmallChunk;                        // 2 chunks: B
   float* inbox = reinterpret_cast<float*>(Bs + 2 * kSmallChunk);
-  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(inbox) + kQuadInbox);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
+  uint8_t* outbox = reinterpret_cast<uint8_t*>(inbox) + kQuadInbox;
+  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(outbox + kQuadOutbox);
+  uint64_t* inbox_bar = mma_bar + 1;                         // the three other CTAs' partials of this CTA's rows
+  uint64_t* a_bar = mma_bar + 2;                             // the three other CTAs' rows of A
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 3);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(abort_flag + 1);    // [0..3] warp partials, [4..7] the CTAs' partials
 
@@ -1880,6 +1894,8 @@ __global__ void __launch_bounds__(kQuadThreads, 1) ns_quad_kernel(const __grid_c
 
   if (tid == 0) {
     mbar_init(mma_bar, 1);
+    mbar_init(inbox_bar, 1);
+    mbar_init(a_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -2047,10 +2063,12 @@ __global__ void __launch_bounds__(kQuadThreads, 1) ns_quad_kernel(const __grid_c
     tc_fence_after();
   };
   // W -= lr * O (or O = result) for X columns c0 + 32 cc .. +31 of this thread's
-  // row r, staged in the A buffer (free by then), then read-modified-written in
+  // row r, staged in the outbox (free by then: the last partials it sent were
+  // received before the last rows of A came back; the A buffer may still be
+  // the source of this CTA's last bulk copies), then read-modified-written in
   // whole 128-byte rows
   auto apply_chunk = [&](int cc, const float* v) {
-    float* S = reinterpret_cast<float*>(As);
+    float* S = reinterpret_cast<float*>(outbox);
     if (!M.trans) {
 #pragma unroll
       for (int j = 0; j < 8; ++j)
@@ -2105,29 +2123,50 @@ __global__ void __launch_bounds__(kQuadThreads, 1) ns_quad_kernel(const __grid_c
     const float s = it == 0 ? scale : 1.0f;
     const bool last = it == p.ns_steps - 1;
     // ---- partial Gram of this quarter: P = X_q X_q^T (K = 128 columns)
-    if (tid == 0 && ok) {
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t d = smem_desc_sw128(smem_u32(Xs) + (kk >> 2) * kSmallChunk + (kk & 3) * 32, 16, 1024);
-        tc_mma_bf16(tmem, d, d, idesc_kk, kk > 0 ? 1u : 0u);
+    if (tid == 0) {
+      // this iteration's incoming bytes: three partials of this CTA's rows and
+      // three blocks of rows of A (two 64-column chunks each)
+      mbar_arrive_expect_tx(inbox_bar, 3u * kQuadSlot);
+      mbar_arrive_expect_tx(a_bar, 3u * 2u * kQuadARows);
+      if (ok) {
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t d = smem_desc_sw128(smem_u32(Xs) + (kk >> 2) * kSmallChunk + (kk & 3) * 32, 16, 1024);
+          tc_mma_bf16(tmem, d, d, idesc_kk, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(mma_bar);
       }
-      tc_commit(mma_bar);
     }
     wait_mma();
     if (ok) {
-      // row r of P goes to CTA warp (the owner of rows 32 warp .. +31), slot `rank`
-      const uint32_t dst = mapa_shared(inbox, (uint32_t)warp);
+      // row r of P belongs to CTA `warp` (the owner of rows 32 warp .. +31), slot
+      // `rank` of its inbox: staged in the slot's layout (in place for this
+      // CTA's own rows), then sent by one bulk copy
+      const uint32_t w = (uint32_t)warp;
+      uint8_t* slot = w == rank ? reinterpret_cast<uint8_t*>(inbox) + rank * kQuadSlot
+                                : outbox + (w - (w > rank ? 1u : 0u)) * kQuadSlot;
 #pragma unroll 1
       for (int c64 = 0; c64 < 2; ++c64) {
         float v[64];
         tmem_ld_32x32b_x64(tl + (uint32_t)(c64 * 64), v);
 #pragma unroll
         for (int q = 0; q < 64; q += 4)
-          st_cluster_v4(dst + quad_inbox_off(rank, (uint32_t)lane, (uint32_t)((c64 * 64 + q) >> 2)),
-                        make_uint4(__float_as_uint(v[q]), __float_as_uint(v[q + 1]), __float_as_uint(v[q + 2]),
-                                   __float_as_uint(v[q + 3])));
+          *reinterpret_cast<float4*>(slot + quad_inbox_off(0u, (uint32_t)lane, (uint32_t)((c64 * 64 + q) >> 2))) =
+              make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+      }
+      if (w != rank) {
+        fence_async_shared();                                // the staged rows -> the bulk copy
+        __syncwarp();
+        if (lane == 0)
+          bulk_copy_to_cta(mapa_shared(reinterpret_cast<uint8_t*>(inbox) + rank * kQuadSlot, w), slot, kQuadSlot,
+                           mapa_shared(inbox_bar, w));
       }
     }
-    publish();
+    {
+      // the other CTAs' partials of this CTA's rows have landed (and, through
+      // the CTA barrier, this CTA's own slot)
+      const bool got = ok && mbar_wait_cluster(inbox_bar, (uint32_t)(it & 1), wc, kDevTimeoutDep);
+      ok = __syncthreads_and(got) != 0;
+    }
     // ---- rows 32 rank .. +31 of A = s^2 * (P_0 + P_1 + P_2 + P_3), to every CTA
     if (ok) {
       // this thread: row rr of the block, columns 8 j .. 8 j + 7 for j = (tid & 3) + 4 k
@@ -2156,14 +2195,27 @@ __global__ void __launch_bounds__(kQuadThreads, 1) ns_quad_kernel(const __grid_c
         pk[k] = make_uint4(pack_bf16x2(s2 * acc[k][0], s2 * acc[k][1]), pack_bf16x2(s2 * acc[k][2], s2 * acc[k][3]),
                            pack_bf16x2(s2 * acc[k][4], s2 * acc[k][5]), pack_bf16x2(s2 * acc[k][6], s2 * acc[k][7]));
 #pragma unroll
-      for (int d = 0; d < 4; ++d) {
-        const uint32_t abase = mapa_shared(As, (uint32_t)d);
+      for (int k = 0; k < 4; ++k)
+        *reinterpret_cast<uint4*>(As + chunk_off((uint32_t)row, (uint32_t)(8 * ((tid & 3) + 4 * k)))) = pk[k];
+      fence_async_shared();                                  // this CTA's rows of A -> the bulk copies and MMAs
+    }
+    __syncthreads();
+    if (tid == 0 && ok) {
+      // rows 32 rank .. +31 of each 64-column chunk: 4 KB at the same place in every CTA
+      for (uint32_t d = 1; d < 4; ++d) {
+        const uint32_t peer = (rank + d) & 3u;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          st_cluster_v4(abase + chunk_off((uint32_t)row, (uint32_t)(8 * ((tid & 3) + 4 * k))), pk[k]);
+        for (int c = 0; c < 2; ++c) {
+          const uint8_t* src = As + c * kSmallChunk + rank * kQuadARows;
+          bulk_copy_to_cta(mapa_shared(src, peer), src, kQuadARows, mapa_shared(a_bar, peer));
+        }
       }
     }
-    publish();
+    {
+      const bool got = ok && mbar_wait_cluster(a_bar, (uint32_t)(it & 1), wc, kDevTimeoutDep);
+      ok = __syncthreads_and(got) != 0;
+      tc_fence_after();
+    }
     // ---- B = b A + c A A (A symmetric: both operands K-major rows of A)
     if (tid == 0 && ok) {
       for (int kk = 0; kk < 8; ++kk) {
@@ -2254,6 +2306,9 @@ __global__ void __launch_bounds__(kQuadThreads, 1) ns_quad_kernel(const __grid_c
       apply_chunk(cc, v);
     }
   }
+  // On the abort path, give bulk copies towards this CTA's shared memory time to
+  // land before the cluster leaves (bounded).
+  if (!ok || *reinterpret_cast<volatile int*>(abort_flag)) sleep_ns_bounded(200000);
   tc_fence_before();
   cluster_sync_all();
   if (warp == 0) {
