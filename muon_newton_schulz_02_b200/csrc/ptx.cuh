@@ -173,15 +173,6 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint4 v) {
                "r"(v.w)
                : "memory");
 }
-// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from
-// this CTA's shared memory into a CTA of the cluster; the bytes are counted on
-// an mbarrier in the destination CTA (cluster addresses).
-__device__ __forceinline__ void bulk_copy_to_cta(uint32_t dst_cluster, const void* src, uint32_t bytes,
-                                                 uint32_t bar_cluster) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-               ::"r"(dst_cluster), "r"(smem_u32(src)), "r"(bytes), "r"(bar_cluster)
-               : "memory");
-}
 __device__ __forceinline__ void st_cluster_v2(uint32_t cluster_addr, uint32_t a, uint32_t b) {
   asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};" ::"r"(cluster_addr), "r"(a), "r"(b) : "memory");
 }
