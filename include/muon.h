@@ -274,7 +274,9 @@ int muon_chain_clusters(void);
  * flags bit 1: the same for the next CTA-pair launch, whose first product is
  * not issued, so both CTAs' waits for it run out.
  * flags bit 2 (kept until cleared): run the Newton-Schulz phases as one launch
- * per phase instead of the chained launch (for comparisons). */
+ * per phase instead of the chained launch (for comparisons).
+ * flags bit 3: the next four-CTA launch keeps back one CTA's first Gram
+ * partial, so the waits of every CTA of its clusters run out. */
 int muon_debug_set(int flags, int64_t wait_limit_ns);
 
 /* The work lists of the chained launch for these shapes and `ns_steps`, as

@@ -1005,7 +1005,8 @@ struct SmallMat {
 
 struct SmallArgs {
   int nmats, ns_steps, nesterov, has_buf, assign;
-  int debug_flags;      // bit 0 (CTA-pair kernel): the first product is not issued
+  int debug_flags;      // bit 0: the CTA-pair kernel issues no first product; the four-CTA kernel
+                        // keeps back CTA 1's first partial for CTA 0
   float mu, eps, a, b, c, lr;
   int* status;
   unsigned long long wait_limit_ns;
@@ -2132,18 +2133,19 @@ __global__ void __launch_bounds__(kQuadThreads, 1) ns_quad_kernel(const __grid_c
     const float s = it == 0 ? scale : 1.0f;
     const bool last = it == p.ns_steps - 1;
     // ---- partial Gram of this quarter: P = X_q X_q^T (K = 128 columns)
-    if (tid == 0) {
+    if (tid == 0 && ok) {
       // this iteration's incoming bytes: three partials of this CTA's rows and
-      // three blocks of rows of A (two 64-column chunks each)
+      // three blocks of rows of A (two 64-column chunks each).  One arrival per
+      // phase, and none once the CTA has given up (a phase left incomplete then
+      // only collects the bytes of copies already under way, well inside the
+      // mbarrier's transaction range)
       mbar_arrive_expect_tx(inbox_bar, 3u * kQuadSlot);
       mbar_arrive_expect_tx(a_bar, 3u * 2u * kQuadARows);
-      if (ok) {
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t d = smem_desc_sw128(smem_u32(Xs) + (kk >> 2) * kSmallChunk + (kk & 3) * 32, 16, 1024);
-          tc_mma_bf16(tmem, d, d, idesc_kk, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(mma_bar);
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t d = smem_desc_sw128(smem_u32(Xs) + (kk >> 2) * kSmallChunk + (kk & 3) * 32, 16, 1024);
+        tc_mma_bf16(tmem, d, d, idesc_kk, kk > 0 ? 1u : 0u);
       }
+      tc_commit(mma_bar);
     }
     wait_mma();
     if (ok) {
@@ -2162,7 +2164,10 @@ __global__ void __launch_bounds__(kQuadThreads, 1) ns_quad_kernel(const __grid_c
           *reinterpret_cast<float4*>(slot + quad_inbox_off(0u, (uint32_t)lane, (uint32_t)((c64 * 64 + q) >> 2))) =
               make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
       }
-      if (w != rank) {
+      // fault injection (debug bit 0): CTA 1 keeps back its first partial for CTA 0,
+      // so CTA 0's wait for it runs out, and then every other CTA's wait for CTA 0's rows
+      const bool inject_skip = (p.debug_flags & 1) && it == 0 && rank == 1u && w == 0u;
+      if (w != rank && !inject_skip) {
         fence_async_shared();                                // the staged rows -> the bulk copy
         __syncwarp();
         if (lane == 0)

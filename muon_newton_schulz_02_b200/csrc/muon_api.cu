@@ -1152,6 +1152,7 @@ int run_pair(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& mats, cons
 int run_quad(Ctx* c, cudaStream_t stream, const std::vector<MatDesc>& mats, const StepIO& io, int* status) {
   const int nm = (int)mats.size();
   auto sa = fused_args(mats, 0, nm, io, status, false);
+  if (g_debug_flags & 8) { sa->debug_flags = 1; g_debug_flags &= ~8; }
   return launch_fused(c, MUON_KIND_QUAD, [&] {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(4 * nm, 1, 1);

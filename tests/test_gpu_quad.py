@@ -123,3 +123,24 @@ def test_quad_deterministic_and_unaligned():
     torch.cuda.synchronize()
     assert muon.sync_status() == 0, muon.last_error()
     _check(W, g, b, [x.cpu().numpy() for x in Wd], [x.cpu().numpy() for x in bd])
+
+
+def test_quad_bounded_wait_timeout_is_reported_and_context_survives():
+    shapes = [(128, 512), (300, 100)]
+    W, g, b = _inputs(shapes, seed=8)
+    dev = torch.device("cuda:0")
+    Wd = [torch.as_tensor(x).to(dev) for x in W]
+    gd = [torch.as_tensor(x).to(dev) for x in g]
+    bd = [torch.as_tensor(x).to(dev) for x in b]
+    # the next four-CTA launch keeps back one CTA's first Gram partial: the owner's
+    # wait for it runs out, then every other CTA's wait for the owner's rows of A
+    muon.debug_set(8, 20_000_000)
+    try:
+        muon.step(Wd, gd, bd, lr=0.02, mu=0.95)
+        assert muon.sync_status() == -5               # MUON_ERR_TIMEOUT
+        assert "bounded wait" in muon.last_error()
+    finally:
+        muon.debug_set(0, 0)
+    # the context is still usable and the next step is right
+    W_new, b_new = gpu_step(W, g, b, 0.02, 0.95)
+    _check(W, g, b, W_new, b_new)
