@@ -144,3 +144,20 @@ def test_quad_bounded_wait_timeout_is_reported_and_context_survives():
     # the context is still usable and the next step is right
     W_new, b_new = gpu_step(W, g, b, 0.02, 0.95)
     _check(W, g, b, W_new, b_new)
+
+
+@pytest.mark.parametrize("count,kind", [(37, "quad"), (38, "small")])
+def test_quad_batch_limit(count, kind):
+    # 37 clusters of four CTAs fill one wave of 148 SMs; one matrix more takes
+    # the single-CTA kernel for the whole batch
+    shapes = [(128, 512) if i % 2 == 0 else (300, 96) for i in range(count)]
+    muon.profile_enable(True)
+    muon.profile_read()
+    W, g, b = _inputs(shapes, seed=9)
+    W_new, b_new = gpu_step(W, g, b, 0.02, 0.95)
+    muon.profile_enable(False)
+    prof = muon.profile_read()
+    assert prof[kind][1] == 1 and prof["quad" if kind == "small" else "small"][1] == 0
+    sub = [0, 1, count // 2, count - 1]
+    _check([W[i] for i in sub], [g[i] for i in sub], [b[i] for i in sub],
+           [W_new[i] for i in sub], [b_new[i] for i in sub])
