@@ -56,6 +56,16 @@ def ns_flops(shapes, ns_steps=5) -> float:
     return tot
 
 
+def ns_flops_dense(shapes, ns_steps=5) -> float:
+    """Dense-equivalent flops: the same products without the symmetry of X X^T
+    and A A (every Gram and polynomial output element computed)."""
+    tot = 0.0
+    for r, c in shapes:
+        k, l = min(r, c), max(r, c)
+        tot += ns_steps * (4 * k * k * l + 2 * k * k * k)
+    return tot
+
+
 def flops_by_kind(shapes, ns_steps=5):
     g = p = u = 0.0
     for r, c in shapes:
@@ -607,6 +617,9 @@ def run_ours(args):
                        "cold_l2": "a 1 GiB buffer is written before each cold step (evicts the 126 MB L2)"},
         "kernels": kinds,
         "sweep": sweep,
+        "dense_equivalent": {"value": value * ns_flops_dense(w.shapes) / flops_step, "unit": UNIT,
+                             "what": "the same step counted as dense products (X X^T and A A in full): "
+                                     "a label for comparison, not work done"},
         "frac_of_dense_peak": value / world / burst,
         "frac_of_dense_spec": value / world / 2250.0,
         "peaks": {"source": peak_src, "bf16_tflops": peaks.get("bf16_tflops"),

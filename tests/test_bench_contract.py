@@ -53,6 +53,8 @@ def test_gpu_arm_line():
     assert f8["fp8_iters"] == 2 and f8["ms_per_step"] > 0 and f8["ms_per_step_bf16"] > 0
     assert abs(f8["speedup"] - f8["ms_per_step_bf16"] / f8["ms_per_step"]) < 1e-9
     assert "fp8_variant" not in sw                       # the chained launch keeps bf16 operands
+    de = d["dense_equivalent"]
+    assert de["unit"] == "TFLOP/s" and abs(de["value"] / d["value"] - 1.6307 / 1.1422) < 1e-3
 
 
 def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
@@ -91,6 +93,9 @@ def test_flop_counts_use_the_symmetric_products_once():
     shapes = workloads.get("gpt2_124m").shapes
     assert sum(bench.flops_by_kind(shapes).values()) == bench.ns_flops(shapes)
     assert abs(bench.ns_flops(shapes) / 1.142e12 - 1) < 5e-3              # the step total the docs quote
+    # dense-equivalent: X X^T and A A in full, 2k^2 l + 2k^3 + 2k^2 l per iteration
+    assert bench.ns_flops_dense([(k, l)]) == 5 * (4 * k * k * l + 2 * k ** 3) == bench.ns_flops_dense([(l, k)])
+    assert abs(bench.ns_flops_dense(shapes) / 1.631e12 - 1) < 5e-3
 
 
 def test_traffic_is_reported_only_for_the_profiled_kernel_source(monkeypatch):
