@@ -162,6 +162,21 @@ def test_host_buffer_entry_point_matches_device_path():
         assert np.array_equal(x.numpy(), y)
 
 
+def test_host_buffer_entry_point_over_several_chunks_matches_device_path():
+    # eight matrices of mixed sizes, more bytes than one 32 MB chunk of the
+    # host-buffer pipeline: no path's result depends on which matrices share a
+    # launch, so the two entry points agree bitwise
+    shapes = [(768, 768), (384, 1024), (1024, 384), (300, 700), (128, 200), (640, 640), (96, 200), (1100, 900)]
+    W, g, b = _inputs(shapes, 9)
+    W_dev, b_dev = gpu_step(W, g, b, 0.02, 0.95)
+    Wh = [torch.as_tensor(x.copy()).pin_memory() for x in W]
+    gh = [torch.as_tensor(x.copy()).pin_memory() for x in g]
+    bh = [torch.as_tensor(x.copy()).pin_memory() for x in b]
+    muon.step_host(Wh, gh, bh, lr=0.02, mu=0.95)
+    for x, y in zip(Wh + bh, W_dev + b_dev):
+        assert np.array_equal(x.numpy(), y)
+
+
 @pytest.mark.parametrize("shape,flag", [((384, 384), 1), ((256, 256), 2)], ids=["gemm", "pair"])
 def test_bounded_wait_timeout_is_reported_and_context_survives(shape, flag):
     shapes = [shape]
