@@ -276,8 +276,25 @@ int muon_chain_clusters(void);
  * flags bit 2 (kept until cleared): run the Newton-Schulz phases as one launch
  * per phase instead of the chained launch (for comparisons).
  * flags bit 3: the next four-CTA launch keeps back one CTA's first Gram
- * partial, so the waits of every CTA of its clusters run out. */
+ * partial, so the waits of every CTA of its clusters run out.
+ * flags bit 5 (bounds-checking build only, libmuon_b200_debug.so): the next
+ * GEMM launch that runs one phase gets one tile index past the end of its grid
+ * for every cluster; the device bounds checks stop it before it touches memory
+ * and the call reports MUON_ERR_DEVICE. */
 int muon_debug_set(int flags, int64_t wait_limit_ns);
+
+/* Guard bands (a debugging aid).  With MUON_GUARD_BANDS=1 in the environment
+ * when the library is loaded, the workspace layout leaves 4 KiB of a fixed
+ * byte (0xA5) after every region of a group (iterates, Gram and polynomial
+ * matrices, norm partials, scales, completion counters), written on `stream`
+ * before the group's launches.  This call waits for `stream` and returns how
+ * many of those bytes of the last group run on it no longer hold the fixed
+ * byte (0: no launch wrote past the end of a region), MUON_ERR_UNSUPPORTED
+ * when guard bands are off, or another MUON_ERR_* on failure.  Covers the
+ * workspace of muon_step, muon_step_ex, muon_step_fp8's bf16 regions,
+ * muon_orthogonalize and muon_update_bf16, not the static scratch of
+ * muon_step_noalloc. */
+int muon_guard_check(void* stream);
 
 /* The work lists of the chained launch for these shapes and `ns_steps`, as
  * the library would build them for a device that holds `nclusters` clusters of

@@ -20,13 +20,17 @@ from array import array
 
 __all__ = [
     "step", "PreparedStep", "orthogonalize", "step_host", "step_noalloc", "workspace_size", "sync_status", "last_error", "release",
-    "profile_enable", "profile_read", "launch_count", "chain_clusters", "debug_set", "chain_plan", "lib", "MuonError", "KINDS",
+    "profile_enable", "profile_read", "launch_count", "chain_clusters", "debug_set", "guard_check", "chain_plan", "lib",
+    "MuonError", "KINDS",
     "update_bf16", "apply_bf16",
-    "NS_A", "NS_B", "NS_C", "NS_STEPS", "NS_EPS", "LIB_PATH", "header_functions",
+    "NS_A", "NS_B", "NS_C", "NS_STEPS", "NS_EPS", "LIB_PATH", "DEBUG_LIB_PATH", "header_functions",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmuon_b200.so")
+# the same library with device bounds checks compiled in (tests and debugging):
+# set LIB_PATH to it before the first call
+DEBUG_LIB_PATH = os.path.join(HERE, "libmuon_b200_debug.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "muon.h")
 
 NS_A, NS_B, NS_C, NS_STEPS, NS_EPS = 3.4445, -4.7750, 2.0315, 5, 1e-7
@@ -100,6 +104,8 @@ def lib() -> ctypes.CDLL:
     L.muon_chain_clusters.restype = ctypes.c_int
     L.muon_debug_set.argtypes = [ctypes.c_int, ctypes.c_int64]
     L.muon_debug_set.restype = ctypes.c_int
+    L.muon_guard_check.argtypes = [ctypes.c_void_p]
+    L.muon_guard_check.restype = ctypes.c_int
     L.muon_chain_plan.argtypes = [_I64P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int32),
                                   ctypes.c_int64, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64)]
     L.muon_chain_plan.restype = ctypes.c_int
@@ -335,6 +341,16 @@ def chain_clusters() -> int:
 
 def debug_set(flags: int = 0, wait_limit_ns: int = 0):
     _check(lib().muon_debug_set(int(flags), int(wait_limit_ns)))
+
+
+def guard_check(stream=None) -> int:
+    """Guard-band bytes of the last group run on the stream that a launch
+    changed (0: none); raises MuonError when the library was loaded without
+    MUON_GUARD_BANDS=1."""
+    rc = lib().muon_guard_check(_stream(stream))
+    if rc < 0:
+        _check(rc)
+    return rc
 
 
 def chain_plan(shapes, ns_steps: int = NS_STEPS, nclusters: int = 74):

@@ -39,6 +39,15 @@ constexpr int kBN = 256;            // columns of the pair tile (TMEM fp32 colum
 constexpr int kBNh = 128;           // B-operand rows / columns loaded by one CTA (half of kBN)
 constexpr int kBK = 64;             // K per pipeline stage: one 128-byte swizzle row of bf16
 constexpr int kUmmaK = 16;          // K of one tcgen05.mma kind::f16
+// The bounds-checking build (MUON_DEBUG_BOUNDS) checks every tile a GEMM role
+// takes against its class, matrix and tile grid before touching memory for it;
+// a tile outside them stops the launch with kDevBounds in the status word.
+#ifdef MUON_DEBUG_BOUNDS
+constexpr bool kBoundsChecks = true;
+#else
+constexpr bool kBoundsChecks = false;
+#endif
+
 constexpr int kStages = 5;          // operand stages of the per-phase launches
 constexpr int kChainStages = 4;     // of the chained launch (measured faster there, slower per phase)
 constexpr int kGemmThreads = 224;   // warp 0 TMA, warp 1 MMA (+TMEM alloc), warp 2 epilogue DMA, warps 3..6 epilogue math
@@ -532,6 +541,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   const uint32_t tmem_base = ctl->tmem_base;
   WaitCtx wc{&ctl->abort_flag, p.status, p.wait_limit_ns, mapa_shared(&ctl->abort_flag, rank ^ 1u)};
   bool aborted = false;
+  // bounds-checking build: a tile outside its class's matrices and tile grid
+  auto out_of_range = [&](const Tile& T) {
+    if constexpr (!kBoundsChecks) {
+      return false;
+    } else {
+      bool in = T.cls >= 0 && T.cls < p.nclasses;
+      if (in) {
+        const GemmClass& C = p.cls[T.cls];
+        const int tiles_k = (C.kp + kTile - 1) / kTile, tiles_l = (C.lp + kTile - 1) / kTile;
+        in = T.b >= 0 && T.b < C.batch && T.mat == C.mat_first + T.b && T.mat < kMaxMats && T.tm >= 0 &&
+             T.tm < tiles_k && T.tn >= 0 && T.tn < (T.mode == kModeUpdate ? tiles_l : tiles_k) &&
+             (T.mode == kModeUpdate || T.tm <= T.tn);
+      }
+      if (!in) raise_error(wc, kDevBounds);
+      return !in;
+    }
+  };
   // set-up above overlaps the previous launch; its outputs are read only below
   griddep_launch_dependents();
   griddep_wait();
@@ -557,6 +583,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       bool ok = true;
       for (int it = 0; it < my_tiles && ok; ++it) {
         const Tile T = tile_of(it);
+        if (out_of_range(T)) { ok = false; break; }
         const GemmClass& C = p.cls[T.cls];
         const bool sym = T.mode != kModeUpdate;
         if (kChain && T.need > 0) {
@@ -635,6 +662,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       bool issued_any = false;
       for (int it = 0; it < my_tiles && ok; ++it) {
         const Tile T = tile_of(it);
+        if (out_of_range(T)) { ok = false; break; }
         const GemmClass& C = p.cls[T.cls];
         const bool sym = T.mode != kModeUpdate;
         const int acc = it & 1;
@@ -723,6 +751,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       };
       auto arm_until = [&](int limit, int drain_tile) {
         while (ok && armed < limit && ia < my_tiles && !deferred(drain_tile)) {
+          if (out_of_range(TA)) { ok = false; return; }
           const int b = armed & 3;
           if (TA.mode == kModePoly) {
             if (kChain && ha == 0 && TA.need > 0) {
@@ -749,6 +778,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       int q = 0;                                   // next chunk to drain
       for (int i = 0; i < my_tiles && ok; ++i) {
         const Tile T = tile_of(i);
+        if (out_of_range(T)) { ok = false; break; }
         const GemmClass& C = p.cls[T.cls];
         const int row0 = T.tm * kTile + (int)rank * kBM;
         const int nch = 4 * T.nsub;
@@ -823,6 +853,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     };
     for (int it = 0; it < my_tiles && ok; ++it) {
       const Tile T = tile_of(it);
+      if (out_of_range(T)) { ok = false; break; }
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)((it >> 1) & 1);
       ok = __all_sync(0xffffffffu, mbar_wait(&ctl->tmem_full[acc], acc_phase, wc, kDevTimeoutAccum));

@@ -94,6 +94,7 @@ struct Group {
   size_t data_bytes = 0;
   int sym_tiles = 0, upd_tiles = 0;
   std::vector<GemmClass> sym_cls, upd_cls;
+  std::vector<size_t> guards;      // guard-band offsets (MUON_GUARD_BANDS=1), kGuardBytes each
 };
 
 // The first kTicketBytes of every workspace hold the per-matrix arrival
@@ -102,6 +103,21 @@ struct Group {
 // plan may place anything else there.
 constexpr size_t kTicketBytes = 4096;
 static_assert(kMaxMats * 4 <= kTicketBytes, "ticket region too small");
+
+// Guard bands (a debugging aid, MUON_GUARD_BANDS=1 in the environment when the
+// library is loaded): kGuardBytes of a fixed byte after every workspace region
+// of a group, written before the group's launches; muon_guard_check reports
+// any byte a launch changed, i.e. a write past the end of a region.
+constexpr size_t kGuardBytes = 4096;
+constexpr unsigned char kGuardByte = 0xA5;
+bool guard_bands() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = std::getenv("MUON_GUARD_BANDS");
+    on = (e && std::atoi(e) != 0) ? 1 : 0;
+  }
+  return on == 1;
+}
 
 // Work lists of one chained launch (see ns_gemm_kernel<..., true>) for one
 // group and one iteration count, in device memory: the items of every
@@ -214,15 +230,21 @@ int build_layout(const int64_t* shapes, int n, Plan& plan) {
     std::map<std::pair<int, int>, std::vector<MatDesc>> by;
     for (const auto& d : gm) by[{-d.lp, -d.kp}].push_back(d);
     size_t off = kTicketBytes;
+    // the next region starts at `off`; `end` is the end of the one just placed
+    auto place = [&](size_t end) {
+      off = align_up(end, 1024);
+      if (guard_bands()) { g.guards.push_back(off); off += kGuardBytes; }
+    };
+    place(off);
     for (auto& kv : by) {
       ClassDesc c;
       c.kp = -kv.first.second; c.lp = -kv.first.first;
       const size_t batch = kv.second.size();
       const size_t xb = batch * (size_t)c.kp * c.lp * 2, ab = batch * (size_t)c.kp * c.kp * 2;
-      c.off_x0 = off; off = align_up(off + xb, 1024);
-      c.off_x1 = off; off = align_up(off + xb, 1024);
-      c.off_a = off; off = align_up(off + ab, 1024);
-      c.off_b = off; off = align_up(off + ab, 1024);
+      c.off_x0 = off; place(off + xb);
+      c.off_x1 = off; place(off + xb);
+      c.off_a = off; place(off + ab);
+      c.off_b = off; place(off + ab);
       for (auto& d : kv.second) { c.mats.push_back((int)g.mats.size()); g.mats.push_back(d); }
       g.classes.push_back(c);
     }
@@ -230,9 +252,9 @@ int build_layout(const int64_t* shapes, int n, Plan& plan) {
       g.pro_tile_begin.push_back(g.pro_tiles);
       g.pro_tiles += (d.kp / kProRows) * (d.lp / kProCols);
     }
-    g.off_partials = off; off = align_up(off + (size_t)g.pro_tiles * 4, 1024);
-    g.off_scale = off; off = align_up(off + g.mats.size() * 4, 1024);
-    g.off_done = off; off = align_up(off + g.mats.size() * 4, 1024);
+    g.off_partials = off; place(off + (size_t)g.pro_tiles * 4);
+    g.off_scale = off; place(off + g.mats.size() * 4);
+    g.off_done = off; place(off + g.mats.size() * 4);
     g.data_bytes = off;
     data_max = std::max(data_max, off);
     // GEMM tile bookkeeping
@@ -582,6 +604,7 @@ struct Ctx {
   int sm_count = 148;
   cudaStream_t h2d = nullptr, d2h = nullptr;       // copy streams of muon_step_host
   std::vector<cudaEvent_t> host_events;            // per-chunk ordering events of muon_step_host
+  std::vector<size_t> guards;                      // guard bands of the last group run (MUON_GUARD_BANDS=1)
 };
 
 std::map<std::pair<int, void*>, std::unique_ptr<Ctx>> g_ctx;
@@ -841,12 +864,19 @@ void e4m3_scales(float a, float b, float c, float* sx8, float* sa8) {
   }
 }
 
+// The error a device status code reports (`what`: the launches it came from).
+int status_error(int s, const std::string& what) {
+  if (s == kDevBounds)
+    return fail(MUON_ERR_DEVICE, what + " met a tile outside its class, matrix or tile grid (device bounds check, "
+                                        "code " + std::to_string(s) + ")");
+  return fail(MUON_ERR_TIMEOUT, what + " gave up on a bounded wait (device code " + std::to_string(s) + ")");
+}
+
 int check_status(Ctx& c) {
   const int s = *(volatile int*)c.status_h;
   if (s != 0) {
     *(volatile int*)c.status_h = 0;
-    return fail(MUON_ERR_TIMEOUT, "an earlier launch on this stream gave up on a bounded wait (device code " +
-                                      std::to_string(s) + ")");
+    return status_error(s, "an earlier launch on this stream");
   }
   return MUON_OK;
 }
@@ -940,6 +970,11 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
   bool chain = io.ns_steps >= 1 && g_chain_clusters[c.dev] > 0 && !(g_debug_flags & 4);
   for (const auto& cd : g.classes) chain = chain && cd.kp <= kChainMaxK;
   chain = chain && chain_items(g, io.ns_steps) <= kChainMaxItems;   // lists of bounded size and build time
+
+  if (guard_bands()) {
+    for (size_t off : g.guards) CUDA_TRY(cudaMemsetAsync(base + off, kGuardByte, kGuardBytes, c.stream));
+    c.guards = g.guards;
+  }
 
   // 1. prologue
   {
@@ -1052,6 +1087,10 @@ int run_group(Ctx& c, Plan& plan, size_t gidx, const StepIO& io) {
         if (mode == kModePoly) ga->cls[ci].kblocks = cls[ci].kp / kBK;
       }
       ga->total_tiles = sym ? g.sym_tiles : g.upd_tiles;
+#ifdef MUON_DEBUG_BOUNDS
+      // injection (debug bit 5): one tile index past the end for every cluster
+      if (g_debug_flags & 32) { ga->total_tiles += std::max(1, c.sm_count / 2); g_debug_flags &= ~32; }
+#endif
       ga->mode = mode;
       ga->x_in = it & 1;
       ga->first = it == 0;
@@ -1435,6 +1474,22 @@ int muon_step_host(float* const* params, const float* const* grads, float* const
   return check_status(*c);
 }
 
+int muon_guard_check(void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!guard_bands()) return fail(MUON_ERR_UNSUPPORTED, "guard bands are off (MUON_GUARD_BANDS=1 when loading)");
+  Ctx* c = nullptr;
+  int rc = get_ctx(stream, &c);
+  if (rc) return rc;
+  CUDA_TRY(cudaStreamSynchronize(c->stream));
+  std::vector<unsigned char> h(kGuardBytes);
+  long long changed = 0;
+  for (size_t off : c->guards) {
+    CUDA_TRY(cudaMemcpy(h.data(), (char*)c->ws + off, kGuardBytes, cudaMemcpyDeviceToHost));
+    for (unsigned char v : h) changed += v != kGuardByte;
+  }
+  return (int)std::min<long long>(changed, 0x7fffffff);
+}
+
 size_t muon_workspace_size(const int64_t* shapes, int n) {
   if (!shapes || n <= 0) return 0;
   for (int i = 0; i < 2 * n; ++i)
@@ -1736,8 +1791,7 @@ extern "C" int muon_step_noalloc(float* const* params, const float* const* grads
   if (prev != 0) {
     CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), (cudaStream_t)stream));
     CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
-    return fail(MUON_ERR_TIMEOUT, "an earlier muon_step_noalloc call gave up on a bounded wait (device code " +
-                                      std::to_string(prev) + "); nothing was launched by this call");
+    return status_error(prev, "an earlier muon_step_noalloc call (nothing was launched by this one)");
   }
   if (!plan.small.empty() && (rc = run_small(nullptr, (cudaStream_t)stream, plan.small, io, status))) return rc;
   if (!plan.pair.empty() && (rc = run_pair(nullptr, (cudaStream_t)stream, plan.pair, io, status))) return rc;

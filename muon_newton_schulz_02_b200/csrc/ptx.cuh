@@ -25,6 +25,7 @@ enum DeviceError : int {
   kDevTimeoutEpi = 4,       // waited too long for an epilogue input tile
   kDevTimeoutDrain = 5,     // waited too long for in-flight copies at exit
   kDevTimeoutDep = 6,       // waited too long for another tile's results (chained launch)
+  kDevBounds = 7,           // a tile outside its class, matrix or grid (bounds-checking build only)
 };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {

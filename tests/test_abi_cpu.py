@@ -27,6 +27,21 @@ def test_exports_every_declared_function(L):
         assert hasattr(L, f), f
 
 
+def test_bounds_checking_build_exports_the_same_functions():
+    # the twin library with device bounds checks (MUON_DEBUG_BOUNDS) loads on a
+    # host without a GPU and exports every declared function too
+    D = ctypes.CDLL(muon.DEBUG_LIB_PATH)
+    for f in muon.header_functions():
+        assert hasattr(D, f), f
+    assert "muon_guard_check" in muon.header_functions()
+
+
+def test_guard_check_is_refused_without_guard_bands(L):
+    # guard bands are chosen at load time (MUON_GUARD_BANDS=1); without them the
+    # hook refuses before touching any device
+    assert L.muon_guard_check(None) == -7                # MUON_ERR_UNSUPPORTED
+
+
 def _arr(n, v=1):
     return (ctypes.c_void_p * n)(*[ctypes.c_void_p(v)] * n)
 
