@@ -27,10 +27,10 @@ __all__ = [
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libmuon_b200.so")
 # the same library with device bounds checks compiled in (tests and debugging):
-# set LIB_PATH to it before the first call
+# MUON_BOUNDS_CHECKS=1 in the environment, or LIB_PATH set to it before the first call
 DEBUG_LIB_PATH = os.path.join(HERE, "libmuon_b200_debug.so")
+LIB_PATH = DEBUG_LIB_PATH if os.environ.get("MUON_BOUNDS_CHECKS") == "1" else os.path.join(HERE, "libmuon_b200.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "muon.h")
 
 NS_A, NS_B, NS_C, NS_STEPS, NS_EPS = 3.4445, -4.7750, 2.0315, 5, 1e-7

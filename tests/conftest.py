@@ -28,3 +28,18 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _guard_bands_intact(request):
+    """With MUON_GUARD_BANDS=1 (the library lays out guard bands after every
+    workspace region), every GPU test ends by checking that no launch wrote
+    into them."""
+    yield
+    if os.environ.get("MUON_GUARD_BANDS") != "1" or "gpu" not in request.keywords or not _has_cuda():
+        return
+    import muon_newton_schulz_02_b200 as muon
+    if muon._lib is None:
+        return
+    changed = muon.guard_check()
+    assert changed == 0, f"{changed} guard-band bytes were overwritten"
