@@ -122,6 +122,37 @@ def test_workspace_size_matches_layout(L, shapes):
     assert _ws(shapes) == _expect_ws(shapes)
 
 
+def test_guard_bands_add_one_band_after_every_region():
+    # MUON_GUARD_BANDS=1 (read when the library loads, so in a child process):
+    # 4 KiB after the counter region and after each of the four buffers per shape
+    # class, the norm partials, the scales and the completion counters
+    import json
+    import os
+    import subprocess
+    import sys
+    sets = [[(768, 768)] * 4 + [(768, 3072), (3072, 768)], [(1, 1), (127, 129), (129, 127), (1000, 300)]]
+    code = f"""
+import ctypes, json, sys
+sys.path.insert(0, {muon.HERE + '/..'!r})
+import muon_newton_schulz_02_b200 as muon
+out = []
+for shapes in {sets!r}:
+    flat = [v for s in shapes for v in s]
+    out.append(muon.lib().muon_workspace_size((ctypes.c_int64 * len(flat))(*flat), len(shapes)))
+print(json.dumps(out))
+"""
+    env = dict(os.environ, MUON_GUARD_BANDS="1")
+    res = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=120)
+    assert res.returncode == 0, res.stderr[-2000:]
+    got = json.loads(res.stdout.strip().splitlines()[-1])
+    up = lambda v, a: (v + a - 1) // a * a
+    for shapes, ws in zip(sets, got):
+        classes = {(up(min(r, c), 128), up(max(r, c), 128)) for r, c in shapes
+                   if not ((min(r, c) <= 128 and up(max(r, c), 64) <= 512) or (min(r, c) <= 256 and max(r, c) <= 256))}
+        bands = 1 + 4 * len(classes) + 3
+        assert ws == _expect_ws(shapes) + bands * 4096, (shapes, ws)
+
+
 def test_workspace_size_rejects_bad_input(L):
     assert _ws([(0, 4)]) == 0
     assert muon.lib().muon_workspace_size(None, 1) == 0
