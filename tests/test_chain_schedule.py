@@ -61,6 +61,20 @@ def test_lists_cover_every_tile_once_and_cannot_deadlock(name, ns_steps, ncluste
         assert key not in seen, f"tile {key} listed twice"
         seen[key] = need
     assert seen == expect
+    # one (class, index in class) per matrix and one matrix per (class, index), the
+    # classes holding one padded shape each, indices 0.. without gaps: what the
+    # bounds-checking build verifies on the device for every item
+    slot = {}
+    for need, m, cls, b, tm, tn, mode, it in items:
+        assert slot.setdefault(m, (cls, b)) == (cls, b), f"matrix {m} under two classes or indices"
+    assert len(set(slot.values())) == len(slot)
+    by_cls = {}
+    for m, (cls, b) in slot.items():
+        r, c = shapes[m]
+        by_cls.setdefault(cls, {})[b] = (math.ceil(min(r, c) / 128), math.ceil(max(r, c) / 128))
+    for cls, members in by_cls.items():
+        assert sorted(members) == list(range(len(members))), f"class {cls} indices {sorted(members)}"
+        assert len(set(members.values())) == 1, f"class {cls} mixes padded shapes"
     # every cluster runs its list in order; run ready heads until nothing moves
     heads = [off[c] for c in range(nclusters)]
     done = {}
